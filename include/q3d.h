@@ -1,0 +1,160 @@
+/*
+ * q3d.h -- C ABI of the B200 (sm_100a) Conv3D implicit-GEMM library with
+ * fused NVFP4 activation fake-quantisation.
+ *
+ * The operations follow the Model-Optimizer "Conv3D Implicit GEMM CUDA kernel"
+ * article (lpqz.cn/news/178135):
+ *   - conv3d_implicit_gemm*: sec. 5.1 (convolution as a GEMM with
+ *     M = N*OD*OH*OW, Ngemm = Cout, K = Cin*kD*kH*kW, rows decomposed as
+ *     (n, od, oh, ow), columns as (c, kd, kh, kw), no materialised im2col),
+ *     sec. 3 (FP32/FP16/BF16 in and out, BF16 tensor-core arithmetic with
+ *     FP32 accumulation) and sec. 7.1 (arguments, asymmetric padding, output
+ *     shape of torch.nn.functional.conv3d, groups == 1);
+ *   - fused activation quantisation: sec. 6.1-6.3 (E2M1 values, E4M3 block
+ *     scales, blocks of 16 consecutive K elements of one A row, global scale
+ *     act_amax / (6*448), tiny-scale fallback 1.0), rounding to nearest even;
+ *   - fp4_fake_quant: sec. 6.4 and 7.3 (the same quantiser on a flat tensor
+ *     viewed as [numel/16, 16]).
+ *
+ * Conventions for every call:
+ *   - All tensor data pointers are DEVICE pointers to contiguous row-major
+ *     storage on the current CUDA device.  The caller owns every buffer; the
+ *     library never retains or frees a caller pointer.
+ *   - Calls enqueue work on `stream` (NULL = legacy default stream) and
+ *     return without synchronising.  Arguments are validated on the host
+ *     before anything is enqueued; on any non-OK status nothing has been
+ *     enqueued, except for Q3D_ERR_CUDA from a failed launch.
+ *   - Every device-side wait of the library is bounded; a wait that gives
+ *     up sets a device error word, which q3d_check_device_error() reports as
+ *     Q3D_ERR_DEVICE_TIMEOUT (the output is then unspecified).
+ *   - Errors are returned as q3d_status; q3d_last_error() gives a message
+ *     for the last non-OK status on the calling host thread.
+ *   - Requires a compute-capability 10.x device (B200); otherwise
+ *     Q3D_ERR_ARCH.
+ */
+#ifndef Q3D_H_
+#define Q3D_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define Q3D_API __attribute__((visibility("default")))
+#else
+#define Q3D_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* q3d_stream_t;
+
+typedef enum {
+  Q3D_F32 = 0,
+  Q3D_F16 = 1,
+  Q3D_BF16 = 2
+} q3d_dtype;
+
+/* A contiguous tensor: `ndim` leading entries of `shape` are used. */
+typedef struct {
+  void* data;       /* device pointer */
+  int32_t dtype;    /* q3d_dtype */
+  int32_t ndim;
+  int64_t shape[5];
+} q3d_tensor;
+
+typedef enum {
+  Q3D_OK = 0,
+  Q3D_ERR_NULLPTR = 1,            /* a required pointer is NULL */
+  Q3D_ERR_INVALID_ARG = 2,        /* rank, shape, groups != 1, stride/dilation < 1, pad < 0,
+                                     empty output extent, aliasing, numel % 16 != 0 */
+  Q3D_ERR_UNSUPPORTED_DTYPE = 3,  /* dtype not F32/F16/BF16, or w/bias/out dtype != x dtype */
+  Q3D_ERR_ARCH = 4,               /* current device is not compute capability 10.x */
+  Q3D_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  Q3D_ERR_DEVICE_TIMEOUT = 6,     /* a bounded device wait gave up (see q3d_check_device_error) */
+  Q3D_ERR_UNSUPPORTED_SHAPE = 7   /* valid convolution outside the library's limits (e.g. 32-bit index range) */
+} q3d_status;
+
+/*
+ * conv3d_implicit_gemm -- y = conv3d(x, w) + bias with symmetric padding,
+ * optionally fake-quantising the activation operand to NVFP4 on the fly.
+ *
+ *   x        [N, Cin, D, H, W], dtype F32/F16/BF16.
+ *   w        [Cout, Cin, kD, kH, kW], same dtype as x (groups == 1: the
+ *            Cin of w must equal the Cin of x).  Rounded to BF16 for the
+ *            tensor cores.
+ *   bias     [Cout] in x's dtype, or NULL.  Added in FP32 to the FP32
+ *            accumulator.
+ *   act_amax device pointer to one float: the tensor-wide max|x| that sets
+ *            the NVFP4 global scale; must be finite and >= 0.  Read on the
+ *            device (no host sync).  Required iff quant_act != 0.
+ *   stride, pad, dil  (d, h, w); stride >= 1, dil >= 1, pad >= 0.
+ *   quant_act  nonzero: every element of the implicit im2col matrix A is
+ *            fake-quantised (blocks of 16 consecutive K columns of one row, K
+ *            ordered (c, kd, kh, kw), zeros of the padding included) before
+ *            its BF16 rounding.
+ *   out      [N, Cout, OD, OH, OW] in x's dtype, preallocated, must not
+ *            overlap x or w.  OD = floor((D + 2*pad_d - dil_d*(kD-1) - 1) /
+ *            stride_d) + 1, likewise OH, OW.
+ * Returns Q3D_OK or an error status (see above).  N == 0 or Cout == 0 is a
+ * valid no-op.
+ */
+Q3D_API q3d_status conv3d_implicit_gemm(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                const float* act_amax, const int32_t stride[3], const int32_t pad[3],
+                                const int32_t dil[3], int32_t quant_act, q3d_tensor* out,
+                                q3d_stream_t stream);
+
+/*
+ * conv3d_implicit_gemm_pad2 -- as conv3d_implicit_gemm, with separate
+ * leading and trailing padding per dimension (d, h, w), e.g. causal temporal
+ * padding (2, 0).  The article applies such asymmetric (6-tuple) padding on
+ * the host before the kernel (sec. 7.1); here the padding is never
+ * materialised: out-of-range taps read as zero.
+ * OD = floor((D + pad_lo_d + pad_hi_d - dil_d*(kD-1) - 1) / stride_d) + 1.
+ */
+Q3D_API q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                     const float* act_amax, const int32_t stride[3],
+                                     const int32_t pad_lo[3], const int32_t pad_hi[3],
+                                     const int32_t dil[3], int32_t quant_act, q3d_tensor* out,
+                                     q3d_stream_t stream);
+
+/*
+ * fp4_fake_quant -- out = NVFP4 fake-quantisation of x (sec. 6.4, 7.3).
+ *   x     any rank 1..5, dtype F32/F16/BF16, numel % 16 == 0; consecutive
+ *         groups of 16 elements in memory order form the blocks.
+ *   amax  device pointer to one float (finite, >= 0): the global amax.
+ *   out   same shape and dtype as x; may be the same buffer as x (in place)
+ *         but must not partially overlap it.
+ * Each output is the binary32 result sign * E2M1(|v|/s) * s rounded (RNE) to
+ * the dtype; bit-exact with the CPU oracle.
+ */
+Q3D_API q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if
+ * none).  The pointer stays valid until the next call on this thread. */
+Q3D_API const char* q3d_last_error(void);
+
+/* Synchronise `stream`, then read and clear the device error word set by
+ * bounded waits that gave up.  Returns Q3D_OK, Q3D_ERR_DEVICE_TIMEOUT or
+ * Q3D_ERR_CUDA.  *site_bits (if not NULL) receives the bit mask of the
+ * waits that gave up. */
+Q3D_API q3d_status q3d_check_device_error(q3d_stream_t stream, uint32_t* site_bits);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+Q3D_API int32_t q3d_version(void);
+
+/*
+ * q3d_selftest_formats -- TEST HOOK, not part of the convolution path.
+ * Applies the device format conversions of the quantiser to n binary32
+ * inputs: e2m1[i] = E2M1 RNE-saturating value of in[i] (sign kept),
+ * e4m3[i] = E4M3 RNE-saturating value of |in[i]|.  All pointers are device
+ * pointers; enqueued on `stream`.
+ */
+Q3D_API q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* Q3D_H_ */

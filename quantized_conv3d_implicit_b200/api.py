@@ -1,0 +1,199 @@
+"""Python binding of libq3d.so (include/q3d.h): argument marshalling only.
+
+Every step of the computation runs in the library's sm_100a kernels.  If the
+library is missing or cannot be loaded, the calls raise RuntimeError; there is
+no CPU or PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence, Union
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libq3d.so")
+
+Q3D_F32, Q3D_F16, Q3D_BF16 = 0, 1, 2
+_DTYPES = {torch.float32: Q3D_F32, torch.float16: Q3D_F16, torch.bfloat16: Q3D_BF16}
+
+STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_ERR_UNSUPPORTED_DTYPE",
+          4: "Q3D_ERR_ARCH", 5: "Q3D_ERR_CUDA", 6: "Q3D_ERR_DEVICE_TIMEOUT", 7: "Q3D_ERR_UNSUPPORTED_SHAPE"}
+
+# names of the exported C entry points (checked against include/q3d.h by the tests)
+EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "fp4_fake_quant", "q3d_last_error",
+           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats")
+
+
+class Q3DTensor(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("ndim", ctypes.c_int32),
+                ("shape", ctypes.c_int64 * 5)]
+
+
+class Q3DError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: Optional[str] = None):
+    """Load libq3d.so (raises RuntimeError when it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"{p} is missing: build it with `python -m quantized_conv3d_implicit_b200.build` "
+                               "(there is no fallback implementation)")
+        lib = ctypes.CDLL(p)
+        T = ctypes.POINTER(Q3DTensor)
+        i32x3 = ctypes.POINTER(ctypes.c_int32)
+        vp = ctypes.c_void_p
+        lib.conv3d_implicit_gemm.restype = ctypes.c_int
+        lib.conv3d_implicit_gemm.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
+        lib.conv3d_implicit_gemm_pad2.restype = ctypes.c_int
+        lib.conv3d_implicit_gemm_pad2.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
+        lib.fp4_fake_quant.restype = ctypes.c_int
+        lib.fp4_fake_quant.argtypes = [T, vp, T, vp]
+        lib.q3d_last_error.restype = ctypes.c_char_p
+        lib.q3d_last_error.argtypes = []
+        lib.q3d_check_device_error.restype = ctypes.c_int
+        lib.q3d_check_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+        lib.q3d_version.restype = ctypes.c_int32
+        lib.q3d_selftest_formats.restype = ctypes.c_int
+        lib.q3d_selftest_formats.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def _tensor(t: Optional[torch.Tensor]) -> Optional[Q3DTensor]:
+    if t is None:
+        return None
+    if t.dtype not in _DTYPES:
+        raise Q3DError(3, f"unsupported dtype {t.dtype}")
+    if not t.is_contiguous():
+        raise Q3DError(2, "tensors must be contiguous")
+    s = Q3DTensor()
+    s.data = t.data_ptr() if t.numel() > 0 else None
+    s.dtype = _DTYPES[t.dtype]
+    s.ndim = t.dim()
+    for i, d in enumerate(t.shape):
+        s.shape[i] = d
+    return s
+
+
+def _ref(s):
+    return ctypes.byref(s) if s is not None else None
+
+
+def _triple(v: Union[int, Sequence[int]]) -> tuple:
+    if isinstance(v, int):
+        return (v, v, v)
+    v = tuple(int(t) for t in v)
+    if len(v) != 3:
+        raise ValueError("expected an int or a 3-tuple")
+    return v
+
+
+def _pads(padding) -> tuple:
+    """int, 3-tuple (symmetric) or 6-tuple (d_lo, d_hi, h_lo, h_hi, w_lo, w_hi)."""
+    if isinstance(padding, int):
+        return (padding,) * 3, (padding,) * 3
+    p = tuple(int(t) for t in padding)
+    if len(p) == 3:
+        return p, p
+    if len(p) == 6:
+        return (p[0], p[2], p[4]), (p[1], p[3], p[5])
+    raise ValueError("padding must be an int, a 3-tuple or a 6-tuple")
+
+
+def _stream_handle(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if stream.cuda_stream != 0 else None
+
+
+def _check(lib, status: int):
+    if status != 0:
+        msg = lib.q3d_last_error().decode(errors="replace")
+        raise Q3DError(status, msg)
+
+
+def out_shape(x_shape, w_shape, stride=1, padding=0, dilation=1):
+    s, d = _triple(stride), _triple(dilation)
+    lo, hi = _pads(padding)
+    dims = []
+    for i in range(3):
+        span = x_shape[2 + i] + lo[i] + hi[i] - d[i] * (w_shape[2 + i] - 1) - 1
+        dims.append(span // s[i] + 1 if span >= 0 else 0)
+    return (x_shape[0], w_shape[0], *dims)
+
+
+def conv3d_implicit_gemm(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                         stride=1, padding=0, dilation=1, act_amax: Optional[torch.Tensor] = None,
+                         quant_act: bool = False, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y = conv3d(x, w) + bias through libq3d (BF16 tensor cores, FP32
+    accumulation, result in x.dtype), optionally fake-quantising the
+    activation operand to NVFP4 (act_amax: float32 device tensor with one
+    element).  padding may be an int, a 3-tuple or a 6-tuple
+    (d_lo, d_hi, h_lo, h_hi, w_lo, w_hi)."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    if out is None:
+        out = torch.empty(out_shape(x.shape, w.shape, stride, padding, dilation), dtype=x.dtype, device=x.device)
+    if quant_act:
+        if act_amax is None:
+            raise ValueError("quant_act requires act_amax")
+        if act_amax.dtype != torch.float32 or act_amax.numel() != 1 or act_amax.device != x.device:
+            raise ValueError("act_amax must be a one-element float32 tensor on x's device")
+    arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    xs, ws, os_, bs = _tensor(x), _tensor(w), _tensor(out), _tensor(bias)
+    amax_ptr = act_amax.data_ptr() if (quant_act and act_amax is not None) else None
+    st = lib.conv3d_implicit_gemm_pad2(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
+                                       arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
+                                       _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
+def fp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """NVFP4 fake-quantisation (blocks of 16 consecutive elements) through libq3d."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty_like(x)
+    if amax.dtype != torch.float32 or amax.numel() != 1:
+        raise ValueError("amax must be a one-element float32 tensor")
+    xs, os_ = _tensor(x), _tensor(out)
+    st = lib.fp4_fake_quant(_ref(xs), amax.data_ptr(), _ref(os_), _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronise the stream and return the device error bits (0 = none);
+    raises Q3DError when a bounded device wait gave up."""
+    lib = load_library()
+    bits = ctypes.c_uint32(0)
+    st = lib.q3d_check_device_error(_stream_handle(stream), ctypes.byref(bits))
+    _check(lib, st)
+    return bits.value
+
+
+def selftest_formats(v: torch.Tensor, stream=None):
+    """Test hook: device E2M1 and E4M3 conversions of float32 values."""
+    lib = load_library()
+    assert v.dtype == torch.float32 and v.is_cuda and v.is_contiguous()
+    e2m1 = torch.empty_like(v)
+    e4m3 = torch.empty_like(v)
+    st = lib.q3d_selftest_formats(v.data_ptr(), v.numel(), e2m1.data_ptr(), e4m3.data_ptr(), _stream_handle(stream))
+    _check(lib, st)
+    return e2m1, e4m3

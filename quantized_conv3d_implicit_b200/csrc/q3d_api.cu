@@ -1,0 +1,297 @@
+// q3d_api.cu -- the C ABI declared in include/q3d.h: host-side argument
+// validation, output-extent arithmetic, dispatch, and the device error word.
+//
+// Argument rules follow the Model-Optimizer "Conv3D Implicit GEMM CUDA
+// kernel" article, sec. 7.1 and 7.3 (5-D tensors, the Cin of w equal to the
+// Cin of x since groups must be 1, numel divisible by the block size for the
+// standalone call, output dtype equal to the input dtype) and sec. 5.4 (the
+// device architecture is checked before dispatch; here compute capability
+// 10.x, the only target this library is built for).
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/q3d.h"
+#include "q3d_internal.h"
+
+namespace q3d {
+cudaError_t launch_conv3d_basic(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why);
+cudaError_t launch_conv3d_fast(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
+                               bool* handled);
+}  // namespace q3d
+
+namespace {
+
+thread_local std::string g_last_error;
+
+// One word per device; bounded waits that give up OR their site bit into it.
+__device__ unsigned int g_device_error_word;
+
+q3d_status fail(q3d_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+q3d_status fail(q3d_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+q3d_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(Q3D_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+struct DeviceInfo {
+  bool init = false;
+  int major = 0, minor = 0, sm_count = 0;
+  unsigned int* err_word = nullptr;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Resolve the current device, check its architecture, and fetch the device
+// address of its error word (once per device).
+q3d_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(Q3D_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    d.major = prop.major;
+    d.minor = prop.minor;
+    d.sm_count = prop.multiProcessorCount;
+    if (d.major == 10) {
+      void* p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_device_error_word);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
+      d.err_word = static_cast<unsigned int*>(p);
+    }
+    d.init = true;
+  }
+  if (d.major != 10)
+    return fail(Q3D_ERR_ARCH, "device %d has compute capability %d.%d; this library needs 10.x (sm_100a)", dev,
+                d.major, d.minor);
+  *out = &d;
+  return Q3D_OK;
+}
+
+bool dtype_ok(int32_t dt) { return dt == Q3D_F32 || dt == Q3D_F16 || dt == Q3D_BF16; }
+int64_t dtype_size(int32_t dt) { return dt == Q3D_F32 ? 4 : 2; }
+
+int64_t numel(const q3d_tensor* t) {
+  int64_t n = 1;
+  for (int i = 0; i < t->ndim; ++i) n *= t->shape[i];
+  return n;
+}
+
+bool overlaps(const q3d_tensor* a, const q3d_tensor* b) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a->data), b0 = reinterpret_cast<uintptr_t>(b->data);
+  const uintptr_t a1 = a0 + static_cast<uintptr_t>(numel(a) * dtype_size(a->dtype));
+  const uintptr_t b1 = b0 + static_cast<uintptr_t>(numel(b) * dtype_size(b->dtype));
+  return a0 < b1 && b0 < a1 && a1 > a0 && b1 > b0;
+}
+
+q3d_status check_tensor(const q3d_tensor* t, const char* name, int ndim) {
+  if (!t) return fail(Q3D_ERR_NULLPTR, "%s is NULL", name);
+  if (t->ndim != ndim) return fail(Q3D_ERR_INVALID_ARG, "%s must have rank %d (got %d)", name, ndim, t->ndim);
+  for (int i = 0; i < ndim; ++i)
+    if (t->shape[i] < 0) return fail(Q3D_ERR_INVALID_ARG, "%s.shape[%d] is negative", name, i);
+  if (!dtype_ok(t->dtype)) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "%s dtype %d is not F32/F16/BF16", name, t->dtype);
+  if (!t->data && numel(t) > 0) return fail(Q3D_ERR_NULLPTR, "%s.data is NULL", name);
+  return Q3D_OK;
+}
+
+}  // namespace
+
+namespace q3d {
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace q3d
+
+extern "C" {
+
+const char* q3d_last_error(void) { return g_last_error.c_str(); }
+
+int32_t q3d_version(void) { return 100; }
+
+q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                     const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
+                                     const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_act,
+                                     q3d_tensor* out, q3d_stream_t stream) {
+  q3d_status st;
+  if ((st = check_tensor(x, "x", 5)) != Q3D_OK) return st;
+  if ((st = check_tensor(w, "w", 5)) != Q3D_OK) return st;
+  if ((st = check_tensor(out, "out", 5)) != Q3D_OK) return st;
+  if (bias && (st = check_tensor(bias, "bias", 1)) != Q3D_OK) return st;
+  if (!stride || !pad_lo || !pad_hi || !dil) return fail(Q3D_ERR_NULLPTR, "stride/pad/dil array is NULL");
+  if (quant_act && !act_amax) return fail(Q3D_ERR_NULLPTR, "quant_act requires act_amax");
+  if (w->dtype != x->dtype || out->dtype != x->dtype || (bias && bias->dtype != x->dtype))
+    return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "w, bias and out must have the dtype of x");
+  for (int i = 0; i < 3; ++i) {
+    if (stride[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "stride[%d] = %d must be >= 1", i, stride[i]);
+    if (dil[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "dilation[%d] = %d must be >= 1", i, dil[i]);
+    if (pad_lo[i] < 0 || pad_hi[i] < 0) return fail(Q3D_ERR_INVALID_ARG, "padding[%d] must be >= 0", i);
+  }
+  const int64_t N = x->shape[0], C = x->shape[1], D = x->shape[2], H = x->shape[3], W = x->shape[4];
+  const int64_t Cout = w->shape[0], KD = w->shape[2], KH = w->shape[3], KW = w->shape[4];
+  if (w->shape[1] != C)
+    return fail(Q3D_ERR_INVALID_ARG, "w has %lld input channels but x has %lld (groups != 1 is not supported)",
+                (long long)w->shape[1], (long long)C);
+  if (C < 1 || KD < 1 || KH < 1 || KW < 1)
+    return fail(Q3D_ERR_INVALID_ARG, "Cin and kernel extents must be >= 1");
+  if (bias && bias->shape[0] != Cout) return fail(Q3D_ERR_INVALID_ARG, "bias must have shape [Cout]");
+  const int64_t in_dims[3] = {D, H, W}, k_dims[3] = {KD, KH, KW};
+  int64_t o_dims[3];
+  for (int i = 0; i < 3; ++i) {
+    const int64_t span = in_dims[i] + pad_lo[i] + pad_hi[i] - static_cast<int64_t>(dil[i]) * (k_dims[i] - 1) - 1;
+    if (span < 0)
+      return fail(Q3D_ERR_INVALID_ARG, "kernel extent exceeds the padded input along dim %d (empty output)", i);
+    o_dims[i] = span / stride[i] + 1;
+  }
+  if (out->shape[0] != N || out->shape[1] != Cout || out->shape[2] != o_dims[0] || out->shape[3] != o_dims[1] ||
+      out->shape[4] != o_dims[2])
+    return fail(Q3D_ERR_INVALID_ARG, "out must have shape [%lld, %lld, %lld, %lld, %lld]", (long long)N,
+                (long long)Cout, (long long)o_dims[0], (long long)o_dims[1], (long long)o_dims[2]);
+  if (N == 0 || Cout == 0) return Q3D_OK;  // empty batch or no output channels: nothing to compute
+  if (overlaps(out, x) || overlaps(out, w) || (bias && overlaps(out, bias)))
+    return fail(Q3D_ERR_INVALID_ARG, "out overlaps an input tensor");
+  const int64_t K = C * KD * KH * KW;
+  const int64_t M = N * o_dims[0] * o_dims[1] * o_dims[2];
+  if (K > 0x7FFFFFFFll / 2 || Cout > 0x7FFFFFFFll || numel(x) > 0x7FFFFFFFll || numel(out) > (1ll << 40) ||
+      C * D * H * W > 0x7FFFFFFFll)
+    return fail(Q3D_ERR_UNSUPPORTED_SHAPE, "problem exceeds the 32-bit per-sample index range of the kernels");
+
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  q3d::ConvGeom g;
+  g.N = (int32_t)N; g.C = (int32_t)C; g.D = (int32_t)D; g.H = (int32_t)H; g.W = (int32_t)W;
+  g.Cout = (int32_t)Cout; g.KD = (int32_t)KD; g.KH = (int32_t)KH; g.KW = (int32_t)KW;
+  g.sd = stride[0]; g.sh = stride[1]; g.sw = stride[2];
+  g.pd = pad_lo[0]; g.ph = pad_lo[1]; g.pw = pad_lo[2];
+  g.dd = dil[0]; g.dh = dil[1]; g.dw = dil[2];
+  g.OD = (int32_t)o_dims[0]; g.OH = (int32_t)o_dims[1]; g.OW = (int32_t)o_dims[2];
+  g.M = M; g.K = (int32_t)K; g.taps = (int32_t)(KD * KH * KW);
+
+  q3d::ConvLaunch L;
+  L.x = x->data; L.bias = bias ? bias->data : nullptr; L.y = out->data;
+  L.act_amax = quant_act ? act_amax : nullptr;
+  L.dtype = x->dtype; L.quant = quant_act ? 1 : 0; L.err = dev->err_word; L.sm_count = dev->sm_count;
+
+  // B operand: BF16 [Cout, ld] with a 16-byte row pitch.  BF16 weights with
+  // K % 8 == 0 and a 16-byte aligned base are used in place; otherwise a
+  // stream-ordered scratch copy is made.
+  void* scratch = nullptr;
+  cudaError_t e;
+  if (x->dtype == Q3D_BF16 && K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {
+    L.w_bf16 = w->data;
+    L.w_ld = K;
+  } else {
+    const int64_t ld = (K + 7) / 8 * 8;
+    e = cudaMallocAsync(&scratch, static_cast<size_t>(Cout * ld * 2), s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(weight staging)");
+    e = q3d::launch_stage_weights(w->data, x->dtype, (int32_t)Cout, (int32_t)K, ld, scratch, s);
+    if (e != cudaSuccess) { cudaFreeAsync(scratch, s); return cuda_fail(e, "weight staging launch"); }
+    L.w_bf16 = scratch;
+    L.w_ld = ld;
+  }
+
+  const char* why = nullptr;
+  bool handled = false;
+  e = q3d::launch_conv3d_fast(g, L, s, &why, &handled);
+  if (e == cudaSuccess && !handled) e = q3d::launch_conv3d_basic(g, L, s, &why);
+  if (scratch) cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) {
+    if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
+    return cuda_fail(e, "conv3d launch");
+  }
+  return Q3D_OK;
+}
+
+q3d_status conv3d_implicit_gemm(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                const float* act_amax, const int32_t stride[3], const int32_t pad[3],
+                                const int32_t dil[3], int32_t quant_act, q3d_tensor* out, q3d_stream_t stream) {
+  if (!pad) return fail(Q3D_ERR_NULLPTR, "pad is NULL");
+  return conv3d_implicit_gemm_pad2(x, w, bias, act_amax, stride, pad, pad, dil, quant_act, out, stream);
+}
+
+q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream) {
+  if (!x || !out) return fail(Q3D_ERR_NULLPTR, "x or out is NULL");
+  if (!amax) return fail(Q3D_ERR_NULLPTR, "amax is NULL");
+  if (x->ndim < 1 || x->ndim > 5) return fail(Q3D_ERR_INVALID_ARG, "x must have rank 1..5");
+  q3d_status st;
+  if ((st = check_tensor(x, "x", x->ndim)) != Q3D_OK) return st;
+  if ((st = check_tensor(out, "out", x->ndim)) != Q3D_OK) return st;
+  if (out->dtype != x->dtype) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "out must have the dtype of x");
+  for (int i = 0; i < x->ndim; ++i)
+    if (out->shape[i] != x->shape[i]) return fail(Q3D_ERR_INVALID_ARG, "out must have the shape of x");
+  const int64_t n = numel(x);
+  if (n % 16 != 0) return fail(Q3D_ERR_INVALID_ARG, "numel (%lld) must be a multiple of 16", (long long)n);
+  if (n == 0) return Q3D_OK;
+  if (out->data != x->data && overlaps(out, x))
+    return fail(Q3D_ERR_INVALID_ARG, "out partially overlaps x");
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaError_t e = q3d::launch_fp4_fake_quant(x->data, out->data, x->dtype, n, amax,
+                                             reinterpret_cast<cudaStream_t>(stream), dev->sm_count);
+  if (e != cudaSuccess) return cuda_fail(e, "fp4_fake_quant launch");
+  return Q3D_OK;
+}
+
+q3d_status q3d_check_device_error(q3d_stream_t stream, uint32_t* site_bits) {
+  DeviceInfo* dev = nullptr;
+  q3d_status st;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int v = 0;
+  e = cudaMemcpy(&v, dev->err_word, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (site_bits) *site_bits = v;
+  if (v) {
+    const unsigned int zero = 0;
+    e = cudaMemcpy(dev->err_word, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "clear device error word");
+    return fail(Q3D_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up (site bits 0x%x)", v);
+  }
+  return Q3D_OK;
+}
+
+q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream) {
+  if (!in || !e2m1 || !e4m3) return fail(Q3D_ERR_NULLPTR, "NULL pointer");
+  if (n < 0) return fail(Q3D_ERR_INVALID_ARG, "n < 0");
+  DeviceInfo* dev = nullptr;
+  q3d_status st;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaError_t e = q3d::launch_selftest_formats(in, n, e2m1, e4m3, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return Q3D_OK;
+}
+
+}  // extern "C"

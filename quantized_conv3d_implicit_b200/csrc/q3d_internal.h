@@ -1,0 +1,70 @@
+// q3d_internal.h -- declarations shared between the C-ABI layer and the
+// kernel translation units (not installed, not part of the ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace q3d {
+
+// Site bits recorded in the device error word when a bounded wait gives up.
+enum WaitSite : unsigned int {
+  kSiteProducerEmpty = 1u << 0,   // producer waiting for a free pipeline stage
+  kSiteTmaFull = 1u << 1,         // consumer waiting for a TMA stage to land
+  kSiteAStageFull = 1u << 2,      // MMA issuer waiting for the transformed A stage
+  kSiteMmaDone = 1u << 3,         // waiting for tensor-core completion of a stage
+  kSiteAccFull = 1u << 4,         // epilogue waiting for an accumulator
+  kSiteAccEmpty = 1u << 5,        // MMA issuer waiting for the epilogue to drain TMEM
+  kSiteHaloFull = 1u << 6,        // transform waiting for an input halo slot
+  kSiteHaloEmpty = 1u << 7,       // producer waiting for a free halo slot
+  kSiteDrain = 1u << 8,           // final drain of in-flight copies after an abort
+};
+
+// Geometry of one convolution, all in elements.  pd/ph/pw are the leading
+// (low-side) paddings; the trailing ones only enter through OD/OH/OW.
+struct ConvGeom {
+  int32_t N, C, D, H, W;
+  int32_t Cout, KD, KH, KW;
+  int32_t sd, sh, sw;
+  int32_t pd, ph, pw;
+  int32_t dd, dh, dw;
+  int32_t OD, OH, OW;
+  int64_t M;      // N*OD*OH*OW
+  int32_t K;      // C*KD*KH*KW
+  int32_t taps;   // KD*KH*KW
+};
+
+struct ConvLaunch {
+  const void* x;            // [N, C, D, H, W] in dtype
+  const void* bias;         // [Cout] in dtype or nullptr
+  void* y;                  // [N, Cout, OD, OH, OW] in dtype
+  const float* act_amax;    // device scalar or nullptr
+  const void* w_bf16;       // [Cout, w_ld] bf16, K-major (w_ld >= K, w_ld % 8 == 0)
+  int64_t w_ld;             // row pitch of w_bf16 in elements
+  int dtype;                // 0 f32, 1 f16, 2 bf16
+  int quant;
+  unsigned int* err;        // device error word
+  int sm_count;
+};
+
+// Driver entry point for cuTensorMapEncodeTiled (resolved once through the
+// runtime, so the library does not link libcuda directly).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+
+cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, const float* amax,
+                                  cudaStream_t s, int sm_count);
+cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, cudaStream_t s);
+
+// Convert w [Cout, K] (dtype) to bf16 [Cout, ld] with zero columns K..ld-1.
+cudaError_t launch_stage_weights(const void* w, int dtype, int32_t Cout, int32_t K, int64_t ld, void* w_bf16,
+                                 cudaStream_t s);
+
+// The implicit-GEMM convolution; returns a CUDA error or cudaSuccess, and a
+// short reason in *why when it rejects the problem before launching.
+cudaError_t launch_conv3d_igemm(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why);
+
+}  // namespace q3d

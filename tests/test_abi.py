@@ -1,0 +1,128 @@
+"""The C ABI: the library loads without a GPU, exports every entry point the
+header declares, and validates arguments on the host (before any CUDA call),
+so these run on a CPU-only machine with placeholder device pointers that are
+never dereferenced."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from quantized_conv3d_implicit_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "q3d.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load_library()
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"Q3D_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    assert _declared() == sorted(api.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert lib.q3d_version() == 100
+
+
+FAKE = 0x10000
+
+
+def T(shape, dtype=2, data=FAKE):
+    t = api.Q3DTensor()
+    t.data = data
+    t.dtype = dtype
+    t.ndim = len(shape)
+    for i, d in enumerate(shape):
+        t.shape[i] = d
+    return t
+
+
+def conv(lib, x, w, out, bias=None, amax=None, stride=(1, 1, 1), plo=(1, 1, 1), phi=(1, 1, 1), dil=(1, 1, 1),
+         quant=0):
+    arr = lambda v: (ctypes.c_int32 * 3)(*v)  # noqa: E731
+    r = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731
+    return lib.conv3d_implicit_gemm_pad2(r(x), r(w), r(bias), amax, arr(stride), arr(plo), arr(phi), arr(dil),
+                                         quant, r(out), None)
+
+
+GOOD = dict(x=((1, 4, 3, 8, 8),), w=((5, 4, 3, 3, 3),), out=((1, 5, 3, 8, 8),))
+
+
+def good(dtype=2):
+    return (T((1, 4, 3, 8, 8), dtype, FAKE), T((5, 4, 3, 3, 3), dtype, FAKE * 16),
+            T((1, 5, 3, 8, 8), dtype, FAKE * 256))
+
+
+def test_null_pointers(lib):
+    x, w, out = good()
+    assert conv(lib, None, w, out) == 1
+    assert conv(lib, x, None, out) == 1
+    assert conv(lib, x, w, None) == 1
+    assert conv(lib, x, w, out, quant=1) == 1           # quant without act_amax
+    assert b"act_amax" in lib.q3d_last_error()
+    assert conv(lib, T((1, 4, 3, 8, 8), 2, 0), w, out) == 1
+
+
+def test_invalid_shapes(lib):
+    x, w, out = good()
+    assert conv(lib, T((4, 3, 8, 8)), w, out) == 2                    # rank
+    assert conv(lib, x, T((5, 3, 3, 3, 3), 2, FAKE * 16), out) == 2   # groups != 1
+    assert b"groups" in lib.q3d_last_error()
+    assert conv(lib, x, w, T((1, 5, 3, 8, 9), 2, FAKE * 256)) == 2    # wrong out shape
+    assert conv(lib, x, w, out, stride=(0, 1, 1)) == 2
+    assert conv(lib, x, w, out, dil=(1, 0, 1)) == 2
+    assert conv(lib, x, w, out, plo=(-1, 1, 1)) == 2
+    big = T((5, 4, 9, 3, 3), 2, FAKE * 16)                            # kernel larger than padded input
+    assert conv(lib, x, big, out) == 2
+    assert conv(lib, x, w, out, bias=T((4,), 2, FAKE * 4096)) == 2    # bias length != Cout
+    alias = T((1, 5, 3, 8, 8), 2, FAKE)                               # out overlaps x
+    assert conv(lib, x, w, alias) == 2
+
+
+def test_dtype_rules(lib):
+    x, w, out = good()
+    assert conv(lib, x, T((5, 4, 3, 3, 3), 1, FAKE * 16), out) == 3
+    assert conv(lib, x, w, T((1, 5, 3, 8, 8), 0, FAKE * 256)) == 3
+    assert conv(lib, T((1, 4, 3, 8, 8), 7), w, out) == 3
+
+
+def test_empty_batch_is_noop(lib):
+    x = T((0, 4, 3, 8, 8))
+    w = T((5, 4, 3, 3, 3), 2, FAKE * 16)
+    out = T((0, 5, 3, 8, 8), 2, FAKE * 256)
+    assert conv(lib, x, w, out) == 0
+
+
+def test_fake_quant_validation(lib):
+    r = ctypes.byref
+    x = T((3, 7), 2, FAKE)
+    out = T((3, 7), 2, FAKE * 256)
+    assert lib.fp4_fake_quant(r(x), FAKE * 4096, r(out), None) == 2          # 21 % 16 != 0
+    assert lib.fp4_fake_quant(r(T((2, 16))), None, r(T((2, 16), 2, FAKE * 256)), None) == 1
+    assert lib.fp4_fake_quant(r(T((2, 16))), FAKE * 4096, r(T((2, 16), 1, FAKE * 256)), None) == 3
+    assert lib.fp4_fake_quant(r(T((2, 16))), FAKE * 4096, r(T((16, 2), 2, FAKE * 256)), None) == 2
+    assert lib.fp4_fake_quant(r(T((0, 16))), FAKE * 4096, r(T((0, 16), 2, FAKE * 256)), None) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    x, w, out = good()
+    assert conv(lib, x, w, out) in (4, 5)
+    assert lib.q3d_last_error() != b""
+
+
+def test_python_binding_errors_without_library(tmp_path):
+    with pytest.raises(RuntimeError):
+        api.load_library(str(tmp_path / "missing.so"))

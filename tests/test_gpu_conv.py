@@ -1,0 +1,138 @@
+"""GPU parity of the implicit-GEMM Conv3D against the CPU oracle.
+
+Small shapes are compared element by element on the whole output; the
+full-size layer configurations are compared on a seeded sample of output
+rows (every Cout) plus the first and last rows and the rows at the padding
+faces.  Tolerance: max|y - y_ref| <= 2e-3 max|y_ref| and per-element
+relative error <= 1e-2 where |y_ref| > 1e-2 max|y_ref|.  The identity-weight
+readout checks the fused quantiser and the im2col addressing bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_conv3d_implicit_b200 import api, workloads
+from _parity import assert_conv_close, bits, to_np_f32
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(inp, stride, plo, phi, dil, quant):
+    x, w, b, amax = inp["x"], inp["w"], inp["bias"], inp["act_amax"]
+    pad6 = (plo[0], phi[0], plo[1], phi[1], plo[2], phi[2])
+    y = api.conv3d_implicit_gemm(x, w, b, stride=stride, padding=pad6, dilation=dil,
+                                 act_amax=amax if quant else None, quant_act=quant)
+    assert api.check_device_error() == 0
+    return y
+
+
+def _ref(inp, stride, plo, phi, dil, quant, m_list=None):
+    x, w, b, amax = inp["x"], inp["w"], inp["bias"], inp["act_amax"]
+    return oracle.conv3d(to_np_f32(x), to_np_f32(w), None if b is None else to_np_f32(b), stride, plo, phi, dil,
+                         quant_act=quant, act_amax=float(amax.item()), m_list=m_list)
+
+
+# x_shape, cout, kernel, stride, pad_lo, pad_hi, dil
+SHAPES = [
+    ((1, 16, 4, 16, 16), 16, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),   # tiny layer
+    ((1, 8, 3, 10, 12), 24, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1)),    # causal pad, K=216 (tail)
+    ((2, 5, 5, 9, 11), 20, (3, 3, 3), (1, 2, 2), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # stride, K=135, Cout%16
+    ((1, 6, 6, 13, 14), 33, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 2, 2)),    # dilation
+    ((1, 32, 3, 8, 8), 300, (1, 1, 1), (1, 1, 1), (0, 0, 0), (0, 0, 0), (1, 1, 1)),    # pointwise, 2 N tiles
+    ((1, 7, 4, 9, 9), 19, (1, 3, 3), (1, 1, 1), (0, 1, 1), (0, 1, 1), (1, 1, 1)),      # 1x3x3, K=63
+    ((1, 3, 7, 9, 10), 8, (5, 5, 5), (1, 1, 1), (2, 2, 2), (2, 2, 2), (1, 1, 1)),      # 5x5x5, K=375
+    ((1, 4, 5, 8, 8), 16, (3, 3, 3), (2, 3, 1), (0, 1, 2), (1, 0, 0), (2, 1, 3)),      # mixed everything
+    ((1, 7, 3, 3, 3), 5, (3, 3, 3), (1, 1, 1), (0, 0, 0), (0, 0, 0), (1, 1, 1)),       # 1x1x1 output, K=189
+    ((3, 16, 2, 5, 7), 40, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # batch 3, M=210
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("quant", [False, True])
+@pytest.mark.parametrize("case", range(len(SHAPES)))
+def test_conv_small_shapes(cuda_ok, case, quant, dtype):
+    xs, cout, k, s, plo, phi, d = SHAPES[case]
+    inp = workloads.random_conv_inputs(100 + case, xs, cout, k, dtype=dtype, bias=(case % 2 == 0), device="cuda")
+    y = _run(inp, s, plo, phi, d, quant)
+    ref = _ref(inp, s, plo, phi, d, quant)
+    assert_conv_close(to_np_f32(y), ref, f"case {case} quant={quant} {dtype}", dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("quant", [False, True])
+def test_identity_weight_readout_is_bit_exact(cuda_ok, quant, dtype):
+    # one-hot weights: y[:, co] = A[:, k(co)], a single nonzero product per
+    # output, so the FP32 accumulator holds the BF16 operand exactly and the
+    # whole im2col row (quantised or not) is reproduced bit for bit
+    xs, k = (1, 5, 4, 9, 11), (3, 3, 3)
+    K = 5 * 27
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(xs, generator=g) * 3).to(dtype)
+    amax = x.float().abs().max().reshape(1)
+    for start in range(0, K, 128):
+        cols = list(range(start, min(K, start + 128)))
+        w = torch.zeros((len(cols), K), dtype=torch.float32)
+        w[torch.arange(len(cols)), torch.tensor(cols)] = 1.0
+        w = w.reshape(len(cols), 5, 3, 3, 3).to(dtype)
+        inp = dict(x=x.cuda(), w=w.cuda(), bias=None, act_amax=amax.cuda())
+        y = _run(inp, (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1), quant)
+        ref = oracle.conv3d(x.float().numpy(), w.float().numpy(), None, (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1),
+                            quant_act=quant, act_amax=float(amax.item()))
+        ref_bits = oracle.round_to_dtype_bits(ref.astype(np.float32), {torch.float32: "float32",
+                                                                        torch.float16: "float16",
+                                                                        torch.bfloat16: "bfloat16"}[dtype])
+        assert np.array_equal(bits(y), ref_bits), start
+
+
+def test_determinism(cuda_ok):
+    inp = workloads.random_conv_inputs(5, (1, 24, 4, 20, 24), 48, (3, 3, 3), dtype=torch.bfloat16, device="cuda")
+    y1 = _run(inp, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), True)
+    y2 = _run(inp, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), True)
+    assert torch.equal(y1, y2)
+
+
+def test_symmetric_entry_point_and_noop(cuda_ok):
+    inp = workloads.random_conv_inputs(6, (1, 4, 3, 6, 6), 8, (3, 3, 3), dtype=torch.bfloat16, device="cuda")
+    y = api.conv3d_implicit_gemm(inp["x"], inp["w"], inp["bias"], stride=1, padding=1, dilation=1)
+    ref = _ref(inp, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), False)
+    assert_conv_close(to_np_f32(y), ref, "symmetric", torch.bfloat16)
+    e = api.conv3d_implicit_gemm(inp["x"][:0], inp["w"], padding=1)
+    assert e.shape[0] == 0
+
+
+def _sample_rows(wl, rng, n_random):
+    od, oh, ow = wl.out_spatial()
+    M = wl.m_gemm
+    picks = set(rng.integers(0, M, n_random).tolist())
+    picks.update([0, M - 1])
+    # rows at the faces of the output volume (padding taps)
+    for n in range(wl.x_shape[0]):
+        for d in (0, od - 1):
+            for h in (0, oh // 2, oh - 1):
+                for w_ in (0, 1, ow // 2, ow - 2, ow - 1):
+                    picks.add(((n * od + d) * oh + h) * ow + max(0, w_))
+    return np.array(sorted(p for p in picks if 0 <= p < M), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", [n for n in workloads.WORKLOADS if n != workloads.SMALL])
+def test_full_size_layers_sampled(cuda_ok, name):
+    wl = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(wl, device="cuda")
+    y = _run(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act)
+    rng = np.random.default_rng(11)
+    ms = _sample_rows(wl, rng, 384)
+    ref = _ref(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act, m_list=ms)
+    # gather the same rows from the GPU output [N, Cout, OD, OH, OW]
+    N, Co = y.shape[0], y.shape[1]
+    yf = y.permute(0, 2, 3, 4, 1).reshape(-1, Co)
+    got = to_np_f32(yf[torch.from_numpy(ms).cuda()])
+    assert_conv_close(got, ref, name, wl.dtype)
+
+
+def test_small_workload_full_output(cuda_ok):
+    wl = workloads.WORKLOADS[workloads.SMALL]
+    inp = workloads.make_inputs(wl, device="cuda")
+    y = _run(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act)
+    ref = _ref(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act)
+    assert_conv_close(to_np_f32(y), ref, wl.name, wl.dtype)
