@@ -1,0 +1,431 @@
+#!/usr/bin/env python
+"""Benchmark of the Conv3D implicit-GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the workload's
+synthetic input: the convolution with fused NVFP4 activation fake-quant
+(conv3d_implicit_gemm_pad2, quant_act as the workload says) followed by the
+standalone fake-quantisation of the same activation tensor (fp4_fake_quant).
+The metric is 2*M*Cout*K / step time in TFLOP/s (the convolution's
+operations; the fake-quant adds time, not operations).
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
+device synchronisation on both sides, measured with CUDA events on the
+launching stream; the reported time is the maximum over ranks.  Inputs rotate
+over enough copies that the working set exceeds the 126 MB L2, so no step
+starts with its operands in L2.  SM clocks and throttle reasons are sampled
+through NVML during the timed region.
+
+Multi-GPU (torchrun): every rank runs its own independent copy of the layer
+on its own seeded input (weak scaling, no collective on the data path);
+value = all ranks' operations / max-over-ranks time.
+
+--impl reference times the CPU oracle (the test infrastructure's plain
+reference) on the host cores for the same workload, each step a bounded
+sample of output rows; only rank 0 does work.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# clock sampling (NVML reads only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+
+    def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nv = pynvml
+            self.ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, b in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=2)
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def pad6(wl):
+    return (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    from quantized_conv3d_implicit_b200 import api, workloads
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    wl = workloads.WORKLOADS[args.workload]
+    api.load_library()
+    stream = torch.cuda.current_stream(dev)
+
+    # independent seeded input per rank; rotate copies so the working set exceeds L2
+    base = workloads.make_inputs(dataclass_replace(wl, seed=wl.seed + 1000 * rank), device=dev, with_out=True)
+    per_set = sum(t.numel() * t.element_size() for t in (base["x"], base["w"], base["out"]))
+    n_sets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = [base] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in base.items()} for _ in range(n_sets - 1)]
+    for s in sets:
+        s["fq"] = torch.empty_like(s["x"])
+
+    def step(s):
+        api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
+                                 wl.quant_act, out=s["out"], stream=stream)
+        api.fp4_fake_quant(s["x"], s["act_amax"], out=s["fq"], stream=stream)
+
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    torch.cuda.synchronize(dev)
+    if api.check_device_error(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # timed region: K steps; per-kernel events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        s = sets[i % n_sets]
+        a, b, c = ev[i]
+        a.record(stream)
+        api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
+                                 wl.quant_act, out=s["out"], stream=stream)
+        b.record(stream)
+        api.fp4_fake_quant(s["x"], s["act_amax"], out=s["fq"], stream=stream)
+        c.record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier(world, dev)
+    local_ms = t0.elapsed_time(t1)
+    conv_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    fq_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    if api.check_device_error(stream) != 0:
+        raise RuntimeError("device error during timing")
+    total_ms = max_over_ranks(local_ms, world, dev)
+    ms_per_step = total_ms / args.steps
+    tflops = world * wl.flops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end-to-end through the public API with pinned host buffers
+    e2e = run_e2e(args, wl, base, stream, dev, world, step_fn=None)
+
+    peaks, peaks_src = load_peaks()
+    conv_tflops = wl.flops / (conv_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    launches_per_step = 2 + (0 if (wl.dtype == torch.bfloat16 and wl.k_gemm % 8 == 0) else 1)
+    od, oh, ow = wl.out_spatial()
+    result = {
+        "metric": "Conv3D TFLOP/s (2*M*N*K) and % of B200 BF16 dense peak; us/layer",
+        "value": round(tflops, 3),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[wl.dtype] + "->bf16 mma, f32 acc",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(K)) weights)",
+        "config": {
+            "workload": wl.name, "x": list(wl.x_shape), "w": [wl.cout, wl.x_shape[1], *wl.kernel],
+            "stride": list(wl.stride), "pad_lo": list(wl.pad_lo), "pad_hi": list(wl.pad_hi), "dil": list(wl.dil),
+            "quant_act": wl.quant_act, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
+            "step": "conv3d_implicit_gemm(quant_act) + fp4_fake_quant(x)",
+            "l2": f"inputs rotate over {n_sets} copies ({n_sets * per_set / 2**20:.0f} MiB > 126 MiB L2)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "layer_us": round(conv_ms * 1e3, 2),
+        "fake_quant_us": round(fq_ms * 1e3, 2),
+        "layer_frac_of_peak": round(conv_tflops / peak, 4),
+        "roofline": {
+            "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(conv_tflops / peak, 4), "traffic": None,
+            "kernel": "conv3d_igemm (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
+        },
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, base, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def dataclass_replace(wl, **kw):
+    import dataclasses
+    return dataclasses.replace(wl, **kw)
+
+
+def run_e2e(args, wl, base, stream, dev, world, step_fn=None):
+    """Same metric through the public calls with pinned host inputs: every step
+    copies x, w, bias and act_amax host->device, runs the hot path and copies
+    the convolution output and the fake-quantised tensor back."""
+    import torch
+
+    from quantized_conv3d_implicit_b200 import api
+
+    host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in base.items()}
+    dx = torch.empty_like(base["x"])
+    dw = torch.empty_like(base["w"])
+    db = None if base["bias"] is None else torch.empty_like(base["bias"])
+    da = torch.empty_like(base["act_amax"])
+    dy = torch.empty_like(base["out"])
+    dq = torch.empty_like(base["x"])
+    hy = torch.empty(dy.shape, dtype=dy.dtype, pin_memory=True)
+    hq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
+
+    def step():
+        dx.copy_(host["x"], non_blocking=True)
+        dw.copy_(host["w"], non_blocking=True)
+        if db is not None:
+            db.copy_(host["bias"], non_blocking=True)
+        da.copy_(host["act_amax"], non_blocking=True)
+        api.conv3d_implicit_gemm(dx, dw, db, wl.stride, pad6(wl), wl.dil, da, wl.quant_act, out=dy, stream=stream)
+        api.fp4_fake_quant(dx, da, out=dq, stream=stream)
+        hy.copy_(dy, non_blocking=True)
+        hq.copy_(dq, non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (host["x"], host["w"], host["act_amax"])) + \
+        (0 if db is None else db.numel() * db.element_size())
+    d2h = hy.numel() * hy.element_size() + hq.numel() * hq.element_size()
+    return {"value": round(world * wl.flops / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(ms, 4),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (test infrastructure: the only place bench.py runs it)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng):
+    import numpy as np
+
+    import oracle
+    ms = rng.integers(0, wl.m_gemm, rows)
+    t = time.perf_counter()
+    oracle.conv3d(x_np, w_np, b_np, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act, amax, m_list=ms)
+    t_conv = time.perf_counter() - t
+    start = int(rng.integers(0, max(1, x_np.size // 16 - fq_elems // 16))) * 16
+    t = time.perf_counter()
+    oracle.fp4_fake_quant(x_np.reshape(-1)[start:start + fq_elems], amax)
+    t_fq = time.perf_counter() - t
+    return t_conv, t_fq, ms.size
+
+
+def cpu_baseline(wl, base, budget_s: float = 15.0):
+    import numpy as np
+    x_np = base["x"].float().cpu().numpy()
+    w_np = base["w"].float().cpu().numpy()
+    b_np = None if base["bias"] is None else base["bias"].float().cpu().numpy()
+    amax = float(base["act_amax"].item())
+    rng = np.random.default_rng(1234)
+    # calibrate on a few rows, then size the sample to the time budget
+    t_conv, _, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, 16, 16 * 1024, rng)
+    per_row = max(t_conv / n, 1e-6)
+    rows = int(max(32, min(wl.m_gemm, budget_s * 0.8 / per_row)))
+    fq_elems = 1 << 20
+    t_conv, t_fq, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng)
+    # extrapolate one full step (all M rows + the whole fake-quant tensor)
+    step_s = t_conv * wl.m_gemm / n + t_fq * (x_np.size / fq_elems)
+    return {"value": wl.flops / step_s / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{n} random output rows x all {wl.cout} channels ({t_conv:.1f} s) + fake-quant of "
+                      f"{fq_elems} elements ({t_fq:.2f} s), extrapolated to the full layer "
+                      f"({step_s:.0f} s per step)"}
+
+
+def run_reference(args, world, rank, local):
+    """The oracle on the host cores, same workload/metric; rank 0 only."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    from quantized_conv3d_implicit_b200 import workloads
+    wl = workloads.WORKLOADS[args.workload]
+    base = workloads.make_inputs(wl, device="cpu")
+    x_np = base["x"].float().numpy()
+    w_np = base["w"].float().numpy()
+    b_np = None if base["bias"] is None else base["bias"].float().numpy()
+    amax = float(base["act_amax"].item())
+    rng = np.random.default_rng(99)
+    t_conv, _, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, 16, 16 * 1024, rng)
+    rows = int(max(32, min(wl.m_gemm, 1.0 / max(t_conv / n, 1e-6))))   # about 1 s of work per step
+    fq_elems = 1 << 18
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, x_np, w_np, b_np, amax, max(8, rows // 8), fq_elems, rng)
+    tot_conv = tot_fq = 0.0
+    for _ in range(args.steps):
+        tc, tf, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng)
+        tot_conv += tc
+        tot_fq += tf
+    step_s = (tot_conv / args.steps) * wl.m_gemm / rows + (tot_fq / args.steps) * (x_np.size / fq_elems)
+    value = wl.flops / step_s / 1e12
+    od, oh, ow = wl.out_spatial()
+    sample = (f"each step: {rows} random output rows x all {wl.cout} channels + fake-quant of {fq_elems} "
+              f"elements, extrapolated to the full layer")
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "Conv3D TFLOP/s (2*M*N*K) and % of B200 BF16 dense peak; us/layer",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 accumulate over bf16/fp4 operands (CPU oracle)", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
+                   "quant_act": wl.quant_act},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    from quantized_conv3d_implicit_b200 import workloads
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus and world > 1:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        run_reference(args, world, rank, local)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -153,6 +153,20 @@ Q3D_API int32_t q3d_version(void);
  */
 Q3D_API q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream);
 
+/*
+ * q3d_plan_conv -- TEST HOOK (host only, no CUDA call): the tiling and
+ * pipeline plan the specialised sm_100a kernel would use for a convolution of
+ * this geometry and dtype.  plan[0..plan_len) receives, in order: applicable
+ * (0/1), TH, TW, n_mt, groups, n_tile, n_ntiles, n_sub, sub_n, K slices per
+ * tile, channels per halo slot, halo slots per tile, halo ring entries,
+ * A stages, B stages, TMEM columns, shared-memory bytes, tiles along OH,
+ * tiles along OW, vectorised halo reads (0/1), halo box W, H and D extents;
+ * further entries are 0.
+ */
+Q3D_API q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                                 const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                                 int32_t dtype, int32_t* plan, int32_t plan_len);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -24,7 +24,8 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "fp4_fake_quant", "q3d_last_error",
-           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats")
+           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats",
+           "q3d_plan_conv")
 
 
 class Q3DTensor(ctypes.Structure):
@@ -69,6 +70,10 @@ def load_library(path: Optional[str] = None):
         lib.q3d_version.restype = ctypes.c_int32
         lib.q3d_selftest_formats.restype = ctypes.c_int
         lib.q3d_selftest_formats.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
+        i64x5 = ctypes.POINTER(ctypes.c_int64)
+        lib.q3d_plan_conv.restype = ctypes.c_int
+        lib.q3d_plan_conv.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32,
+                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
         if path is None:
             _lib = lib
         return lib
@@ -197,3 +202,21 @@ def selftest_formats(v: torch.Tensor, stream=None):
     st = lib.q3d_selftest_formats(v.data_ptr(), v.numel(), e2m1.data_ptr(), e4m3.data_ptr(), _stream_handle(stream))
     _check(lib, st)
     return e2m1, e4m3
+
+
+PLAN_FIELDS = ("applicable", "TH", "TW", "n_mt", "groups", "n_tile", "n_ntiles", "n_sub", "sub_n", "ks", "c_slot",
+               "q_slots", "ring", "sa", "sb", "tmem_cols", "smem", "n_ohb", "n_owb", "vec", "w_box", "h_ext", "kd_ext")
+
+
+def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfloat16) -> dict:
+    """Test hook (host only): the specialised kernel's tiling/pipeline plan."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    a5 = lambda t: (ctypes.c_int64 * 5)(*[int(v) for v in t])  # noqa: E731
+    out = (ctypes.c_int32 * 32)()
+    st = lib.q3d_plan_conv(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)),
+                           _DTYPES[dtype], out, 32)
+    _check(lib, st)
+    return dict(zip(PLAN_FIELDS, list(out)[:len(PLAN_FIELDS)]))
+

@@ -5,31 +5,37 @@
 // article, sec. 5.1 (rows (n, od, oh, ow), columns (c, kd, kh, kw)), with the
 // NVFP4 activation quantiser of sec. 6.3 fused into the A-operand producer.
 //
-// One CTA per SM walks output tiles of 128 positions (TH x TW rectangle of
-// one (n, od) plane) x n_tile output channels.  Roles (16 warps):
-//   warp 0       TMA producer: for every tile, 5-D halo boxes of x (C_slot
-//                channels x KD_ext x H_ext x W_box, out-of-range coordinates
-//                zero-filled, which is exactly the convolution padding) into
-//                a ring of channel slots, and 128B-swizzled 64-wide K slices
-//                of the BF16 weights;
-//   warp 1       TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128,
-//                N = n_tile (split into <= 256 wide instructions), K = 16
-//                (one quantisation block), FP32 accumulators in TMEM, double
-//                buffered when 2 * n_tile <= 512 columns;
-//   warps 4-7    epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//                lanes 32*(w%4)..+31), bias add in FP32, rounding to the
-//                output dtype, bounds-checked NCDHW stores;
-//   warps 8-15   transform: thread (half h, row r) builds the 32 columns
-//                [32h, 32h+32) of row r of each 64-wide A slice from the halo
-//                (on-the-fly (c, kd, kh, kw) decomposition, no tables), and
-//                fake-quantises each 16-column block as a register reduction
-//                (the thread owns the whole block), then writes BF16 in the
-//                swizzled K-major layout; rows of a warp are consecutive so
-//                the 16-byte stores are bank-conflict free.
-// Pipelines: halo ring (full/empty), A stages (full: 8 transform warps,
-// empty: tcgen05.commit), B stages (full: TMA tx, empty: commit),
-// accumulators (full: commit, empty: 4 epilogue warps).  Every wait is
-// bounded and any timeout aborts all roles through a shared flag.
+// One CTA per SM walks output tiles.  A tile is n_mt M-subtiles of 128
+// output positions (each a TH x TW rectangle of one (n, od) plane, stacked
+// along oh) times n_tile output channels.  Every 64-wide K slice of the BF16
+// weights is loaded once per tile and feeds all n_mt subtiles, so the weight
+// traffic per tensor-core cycle shrinks by n_mt; the accumulators of the
+// subtiles (n_mt * n_tile <= 512 FP32 columns) live in tensor memory.
+//
+// Roles (16 warps):
+//   warp 0     weight producer: TMA of 128B-swizzled K-major weight slices;
+//   warp 1     TMEM owner and MMA issuer: tcgen05.mma kind::f16, M = 128,
+//              N = n_tile in <= 256-wide instructions, K = 16 (one
+//              quantisation block), per subtile;
+//   warp 2     halo producer: 5-D TMA boxes of x (C_slot channels x KD_ext x
+//              H_ext x W_box; out-of-range coordinates are zero-filled, which
+//              is exactly the convolution padding) into a ring of slots;
+//   warps 4-7  epilogue: tcgen05.ld (warp w reads TMEM lanes 32*(w%4)..+31),
+//              bias in FP32, rounding to the output dtype, bounds-checked
+//              NCDHW stores; each (subtile, N-part) accumulator is handed
+//              back as soon as it is drained, so the next tile's MMAs start
+//              while the rest is still being written;
+//   warps 8-15 transform: a thread owns 8 consecutive output rows and one
+//              16-column quantisation block.  It walks the block's taps
+//              (c, kd, kh, kw) incrementally (no divisions, no tables),
+//              reads the 8 rows of each tap with 32-bit shared loads and a
+//              byte permute, takes the block maximum of each row as a packed
+//              register reduction, derives the E4M3 scale with an IEEE
+//              division and a per-CTA table of
+//              (scale, 1/scale) per E4M3 code, and writes BF16 in the
+//              MN-major 128B-swizzled layout (one conflict-free 16-byte store
+//              per tap).
+// All waits are bounded; a timeout in any role aborts all roles.
 #include <algorithm>
 #include <cstdint>
 #include <cstdlib>
@@ -45,15 +51,16 @@ namespace q3d {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kWarpProducer = 0;
+constexpr int kWarpB = 0;
 constexpr int kWarpMma = 1;
+constexpr int kWarpHalo = 2;
 constexpr int kWarpEpi0 = 4;
 constexpr int kWarpXf0 = 8;
 constexpr int kNumXfWarps = 8;
-constexpr int kBlockM = 128;
 constexpr int kBlockK = 64;
-constexpr uint32_t kATileBytes = kBlockM * kBlockK * 2;
-constexpr int kMaxSmem = 232448;  // 227 KB dynamic shared memory per CTA
+constexpr uint32_t kASubBytes = 128u * kBlockK * 2u;  // one 128-row subtile of one K slice
+constexpr int kMaxSmem = 232448;                      // 227 KB dynamic shared memory per CTA
+constexpr int kMaxAcc = 8;
 
 struct FastParams {
   ConvGeom g;
@@ -62,30 +69,31 @@ struct FastParams {
   const float* act_amax;
   unsigned int* err;
   int quant;
-  // output tiling
-  int TH, TW, n_ohb, n_owb;
+  // tiling
+  int TH, TW, n_mt;       // subtile = TH x TW = 128 positions; a tile stacks n_mt subtiles along oh
+  int n_ohb, n_owb;
   int n_tile, n_ntiles, n_sub, sub_n;
   int64_t num_tiles;
-  int ks;  // 64-wide K slices per tile
+  int ks;                 // K slices per tile
   // halo staging
-  int align_elems;  // 16 bytes in elements
+  int align;              // 16 bytes in elements
   int w_box, h_ext, kd_ext, c_slot, q_slots, chan_elems;
   uint32_t slot_bytes, slot_tx;
   int ring;
-  // pipeline depths
-  int sa, sb, n_acc, tmem_cols;
-  uint32_t b_stage_bytes;
-  // shared memory map (bytes from the 1024-aligned base)
-  uint32_t off_a, off_b, off_halo, off_bar;
+  // pipelines
+  int sa, sb, groups;     // A stages, B stages, transform groups working on separate slices
+  uint32_t a_stage_bytes, b_stage_bytes;
+  int tmem_cols;
+  int vec;                // 1: unit W stride and 16-bit input -> vectorised halo reads
+  uint32_t off_a, off_b, off_halo, off_tab, off_bar;
 };
 
 struct TileCoord {
   int n, od, oh0, ow0, nt;
 };
 
-// Tile order: output-channel tile fastest, then the frame od, then the
-// spatial blocks; consecutive tiles (running concurrently on neighbouring
-// SMs) share two of their three input frames and their halo columns in L2.
+// Output-channel tile fastest, then the frame od, then the spatial blocks:
+// tiles running concurrently share two of their three input frames in L2.
 __device__ __forceinline__ TileCoord decode_tile(const FastParams& p, int64_t t) {
   TileCoord c;
   c.nt = static_cast<int>(t % p.n_ntiles); t /= p.n_ntiles;
@@ -93,20 +101,25 @@ __device__ __forceinline__ TileCoord decode_tile(const FastParams& p, int64_t t)
   const int owb = static_cast<int>(t % p.n_owb); t /= p.n_owb;
   const int ohb = static_cast<int>(t % p.n_ohb);
   c.n = static_cast<int>(t / p.n_ohb);
-  c.oh0 = ohb * p.TH;
+  c.oh0 = ohb * p.TH * p.n_mt;
   c.ow0 = owb * p.TW;
   return c;
 }
 
 __device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
 
-// First input column covered by the halo of a tile: the leftmost tap,
-// rounded down to a 16-byte boundary (the TMA start coordinate rule).
+// First input column of a tile's halo: the leftmost tap rounded down to a
+// 16-byte boundary (the TMA start-coordinate rule).
 __device__ __forceinline__ int halo_w0(const FastParams& p, int ow0) {
-  return floor_div(ow0 * p.g.sw - p.g.pw, p.align_elems) * p.align_elems;
+  return floor_div(ow0 * p.g.sw - p.g.pw, p.align) * p.align;
 }
 
-// Wait that also gives up early when another role has aborted.
+// Lowest / highest halo slot holding a column of K slice s.
+__device__ __forceinline__ int slot_lo(const FastParams& p, int s) { return ((kBlockK * s) / p.g.taps) / p.c_slot; }
+__device__ __forceinline__ int slot_hi(const FastParams& p, int s) {
+  return (min(kBlockK * s + kBlockK - 1, p.g.K - 1) / p.g.taps) / p.c_slot;
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, unsigned int* err, unsigned int site,
                                               volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -124,17 +137,253 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uns
   }
 }
 
+// Incremental walk over the K columns (c, kd, kh, kw) of one thread's
+// quantisation block, tracking the element offset of the tap inside the halo
+// slot that holds channel c and the byte address of that slot.
+struct TapWalker {
+  int kw, kh, kd, cs;       // tap and channel-within-slot
+  int q;                    // slot index within the tile
+  int u;                    // element offset of the tap inside its slot (without the thread's own offset)
+  uint32_t slot_addr;       // shared address of slot q
+
+  __device__ __forceinline__ void init(const FastParams& p, int k, uint32_t halo_base, uint32_t slot_base) {
+    const ConvGeom& g = p.g;
+    const int c = k / g.taps;
+    int r = k - c * g.taps;
+    const int khw = g.KH * g.KW;
+    kd = r / khw;
+    r -= kd * khw;
+    kh = r / g.KW;
+    kw = r - kh * g.KW;
+    q = c / p.c_slot;
+    cs = c - q * p.c_slot;
+    u = cs * p.chan_elems + kd * g.dd * p.h_ext * p.w_box + kh * g.dh * p.w_box + kw * g.dw;
+    slot_addr = halo_base + ((slot_base + static_cast<uint32_t>(q)) % static_cast<uint32_t>(p.ring)) * p.slot_bytes;
+  }
+
+  __device__ __forceinline__ void step(const FastParams& p, uint32_t halo_base, uint32_t slot_base) {
+    const ConvGeom& g = p.g;
+    u += g.dw;
+    if (++kw == g.KW) {
+      kw = 0;
+      u += g.dh * p.w_box - g.KW * g.dw;
+      if (++kh == g.KH) {
+        kh = 0;
+        u += g.dd * p.h_ext * p.w_box - g.KH * g.dh * p.w_box;
+        if (++kd == g.KD) {
+          kd = 0;
+          u += p.chan_elems - g.KD * g.dd * p.h_ext * p.w_box;
+          if (++cs == p.c_slot) {
+            cs = 0;
+            u = 0;
+            ++q;
+            slot_addr = halo_base + ((slot_base + static_cast<uint32_t>(q)) % static_cast<uint32_t>(p.ring)) *
+                                        p.slot_bytes;
+          }
+        }
+      }
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ uint32_t max_abs_x2_bf16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t max_abs_x2_f16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 template <typename T>
-__device__ __forceinline__ float lds_as_f32(const uint8_t* p);
+struct Pair16;
 template <>
-__device__ __forceinline__ float lds_as_f32<float>(const uint8_t* p) { return *reinterpret_cast<const float*>(p); }
+struct Pair16<__nv_bfloat16> {
+  static __device__ __forceinline__ float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return max_abs_x2_bf16(a, b); }
+  static __device__ __forceinline__ float abs_lo(uint32_t w) { return __uint_as_float((w << 16) & 0x7FFFFFFFu); }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) { return __uint_as_float(w & 0x7FFF0000u); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
+};
 template <>
-__device__ __forceinline__ float lds_as_f32<__half>(const uint8_t* p) {
-  return __half2float(*reinterpret_cast<const __half*>(p));
+struct Pair16<__half> {
+  static __device__ __forceinline__ float lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+  }
+  static __device__ __forceinline__ float hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+  }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return max_abs_x2_f16(a, b); }
+  static __device__ __forceinline__ float abs_lo(uint32_t w) { return fabsf(lo(w)); }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) { return fabsf(hi(w)); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return pack_bf16x2(lo(w), hi(w)); }
+};
+
+// Fake-quantise a pair of values from two different rows (own scales).
+__device__ __forceinline__ uint32_t quant_pair_bf16x2(float v0, float v1, float inv0, float inv1, float s0, float s1) {
+  const float a0 = __fmul_rn(v0, inv0);
+  const float a1 = __fmul_rn(v1, inv1);
+  uint32_t h2;
+  asm("{\n\t.reg .b8 q;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q;\n\t}"
+      : "=r"(h2)
+      : "f"(a1), "f"(a0));
+  const float q0 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+  const float q1 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+  return pack_bf16x2(__fmul_rn(q0, s0), __fmul_rn(q1, s1));
+}
+
+// Scales of two rows from their block maxima: IEEE bmax / (6 g), clamp to
+// 448, E4M3 rounding of both rows in one conversion, then (scale, 1/scale)
+// from the per-CTA table indexed by the E4M3 code.
+__device__ __forceinline__ void row_scales(float bmax0, float bmax1, float t, uint32_t tab,
+                                           float& s0, float& i0, float& s1, float& i1) {
+  const float r0 = fminf(__fdiv_rn(bmax0, t), 448.0f);
+  const float r1 = fminf(__fdiv_rn(bmax1, t), 448.0f);
+  uint16_t codes;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(codes) : "f"(r1), "f"(r0));
+  float2 e0, e1;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(e0.x), "=f"(e0.y) : "r"(tab + (codes & 0x7Fu) * 8u));
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(e1.x), "=f"(e1.y) : "r"(tab + ((codes >> 8) & 0x7Fu) * 8u));
+  s0 = e0.x; i0 = e0.y;
+  s1 = e1.x; i1 = e1.y;
+}
+
+// MN-major swizzled position of 8 rows (row group rg) x column kk of a
+// subtile's K slice: atom (kk/8, rg/8) of 1 KB, K-row kk%8, chunk rg%8.
+__device__ __forceinline__ uint32_t a_chunk_offset(int rg, int kk) {
+  const int kr = kk & 7;
+  return static_cast<uint32_t>(((kk >> 3) * 2 + (rg >> 3)) * 1024 + kr * 128 + (((rg & 7) ^ kr) << 4));
+}
+
+// ---------------------------------------------------------------------------
+// transform: one task = 8 rows (row group rg of subtile i) x 16 columns
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ void transform_task_vec(const FastParams& p, uint32_t a_sub, int rg, int kb, int thr_al,
+                                                  int delta, uint32_t halo_base, uint32_t slot_base,
+                                                  const float t, uint32_t tab) {
+  // 16 columns x 4 words (pairs of rows (2j, 2j+1))
+  uint32_t d[16][4];
+  TapWalker wk;
+  wk.init(p, kb, halo_base, slot_base);
+#pragma unroll
+  for (int kk = 0; kk < 16; ++kk) {
+    if (kb + kk < p.g.K) {
+      const int e = thr_al + wk.u + delta;
+      const uint32_t addr = wk.slot_addr + static_cast<uint32_t>(e & ~1) * 2u;
+      const uint32_t sel = (e & 1) ? 0x5432u : 0x3210u;
+      const uint32_t w0 = lds32(addr), w1 = lds32(addr + 4), w2 = lds32(addr + 8), w3 = lds32(addr + 12),
+                     w4 = lds32(addr + 16);
+      d[kk][0] = __byte_perm(w0, w1, sel);
+      d[kk][1] = __byte_perm(w1, w2, sel);
+      d[kk][2] = __byte_perm(w2, w3, sel);
+      d[kk][3] = __byte_perm(w3, w4, sel);
+    } else {
+      d[kk][0] = d[kk][1] = d[kk][2] = d[kk][3] = 0u;
+    }
+    if (kk < 15) wk.step(p, halo_base, slot_base);
+  }
+  if (p.quant) {
+    uint32_t mx[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      mx[j] = Pair16<T>::maxabs(d[0][j], d[1][j]);
+#pragma unroll
+      for (int kk = 2; kk < 16; ++kk) mx[j] = Pair16<T>::maxabs(mx[j], d[kk][j]);
+    }
+    float sc[8], iv[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      row_scales(Pair16<T>::abs_lo(mx[j]), Pair16<T>::abs_hi(mx[j]), t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1],
+                 iv[2 * j + 1]);
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        d[kk][j] = quant_pair_bf16x2(Pair16<T>::lo(d[kk][j]), Pair16<T>::hi(d[kk][j]), iv[2 * j], iv[2 * j + 1],
+                                     sc[2 * j], sc[2 * j + 1]);
+      sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), d[kk][0], d[kk][1], d[kk][2], d[kk][3]);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk)
+      sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), Pair16<T>::to_bf16x2(d[kk][0]),
+             Pair16<T>::to_bf16x2(d[kk][1]), Pair16<T>::to_bf16x2(d[kk][2]), Pair16<T>::to_bf16x2(d[kk][3]));
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float lds_elem(uint32_t addr);
+template <>
+__device__ __forceinline__ float lds_elem<float>(uint32_t addr) { return __uint_as_float(lds32(addr)); }
+template <>
+__device__ __forceinline__ float lds_elem<__half>(uint32_t addr) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(lds16(addr))));
 }
 template <>
-__device__ __forceinline__ float lds_as_f32<__nv_bfloat16>(const uint8_t* p) {
-  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(p)) << 16);
+__device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t addr) { return __uint_as_float(lds16(addr) << 16); }
+
+// General path (any W stride, any dtype): element loads, two passes (block
+// maxima, then quantisation) so only one column is held at a time.
+template <typename T>
+__device__ __forceinline__ void transform_task_gen(const FastParams& p, uint32_t a_sub, int rg, int kb,
+                                                  const int (&roff)[8], uint32_t halo_base, uint32_t slot_base,
+                                                  const float t, uint32_t tab) {
+  constexpr uint32_t esz = sizeof(T);
+  float sc[8], iv[8];
+  if (p.quant) {
+    float bm[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) bm[r] = 0.0f;
+    TapWalker wk;
+    wk.init(p, kb, halo_base, slot_base);
+#pragma unroll 1
+    for (int kk = 0; kk < 16; ++kk) {
+      if (kb + kk < p.g.K) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+          bm[r] = fmaxf(bm[r], fabsf(lds_elem<T>(wk.slot_addr + static_cast<uint32_t>(wk.u + roff[r]) * esz)));
+      }
+      if (kk < 15) wk.step(p, halo_base, slot_base);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      row_scales(bm[2 * j], bm[2 * j + 1], t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1], iv[2 * j + 1]);
+  }
+  TapWalker wk;
+  wk.init(p, kb, halo_base, slot_base);
+#pragma unroll 1
+  for (int kk = 0; kk < 16; ++kk) {
+    float v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      v[r] = (kb + kk < p.g.K) ? lds_elem<T>(wk.slot_addr + static_cast<uint32_t>(wk.u + roff[r]) * esz) : 0.0f;
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = p.quant ? quant_pair_bf16x2(v[2 * j], v[2 * j + 1], iv[2 * j], iv[2 * j + 1], sc[2 * j], sc[2 * j + 1])
+                     : pack_bf16x2(v[2 * j], v[2 * j + 1]);
+    sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), w[0], w[1], w[2], w[3]);
+    if (kk < 15) wk.step(p, halo_base, slot_base);
+  }
 }
 
 template <typename T>
@@ -146,17 +395,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
 
-  // barrier map
-  const uint32_t bar0 = base + p.off_bar;
-  const uint32_t bar_halo_full = bar0;
+  const uint32_t bar_halo_full = base + p.off_bar;
   const uint32_t bar_halo_empty = bar_halo_full + 8u * p.ring;
   const uint32_t bar_b_full = bar_halo_empty + 8u * p.ring;
   const uint32_t bar_b_empty = bar_b_full + 8u * p.sb;
   const uint32_t bar_a_full = bar_b_empty + 8u * p.sb;
   const uint32_t bar_a_empty = bar_a_full + 8u * p.sa;
   const uint32_t bar_acc_full = bar_a_empty + 8u * p.sa;
-  const uint32_t bar_acc_empty = bar_acc_full + 16u;
-  const uint32_t bar_drain = bar_acc_empty + 16u;
+  const uint32_t bar_acc_empty = bar_acc_full + 8u * kMaxAcc;
+  const uint32_t bar_drain = bar_acc_empty + 8u * kMaxAcc;
   const uint32_t bar_end = bar_drain + 8u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bar_end - base));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + (bar_end - base) + 4);
@@ -164,21 +411,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const ConvGeom& g = p.g;
+  const int xf_warps_per_group = kNumXfWarps / p.groups;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.ring; ++i) {
       mbar_init(bar_halo_full + 8u * i, 1);
-      mbar_init(bar_halo_empty + 8u * i, kNumXfWarps);
+      mbar_init(bar_halo_empty + 8u * i, 1);
     }
     for (int i = 0; i < p.sb; ++i) {
       mbar_init(bar_b_full + 8u * i, 1);
       mbar_init(bar_b_empty + 8u * i, 1);
     }
     for (int i = 0; i < p.sa; ++i) {
-      mbar_init(bar_a_full + 8u * i, kNumXfWarps);
+      mbar_init(bar_a_full + 8u * i, xf_warps_per_group);
       mbar_init(bar_a_empty + 8u * i, 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxAcc; ++i) {
       mbar_init(bar_acc_full + 8u * i, 1);
       mbar_init(bar_acc_empty + 8u * i, 4);
     }
@@ -196,36 +444,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == kWarpProducer) {
-    // ------------------------------------------------------------------ producer
+  if (warp == kWarpB) {
+    // ------------------------------------------------------------ weight producer
     if (lane == 0) {
-      uint32_t slot_ctr = 0, bst = 0;
-      int64_t last_slot = -1, last_b = -1;
+      uint32_t gb = 0;
+      int64_t last = -1;
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
-        const int w0 = halo_w0(p, tc.ow0);
-        const int h0 = tc.oh0 * g.sh - g.ph;
-        const int d0 = tc.od * g.sd - g.pd;
-        int q_issued = 0;
-        for (int s = 0; ok && s < p.ks; ++s) {
-          const int k_last = min(kBlockK * s + kBlockK - 1, g.K - 1);
-          const int q_need = (k_last / g.taps) / p.c_slot;
-          while (q_issued <= q_need) {
-            const uint32_t e = slot_ctr % p.ring, u = slot_ctr / p.ring;
-            if (u > 0 && !wait_or_abort(bar_halo_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteHaloEmpty, abort_flag)) {
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(bar_halo_full + 8u * e, p.slot_tx);
-            tma_load_5d(base + p.off_halo + e * p.slot_bytes, &tmap_x, bar_halo_full + 8u * e, w0, h0, d0,
-                        q_issued * p.c_slot, tc.n);
-            last_slot = slot_ctr;
-            ++q_issued;
-            ++slot_ctr;
-          }
-          if (!ok) break;
-          const uint32_t e = bst % p.sb, u = bst / p.sb;
+        for (int s = 0; s < p.ks; ++s, ++gb) {
+          const uint32_t e = gb % p.sb, u = gb / p.sb;
           if (u > 0 && !wait_or_abort(bar_b_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteProducerEmpty, abort_flag)) {
             ok = false;
             break;
@@ -234,57 +462,91 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < p.n_sub; ++i)
             tma_load_2d(base + p.off_b + e * p.b_stage_bytes + static_cast<uint32_t>(i * p.sub_n) * 128u, &tmap_w,
                         bar_b_full + 8u * e, kBlockK * s, tc.nt * p.n_tile + i * p.sub_n);
-          last_b = bst;
-          ++bst;
+          last = gb;
         }
       }
-      if (!ok) {
-        // let the last copies of each kind land before the CTA exits
-        if (last_slot >= 0)
-          mbar_wait(bar_halo_full + 8u * static_cast<uint32_t>(last_slot % p.ring),
-                    static_cast<uint32_t>(last_slot / p.ring) & 1u, p.err, kSiteDrain);
-        if (last_b >= 0)
-          mbar_wait(bar_b_full + 8u * static_cast<uint32_t>(last_b % p.sb), static_cast<uint32_t>(last_b / p.sb) & 1u,
-                    p.err, kSiteDrain);
-      }
+      if (!ok && last >= 0)
+        mbar_wait(bar_b_full + 8u * static_cast<uint32_t>(last % p.sb), static_cast<uint32_t>(last / p.sb) & 1u, p.err,
+                  kSiteDrain);
     }
-  } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == kWarpHalo) {
+    // ------------------------------------------------------------ halo producer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(kBlockM, static_cast<uint32_t>(p.sub_n));
-      uint32_t ast = 0, bst = 0, acc_ctr = 0;
+      uint32_t gs = 0;
+      int64_t last = -1;
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-        const uint32_t eb = acc_ctr % p.n_acc, ub = acc_ctr / p.n_acc;
-        if (ub > 0 && !wait_or_abort(bar_acc_empty + 8u * eb, (ub - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag)) {
-          ok = false;
-          break;
+        const TileCoord tc = decode_tile(p, t);
+        const int w0 = halo_w0(p, tc.ow0);
+        const int h0 = tc.oh0 * g.sh - g.ph;
+        const int d0 = tc.od * g.sd - g.pd;
+        for (int q = 0; q < p.q_slots; ++q, ++gs) {
+          const uint32_t e = gs % p.ring, u = gs / p.ring;
+          if (u > 0 && !wait_or_abort(bar_halo_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteHaloEmpty, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_halo_full + 8u * e, p.slot_tx);
+          tma_load_5d(base + p.off_halo + e * p.slot_bytes, &tmap_x, bar_halo_full + 8u * e, w0, h0, d0,
+                      q * p.c_slot, tc.n);
+          last = gs;
         }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + eb * static_cast<uint32_t>(p.n_tile);
-        for (int s = 0; s < p.ks; ++s) {
-          const uint32_t ea = ast % p.sa, eB = bst % p.sb;
-          if (!wait_or_abort(bar_a_full + 8u * ea, (ast / p.sa) & 1u, p.err, kSiteAStageFull, abort_flag) ||
-              !wait_or_abort(bar_b_full + 8u * eB, (bst / p.sb) & 1u, p.err, kSiteTmaFull, abort_flag)) {
+      }
+      if (!ok && last >= 0)
+        mbar_wait(bar_halo_full + 8u * static_cast<uint32_t>(last % p.ring),
+                  static_cast<uint32_t>(last / p.ring) & 1u, p.err, kSiteDrain);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32_amn(128, static_cast<uint32_t>(p.sub_n));
+      uint32_t ga = 0, gb = 0, it = 0, gs_base = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+        int released = 0;
+        for (int s = 0; ok && s < p.ks; ++s, ++ga, ++gb) {
+          const uint32_t ea = ga % p.sa, eb = gb % p.sb;
+          if (!wait_or_abort(bar_a_full + 8u * ea, (ga / p.sa) & 1u, p.err, kSiteAStageFull, abort_flag)) {
+            ok = false;
+            break;
+          }
+          // Slices are complete in order up to s, and no later slice reads a
+          // halo slot below the first one slice s+1 needs: hand those back.
+          const int keep = (s + 1 < p.ks) ? slot_lo(p, s + 1) : p.q_slots;
+          for (; released < keep; ++released)
+            mbar_arrive(bar_halo_empty + 8u * ((gs_base + static_cast<uint32_t>(released)) % p.ring));
+          if (!wait_or_abort(bar_b_full + 8u * eb, (gb / p.sb) & 1u, p.err, kSiteTmaFull, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = umma_desc_kmajor_sw128(base + p.off_a + ea * kATileBytes);
-          const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eB * p.b_stage_bytes);
+          const uint32_t a_stage = base + p.off_a + ea * p.a_stage_bytes;
+          const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
+          for (int i = 0; ok && i < p.n_mt; ++i) {
+            const uint64_t adesc =
+                umma_desc_mnmajor_sw128(a_stage + static_cast<uint32_t>(i) * kASubBytes, 1024u, 2048u);
+            for (int ns = 0; ns < p.n_sub; ++ns) {
+              const int acc = i * p.n_sub + ns;
+              if (s == 0 && it > 0) {
+                if (!wait_or_abort(bar_acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
 #pragma unroll
-          for (int j = 0; j < kBlockK / 16; ++j)
-            for (int i = 0; i < p.n_sub; ++i)
-              umma_bf16(d_tmem + static_cast<uint32_t>(i * p.sub_n), adesc + 2u * j,
-                        bdesc + static_cast<uint64_t>(i * p.sub_n * 8) + 2u * j, idesc, (s > 0 || j > 0) ? 1u : 0u);
+              for (int j = 0; j < kBlockK / 16; ++j)
+                umma_bf16(d_tmem, adesc + static_cast<uint64_t>(j * 256),
+                          bdesc + static_cast<uint64_t>(ns * p.sub_n * 8 + 2 * j), idesc, (s > 0 || j > 0) ? 1u : 0u);
+              if (s == p.ks - 1) umma_commit(bar_acc_full + 8u * acc);
+            }
+          }
+          if (!ok) break;
           umma_commit(bar_a_empty + 8u * ea);
-          umma_commit(bar_b_empty + 8u * eB);
-          ++ast;
-          ++bst;
+          umma_commit(bar_b_empty + 8u * eb);
         }
-        if (!ok) break;
-        umma_commit(bar_acc_full + 8u * eb);
-        ++acc_ctr;
+        gs_base += static_cast<uint32_t>(p.q_slots);
       }
       if (!ok) {
         umma_commit(bar_drain);
@@ -292,140 +554,133 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
-    // ------------------------------------------------------------------ epilogue
-    const int ew = warp - kWarpEpi0;
-    const int r = ew * 32 + lane;
+    // ------------------------------------------------------------ epilogue
+    const int qw = warp - kWarpEpi0;
+    const int lr = qw * 32 + lane;  // row within a subtile
+    const int th_l = lr / p.TW, tw_l = lr % p.TW;
     const int S_hw = g.OH * g.OW;
     const int64_t S = static_cast<int64_t>(g.OD) * S_hw;
     T* y = static_cast<T*>(p.y);
     const T* bias = static_cast<const T*>(p.bias);
-    uint32_t acc_ctr = 0;
-    for (int64_t t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
-      const uint32_t eb = acc_ctr % p.n_acc;
-      if (!wait_or_abort(bar_acc_full + 8u * eb, (acc_ctr / p.n_acc) & 1u, p.err, kSiteAccFull, abort_flag)) break;
-      tc_fence_after();
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
       const TileCoord tc = decode_tile(p, t);
-      const int oh = tc.oh0 + r / p.TW, ow = tc.ow0 + r % p.TW;
-      const bool valid = oh < g.OH && ow < g.OW;
-      const int64_t ybase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
-                            static_cast<int64_t>(oh) * g.OW + ow;
-      const int co0 = tc.nt * p.n_tile;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + eb * static_cast<uint32_t>(p.n_tile);
-      for (int c0 = 0; c0 < p.n_tile; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
-        tmem_wait_ld();
-        if (valid) {
+      const int ow = tc.ow0 + tw_l;
+      for (int i = 0; ok && i < p.n_mt; ++i) {
+        const int oh = tc.oh0 + i * p.TH + th_l;
+        const bool valid = oh < g.OH && ow < g.OW;
+        const int64_t ybase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
+                              static_cast<int64_t>(oh) * g.OW + ow;
+        for (int ns = 0; ns < p.n_sub; ++ns) {
+          const int acc = i * p.n_sub + ns;
+          if (!wait_or_abort(bar_acc_full + 8u * acc, it & 1u, p.err, kSiteAccFull, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int co0 = tc.nt * p.n_tile + ns * p.sub_n;
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+          for (int c0 = 0; c0 < p.sub_n; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
+            tmem_wait_ld();
+            if (valid) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int co = co0 + c0 + j;
-            if (co < g.Cout) {
-              float f = __uint_as_float(v[j]);
-              if (bias) f = __fadd_rn(f, DTypeOps<T>::to_f32(bias[co]));
-              y[ybase + static_cast<int64_t>(co) * S] = DTypeOps<T>::from_f32(f);
+              for (int j = 0; j < 16; ++j) {
+                const int co = co0 + c0 + j;
+                if (co < g.Cout) {
+                  float f = __uint_as_float(v[j]);
+                  if (bias) f = __fadd_rn(f, DTypeOps<T>::to_f32(bias[co]));
+                  y[ybase + static_cast<int64_t>(co) * S] = DTypeOps<T>::from_f32(f);
+                }
+              }
             }
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8u * acc);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_acc_empty + 8u * eb);
-      ++acc_ctr;
     }
   } else if (warp >= kWarpXf0) {
-    // ------------------------------------------------------------------ transform
+    // ------------------------------------------------------------ transform
     const int xw = warp - kWarpXf0;
-    const int h = xw >> 2;
-    const int r = (xw & 3) * 32 + lane;
-    const int th = r / p.TW, tw = r % p.TW;
-    const int khw = g.KH * g.KW;
-    const int esz = static_cast<int>(sizeof(T));
-    const int hstride = g.dh * p.w_box;                 // elements between kh taps
-    const int dstride = g.dd * p.h_ext * p.w_box;       // elements between kd taps
-    Nvfp4Global G{0.0f, 0.0f};
-    if (p.quant) G = nvfp4_global(__ldg(p.act_amax));
-    uint32_t slot_base = 0, ast = 0;
+    const int grp = xw / xf_warps_per_group;     // which K slices this warp works on
+    const int lw = xw % xf_warps_per_group;      // 2 warps per subtile
+    const int sub = lw >> 1;
+    const int blk = 2 * (lw & 1) + (lane >> 4);  // 16-column block within the K slice
+    const int rg = lane & 15;                    // 8-row group within the subtile
+    const int lr0 = 8 * rg;
+    const int th = sub * p.TH + lr0 / p.TW;      // row of the tile
+    const int tw0 = lr0 % p.TW;
+    const uint32_t halo_base = base + p.off_halo;
+    const uint32_t tab = base + p.off_tab;
+    const int xf_tid = threadIdx.x - kWarpXf0 * 32;
+
+    // per-CTA table of (scale, 1/scale) for every non-negative E4M3 code
+    float t = 0.0f;
+    {
+      const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f};
+      t = G.t;
+      if (p.quant && xf_tid < 128) {
+        uint32_t h2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
+        const float s8 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+        float s = __fmul_rn(s8, G.g);
+        if (s < 1e-5f) s = 1.0f;
+        float* e = reinterpret_cast<float*>(smem + p.off_tab + xf_tid * 8);
+        e[0] = s;
+        e[1] = __frcp_rn(s);
+      }
+      named_bar_sync(1, kNumXfWarps * 32);
+    }
+
+    int roff[8];
+    uint32_t gs_base = 0;  // global slot counter at the start of the tile
+    uint32_t ga = 0;       // global K-slice counter at the start of the tile
     bool ok = true;
-    for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
-      const TileCoord tc = decode_tile(p, t);
+    for (int64_t tt = blockIdx.x; ok && tt < p.num_tiles; tt += gridDim.x) {
+      const TileCoord tc = decode_tile(p, tt);
       const int w0 = halo_w0(p, tc.ow0);
-      const int thr_off = th * g.sh * p.w_box + tw * g.sw + (tc.ow0 * g.sw - g.pw - w0);
-      int waited = -1, released = 0;
-      for (int s = 0; s < p.ks; ++s) {
-        const uint32_t ea = ast % p.sa, ua = ast / p.sa;
+      const int delta = tc.ow0 * g.sw - g.pw - w0;
+      const int thr_al = th * g.sh * p.w_box + tw0 * g.sw;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) roff[r] = thr_al + r * g.sw + delta;
+      // first K slice of this tile that belongs to this warp's group
+      int s = static_cast<int>((static_cast<uint32_t>(grp) + static_cast<uint32_t>(p.groups) -
+                                ga % static_cast<uint32_t>(p.groups)) % static_cast<uint32_t>(p.groups));
+      for (; s < p.ks; s += p.groups) {
+        const uint32_t gslice = ga + static_cast<uint32_t>(s);
+        const uint32_t ea = gslice % p.sa, ua = gslice / p.sa;
         if (ua > 0 && !wait_or_abort(bar_a_empty + 8u * ea, (ua - 1u) & 1u, p.err, kSiteMmaDone, abort_flag)) {
           ok = false;
           break;
         }
-        const int k_last = min(kBlockK * s + kBlockK - 1, g.K - 1);
-        const int q_need = (k_last / g.taps) / p.c_slot;
-        while (waited < q_need) {
-          ++waited;
-          const uint32_t gs = slot_base + static_cast<uint32_t>(waited);
-          if (!wait_or_abort(bar_halo_full + 8u * (gs % p.ring), (gs / p.ring) & 1u, p.err, kSiteHaloFull,
-                             abort_flag)) {
-            ok = false;
-            break;
-          }
+        for (int q = slot_lo(p, s), qh = slot_hi(p, s); ok && q <= qh; ++q) {
+          const uint32_t gsl = gs_base + static_cast<uint32_t>(q);
+          ok = wait_or_abort(bar_halo_full + 8u * (gsl % p.ring), (gsl / p.ring) & 1u, p.err, kSiteHaloFull,
+                             abort_flag);
         }
         if (!ok) break;
-        uint8_t* a_tile = smem + p.off_a + ea * kATileBytes;
-#pragma unroll 1
-        for (int bb = 0; bb < 2; ++bb) {
-          const int blk = 2 * h + bb;
-          const int kb = kBlockK * s + 16 * blk;
-          int c = kb / g.taps;
-          int rr = kb - c * g.taps;
-          int kd = rr / khw;
-          rr -= kd * khw;
-          int kh = rr / g.KW;
-          int kw = rr - kh * g.KW;
-          float v[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float val = 0.0f;
-            if (kb + j < g.K) {
-              const int q = c / p.c_slot;
-              const uint32_t e = (slot_base + static_cast<uint32_t>(q)) % p.ring;
-              const int off = (c - q * p.c_slot) * p.chan_elems + kd * dstride + kh * hstride + kw * g.dw + thr_off;
-              val = lds_as_f32<T>(smem + p.off_halo + e * p.slot_bytes + off * esz);
-            }
-            v[j] = val;
-            if (++kw == g.KW) {
-              kw = 0;
-              if (++kh == g.KH) {
-                kh = 0;
-                if (++kd == g.KD) { kd = 0; ++c; }
-              }
-            }
-          }
-          if (p.quant) {
-            float bmax = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
-            float scale, inv;
-            nvfp4_block_scale(bmax, G, scale, inv);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) nvfp4_pair(v[2 * i], v[2 * i + 1], inv, scale, v[2 * i], v[2 * i + 1]);
-          }
-          uint32_t w[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-          *reinterpret_cast<uint4*>(a_tile + sw128_offset(r, 2 * blk)) = make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(a_tile + sw128_offset(r, 2 * blk + 1)) = make_uint4(w[4], w[5], w[6], w[7]);
+        const uint32_t a_sub = base + p.off_a + ea * p.a_stage_bytes + static_cast<uint32_t>(sub) * kASubBytes;
+        const int kb = kBlockK * s + 16 * blk;
+        if constexpr (sizeof(T) == 2) {
+          if (p.vec)
+            transform_task_vec<T>(p, a_sub, rg, kb, thr_al, delta, halo_base, gs_base, t, tab);
+          else
+            transform_task_gen<T>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+        } else {
+          transform_task_gen<T>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_a_full + 8u * ea);
-        ++ast;
-        // halo slots below the first one the next slice needs are done
-        const int q_keep = (s + 1 < p.ks) ? ((kBlockK * (s + 1)) / g.taps) / p.c_slot : p.q_slots;
-        while (released < q_keep) {
-          if (lane == 0) mbar_arrive(bar_halo_empty + 8u * ((slot_base + static_cast<uint32_t>(released)) % p.ring));
-          ++released;
-        }
       }
-      slot_base += static_cast<uint32_t>(p.q_slots);
+      if (!ok) break;
+      gs_base += static_cast<uint32_t>(p.q_slots);
+      ga += static_cast<uint32_t>(p.ks);
     }
   }
 
@@ -450,111 +705,150 @@ cudaError_t launch_fast_typed(const FastParams& p, const CUtensorMap& tx, const 
 // result); unset selects the specialised kernel when it applies.
 int kernel_choice() {
   const char* v = getenv("Q3D_KERNEL");
-  if (!v) return 1;
+  if (!v) return 0;
   if (!strcmp(v, "basic")) return 1;
   if (!strcmp(v, "fast")) return 2;
-  return 1;
+  return 0;
 }
 
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
 }  // namespace
+
+// Tiling and pipeline plan of the specialised kernel for one problem (pure
+// host arithmetic).  Returns false when the kernel does not apply.
+static bool plan_fast(const ConvGeom& g, int dtype, FastParams& p, size_t& smem) {
+  const int esz = dtype == 0 ? 4 : 2;
+  const int align = 16 / esz;
+  if ((static_cast<int64_t>(g.W) * esz) % 16 != 0) return false;
+  memset(&p, 0, sizeof(p));
+  p.g = g;
+  p.align = align;
+
+  // output channels per tile: all of Cout up to 512, else tiles of 256
+  int n_ntiles = 1, n_tile = (g.Cout + 15) / 16 * 16;
+  if (n_tile > 512) {
+    n_ntiles = ceil_div(g.Cout, 256);
+    n_tile = (ceil_div(g.Cout, n_ntiles) + 15) / 16 * 16;
+  }
+  const int n_sub = ceil_div(n_tile, 256);
+  const int sub_n = (ceil_div(n_tile, n_sub) + 15) / 16 * 16;
+  n_tile = sub_n * n_sub;
+  p.n_tile = n_tile; p.n_ntiles = n_ntiles; p.n_sub = n_sub; p.sub_n = sub_n;
+  const int max_mt = std::min(4, 512 / n_tile);
+
+  // tile shape: subtile TH x TW = 128, n_mt subtiles stacked along oh
+  const int kd_ext = (g.KD - 1) * g.dd + 1;
+  double best = 1e30;
+  int bTW = 0, bMT = 0;
+  for (int mt = max_mt; mt >= 1; mt /= 2) {
+    if (mt == 3) continue;
+    for (int TW = 128; TW >= 8; TW /= 2) {
+      const int TH = 128 / TW, rows = TH * mt;
+      const int h_ext = (rows - 1) * g.sh + (g.KH - 1) * g.dh + 1;
+      const int w_ext = (TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
+      const int w_box = (w_ext + 2 * (align - 1)) / align * align;
+      if (w_box > 256 || h_ext > 256 || kd_ext > 256) continue;
+      const double waste = (double)(ceil_div(g.OH, rows) * rows) * (ceil_div(g.OW, TW) * TW) / ((double)g.OH * g.OW);
+      const double halo = (double)h_ext * w_box / (128.0 * mt);
+      // fewer subtiles per tile cost weight bandwidth: about 8% per halving
+      const double score = waste * (1.0 + 0.01 * halo) * (1.0 + 0.08 * (mt >= 4 ? 0 : mt == 2 ? 1 : 2));
+      if (score < best - 1e-9) { best = score; bTW = TW; bMT = mt; }
+    }
+  }
+  if (bTW == 0) return false;
+  p.TW = bTW; p.TH = 128 / bTW; p.n_mt = bMT;
+  p.groups = 4 / bMT;
+  p.n_owb = ceil_div(g.OW, p.TW);
+  p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
+  p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;
+  const int w_ext = (p.TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
+  p.w_box = (w_ext + 2 * (align - 1)) / align * align;
+  p.kd_ext = kd_ext;
+  p.chan_elems = p.kd_ext * p.h_ext * p.w_box;
+  p.ks = ceil_div(g.K, kBlockK);
+  p.num_tiles = static_cast<int64_t>(g.N) * g.OD * p.n_ohb * p.n_owb * n_ntiles;
+  p.a_stage_bytes = static_cast<uint32_t>(p.n_mt) * kASubBytes;
+  p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
+  p.vec = (esz == 2 && g.sw == 1) ? 1 : 0;
+  int tmem = 32;
+  while (tmem < p.n_mt * n_tile) tmem <<= 1;
+  p.tmem_cols = tmem;
+
+  const int chan_bytes = p.chan_elems * esz;
+  // Halo ring: the MMA thread hands a slot back once every slice that reads
+  // it is complete, while the transform may run up to sa slices ahead of the
+  // MMA, so the ring must hold the slots of sa consecutive slices (+2 so the
+  // producer can run ahead).  A stages must number at least the transform
+  // groups (each group owns every groups-th slice), or a group could wait on
+  // an A-stage barrier two phases ahead.
+  for (int target = 10240; target >= 1; target = (target > chan_bytes ? target / 2 : 0)) {
+    p.c_slot = std::max(1, std::min(std::min(256, g.C), target / chan_bytes));
+    p.q_slots = ceil_div(g.C, p.c_slot);
+    p.slot_tx = static_cast<uint32_t>(p.c_slot) * chan_bytes;
+    p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
+    auto span_of = [&](int w) {
+      int sp = 1;
+      for (int s0 = 0; s0 < p.ks; ++s0) {
+        const int lo = ((kBlockK * s0) / g.taps) / p.c_slot;
+        const int hi = (std::min(kBlockK * (s0 + w) - 1, g.K - 1) / g.taps) / p.c_slot;
+        sp = std::max(sp, hi - lo + 1);
+      }
+      return sp;
+    };
+    auto total = [&](int a, int b, int r) {
+      const int nbar = 2 * r + 2 * b + 2 * a + 2 * kMaxAcc + 1;
+      return 1024 + a * static_cast<int>(p.a_stage_bytes) + b * static_cast<int>(p.b_stage_bytes) +
+             r * static_cast<int>(p.slot_bytes) + 64 /* pad after the halo ring */ + 1024 /* scale table */ +
+             nbar * 8 + 16;
+    };
+    for (int a = 4; a >= 2; --a) {
+      if (a < p.groups) continue;
+      for (int b = 8; b >= 2; --b) {
+        const int r = span_of(a) + 2;
+        if (total(a, b, r) <= kMaxSmem) {
+          p.sa = a; p.sb = b; p.ring = r;
+          p.off_a = 0;
+          p.off_b = p.off_a + a * p.a_stage_bytes;
+          p.off_halo = p.off_b + b * p.b_stage_bytes;
+          p.off_tab = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
+          p.off_bar = p.off_tab + 1024u;
+          smem = static_cast<size_t>(total(a, b, r));
+          // at most 512 / tmem_cols CTAs may share an SM, so tcgen05.alloc never waits
+          const size_t max_ctas = 512 / static_cast<size_t>(p.tmem_cols);
+          const size_t min_smem = 233472 / (max_ctas + 1) + 1;
+          if (max_ctas < 4 && smem + 1024 < min_smem) smem = min_smem - 1024;
+          return true;
+        }
+      }
+    }
+    if (p.c_slot == 1) break;
+  }
+  return false;
+}
+
+bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
+  FastParams p;
+  size_t smem = 0;
+  const bool ok = plan_fast(g, dtype, p, smem);
+  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, p.groups, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
+                       p.c_slot, p.q_slots, p.ring, p.sa, p.sb, p.tmem_cols, static_cast<int64_t>(smem),
+                       p.n_ohb, p.n_owb, p.vec, p.w_box, p.h_ext, p.kd_ext};
+  const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
+  for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
+  return ok;
+}
 
 cudaError_t launch_conv3d_fast(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
                                bool* handled) {
   *handled = false;
   if (kernel_choice() == 1) return cudaSuccess;
   const int esz = L.dtype == 0 ? 4 : 2;
-  const int align = 16 / esz;
-  // TMA needs 16-byte aligned base and strides for x
-  if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0 || (static_cast<int64_t>(g.W) * esz) % 16 != 0) return cudaSuccess;
-  if (g.Cout > 512 * 64) return cudaSuccess;
-
+  if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   FastParams p;
-  memset(&p, 0, sizeof(p));
-  p.g = g;
+  size_t smem = 0;
+  if (!plan_fast(g, L.dtype, p, smem)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
-  p.align_elems = align;
-
-  // output channels per tile: all of Cout up to 512, else tiles of 256
-  int n_ntiles = 1, n_tile = (g.Cout + 15) / 16 * 16;
-  if (n_tile > 512) {
-    n_ntiles = (g.Cout + 255) / 256;
-    n_tile = ((g.Cout + n_ntiles - 1) / n_ntiles + 15) / 16 * 16;
-  }
-  const int n_sub = (n_tile + 255) / 256;
-  const int sub_n = ((n_tile / n_sub) + 15) / 16 * 16;
-  n_tile = sub_n * n_sub;
-  p.n_tile = n_tile; p.n_ntiles = n_ntiles; p.n_sub = n_sub; p.sub_n = sub_n;
-  p.n_acc = (2 * n_tile <= 512) ? 2 : 1;
-  int tmem = 32;
-  while (tmem < p.n_acc * n_tile) tmem <<= 1;
-  p.tmem_cols = tmem;
-
-  // spatial tile: TH x TW = 128 with the least padding waste
-  const int kd_ext = (g.KD - 1) * g.dd + 1;
-  double best = 1e30;
-  int bTW = 0;
-  for (int TW = 128; TW >= 8; TW /= 2) {
-    const int TH = 128 / TW;
-    const int h_ext = (TH - 1) * g.sh + (g.KH - 1) * g.dh + 1;
-    const int w_ext = (TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
-    const int w_box = (w_ext + align - 1 + align - 1) / align * align;  // worst-case start misalignment
-    if (w_box > 256 || h_ext > 256 || kd_ext > 256) continue;
-    const double waste = (double)((g.OH + TH - 1) / TH * TH) * ((g.OW + TW - 1) / TW * TW) / ((double)g.OH * g.OW);
-    const double halo = (double)h_ext * w_box / 128.0;
-    const double score = waste * (1.0 + 0.02 * halo);
-    if (score < best - 1e-9) { best = score; bTW = TW; }
-  }
-  if (bTW == 0) return cudaSuccess;
-  p.TW = bTW; p.TH = 128 / bTW;
-  p.n_owb = (g.OW + p.TW - 1) / p.TW;
-  p.n_ohb = (g.OH + p.TH - 1) / p.TH;
-  p.h_ext = (p.TH - 1) * g.sh + (g.KH - 1) * g.dh + 1;
-  const int w_ext = (p.TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
-  p.w_box = (w_ext + 2 * (align - 1)) / align * align;
-  p.kd_ext = kd_ext;
-  p.chan_elems = p.kd_ext * p.h_ext * p.w_box;
-  const int chan_bytes = p.chan_elems * esz;
-  p.c_slot = 8192 / chan_bytes;
-  if (p.c_slot < 1) p.c_slot = 1;
-  if (p.c_slot > 256) p.c_slot = 256;
-  if (p.c_slot > g.C) p.c_slot = g.C;
-  p.q_slots = (g.C + p.c_slot - 1) / p.c_slot;
-  p.slot_tx = static_cast<uint32_t>(p.c_slot) * chan_bytes;
-  p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
-  p.ks = (g.K + kBlockK - 1) / kBlockK;
-  p.num_tiles = static_cast<int64_t>(g.N) * g.OD * p.n_ohb * p.n_owb * n_ntiles;
-  p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
-
-  // widest span of halo slots one K slice needs at once
-  int span = 1;
-  for (int s0 = 0; s0 < p.ks; ++s0) {
-    const int qlo = ((kBlockK * s0) / g.taps) / p.c_slot;
-    const int qhi = ((std::min(kBlockK * s0 + kBlockK - 1, g.K - 1)) / g.taps) / p.c_slot;
-    span = std::max(span, qhi - qlo + 1);
-  }
-  // pipeline depths under the shared-memory budget
-  int sa = 4, sb = 4, ring = std::max(span + 3, 4);
-  auto total = [&](int a, int b, int r) {
-    const int nbar = 2 * r + 2 * b + 2 * a + 4 + 1;
-    return 1024 + a * static_cast<int>(kATileBytes) + b * static_cast<int>(p.b_stage_bytes) +
-           r * static_cast<int>(p.slot_bytes) + nbar * 8 + 16;
-  };
-  while (total(sa, sb, ring) > kMaxSmem) {
-    if (sb > 2) --sb;
-    else if (ring > span + 1) --ring;
-    else if (sa > 2) --sa;
-    else return cudaSuccess;  // does not fit: use the general kernel
-  }
-  p.sa = sa; p.sb = sb; p.ring = ring;
-  p.off_a = 0;
-  p.off_b = p.off_a + sa * kATileBytes;
-  p.off_halo = p.off_b + sb * p.b_stage_bytes;
-  p.off_bar = (p.off_halo + ring * p.slot_bytes + 7u) / 8u * 8u;
-  size_t smem = static_cast<size_t>(total(sa, sb, ring));
-  // at most 512 / tmem_cols CTAs may share an SM, so tcgen05.alloc never waits
-  const size_t max_ctas = 512 / static_cast<size_t>(p.tmem_cols);
-  const size_t min_smem = 233472 / (max_ctas + 1) + 1;
-  if (max_ctas < 4 && smem + 1024 < min_smem) smem = min_smem - 1024;
 
   EncodeTiledFn encode = get_encode_tiled();
   if (!encode) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }

@@ -16,7 +16,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/q3d.h"
+#include "q3d.h"
 #include "q3d_internal.h"
 
 namespace q3d {
@@ -294,4 +294,36 @@ q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* 
   return Q3D_OK;
 }
 
+q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                         const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
+                         int32_t* plan, int32_t plan_len) {
+  if (!x_shape || !w_shape || !stride || !pad_lo || !pad_hi || !dil || !plan)
+    return fail(Q3D_ERR_NULLPTR, "NULL pointer");
+  if (!dtype_ok(dtype)) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "dtype");
+  q3d::ConvGeom g;
+  const int64_t k_dims[3] = {w_shape[2], w_shape[3], w_shape[4]};
+  int64_t o_dims[3];
+  for (int i = 0; i < 3; ++i) {
+    if (stride[i] < 1 || dil[i] < 1 || pad_lo[i] < 0 || pad_hi[i] < 0 || k_dims[i] < 1)
+      return fail(Q3D_ERR_INVALID_ARG, "bad stride/pad/dilation/kernel");
+    const int64_t span = x_shape[2 + i] + pad_lo[i] + pad_hi[i] - static_cast<int64_t>(dil[i]) * (k_dims[i] - 1) - 1;
+    if (span < 0) return fail(Q3D_ERR_INVALID_ARG, "empty output");
+    o_dims[i] = span / stride[i] + 1;
+  }
+  if (w_shape[1] != x_shape[1]) return fail(Q3D_ERR_INVALID_ARG, "groups != 1");
+  g.N = (int32_t)x_shape[0]; g.C = (int32_t)x_shape[1]; g.D = (int32_t)x_shape[2]; g.H = (int32_t)x_shape[3];
+  g.W = (int32_t)x_shape[4];
+  g.Cout = (int32_t)w_shape[0]; g.KD = (int32_t)k_dims[0]; g.KH = (int32_t)k_dims[1]; g.KW = (int32_t)k_dims[2];
+  g.sd = stride[0]; g.sh = stride[1]; g.sw = stride[2];
+  g.pd = pad_lo[0]; g.ph = pad_lo[1]; g.pw = pad_lo[2];
+  g.dd = dil[0]; g.dh = dil[1]; g.dw = dil[2];
+  g.OD = (int32_t)o_dims[0]; g.OH = (int32_t)o_dims[1]; g.OW = (int32_t)o_dims[2];
+  g.M = x_shape[0] * o_dims[0] * o_dims[1] * o_dims[2];
+  g.K = (int32_t)(x_shape[1] * k_dims[0] * k_dims[1] * k_dims[2]);
+  g.taps = (int32_t)(k_dims[0] * k_dims[1] * k_dims[2]);
+  q3d::plan_conv3d_fast(g, dtype, plan, plan_len);
+  return Q3D_OK;
+}
+
 }  // extern "C"
+

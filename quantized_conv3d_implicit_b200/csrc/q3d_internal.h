@@ -63,6 +63,10 @@ cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, flo
 cudaError_t launch_stage_weights(const void* w, int dtype, int32_t Cout, int32_t K, int64_t ld, void* w_bf16,
                                  cudaStream_t s);
 
+// Plan of the specialised kernel (test hook): out[0] = applicable, then the
+// tiling and pipeline parameters in a fixed order (see q3d.h).
+bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out);
+
 // The implicit-GEMM convolution; returns a CUDA error or cudaSuccess, and a
 // short reason in *why when it rejects the problem before launching.
 cudaError_t launch_conv3d_igemm(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why);

@@ -182,6 +182,33 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32(uint32_t M, uint32_t 
          | ((M >> 4) << 24);  // M / 16
 }
 
+// Shared-memory matrix descriptor for an MN-major operand in the canonical
+// 128-byte-swizzled layout: atoms of 64 MN elements (one 128-byte row) x 8 K
+// rows (1024 bytes); in K-row r of an atom, 16-byte chunk j (8 MN elements)
+// is stored at chunk (j ^ (r & 7)).  Atoms adjacent along MN are lbo bytes
+// apart, atoms adjacent along K are sbo bytes apart.  Atoms start on
+// 1024-byte boundaries.
+__device__ __forceinline__ uint64_t umma_desc_mnmajor_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// kind::f16 instruction descriptor with an MN-major A operand and a K-major
+// B operand (BF16 x BF16 -> FP32, M x N).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_amn(uint32_t M, uint32_t N) {
+  return umma_idesc_bf16_f32(M, N) | (1u << 15);
+}
+
+// Named barrier over `nthreads` threads (a multiple of 32) with id 1..15.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a
 // 128B-swizzled K-major tile (rows of 128 bytes).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

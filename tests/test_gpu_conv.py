@@ -18,6 +18,17 @@ from _parity import assert_conv_close, bits, to_np_f32
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=["auto", "basic"])
+def kernel(request, monkeypatch):
+    """Run a test with the library's default kernel choice and again with the
+    general-purpose kernel forced (both must meet the same bar)."""
+    if request.param == "basic":
+        monkeypatch.setenv("Q3D_KERNEL", "basic")
+    else:
+        monkeypatch.delenv("Q3D_KERNEL", raising=False)
+    return request.param
+
+
 def _run(inp, stride, plo, phi, dil, quant):
     x, w, b, amax = inp["x"], inp["w"], inp["bias"], inp["act_amax"]
     pad6 = (plo[0], phi[0], plo[1], phi[1], plo[2], phi[2])
@@ -51,7 +62,7 @@ SHAPES = [
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("quant", [False, True])
 @pytest.mark.parametrize("case", range(len(SHAPES)))
-def test_conv_small_shapes(cuda_ok, case, quant, dtype):
+def test_conv_small_shapes(cuda_ok, kernel, case, quant, dtype):
     xs, cout, k, s, plo, phi, d = SHAPES[case]
     inp = workloads.random_conv_inputs(100 + case, xs, cout, k, dtype=dtype, bias=(case % 2 == 0), device="cuda")
     y = _run(inp, s, plo, phi, d, quant)
@@ -61,7 +72,7 @@ def test_conv_small_shapes(cuda_ok, case, quant, dtype):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("quant", [False, True])
-def test_identity_weight_readout_is_bit_exact(cuda_ok, quant, dtype):
+def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, quant, dtype):
     # one-hot weights: y[:, co] = A[:, k(co)], a single nonzero product per
     # output, so the FP32 accumulator holds the BF16 operand exactly and the
     # whole im2col row (quantised or not) is reproduced bit for bit
@@ -85,7 +96,7 @@ def test_identity_weight_readout_is_bit_exact(cuda_ok, quant, dtype):
         assert np.array_equal(bits(y), ref_bits), start
 
 
-def test_determinism(cuda_ok):
+def test_determinism(cuda_ok, kernel):
     inp = workloads.random_conv_inputs(5, (1, 24, 4, 20, 24), 48, (3, 3, 3), dtype=torch.bfloat16, device="cuda")
     y1 = _run(inp, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), True)
     y2 = _run(inp, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), True)

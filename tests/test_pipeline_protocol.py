@@ -1,0 +1,236 @@
+"""Host-side check of the specialised kernel's pipeline protocol.
+
+The sm_100a kernel synchronises its roles (halo producer, weight producer,
+MMA issuer, epilogue, transform groups) with mbarriers whose waits test a
+phase parity.  This test replays that protocol on the CPU for the plans the
+library's own planner (q3d_plan_conv, host code) chooses, and checks that
+  - no interleaving explored here deadlocks (every role finishes), and
+  - every parity wait that succeeds does so for the phase it means, i.e. the
+    barrier has completed exactly that phase and not one two phases earlier
+    (parity aliasing),
+together with the plan invariants the kernel relies on.  Roles are modelled
+as generators yielding ("wait", barrier, phase) or ("arrive", barrier);
+TMA and tcgen05.commit completions are arrivals issued where the kernel
+issues them.  Several schedules (round-robin, reversed, seeded random) are
+explored.
+"""
+import random
+
+import pytest
+import torch
+
+from quantized_conv3d_implicit_b200 import api, workloads
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.phase = count, count, 0
+
+    def arrive(self):
+        self.pending -= 1
+        if self.pending == 0:
+            self.phase += 1
+            self.pending = self.count
+
+    def parity_done(self, phase):
+        return (self.phase & 1) != (phase & 1)
+
+
+def roles(plan, K, taps, ntiles):
+    bars = {}
+
+    def bar(name, i, count):
+        key = (name, i)
+        if key not in bars:
+            bars[key] = Bar(count)
+        return bars[key]
+
+    ks, q_slots, ring, sa, sb, G = (plan[k] for k in ("ks", "q_slots", "ring", "sa", "sb", "groups"))
+    n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
+    wpg = 8 // G
+
+    def slot_lo(s):
+        return ((64 * s) // taps) // c_slot
+
+    def slot_hi(s):
+        return (min(64 * s + 63, K - 1) // taps) // c_slot
+
+    def halo_producer():
+        gs = 0
+        for _ in range(ntiles):
+            for _q in range(q_slots):
+                e, u = gs % ring, gs // ring
+                if u > 0:
+                    yield ("wait", bar("halo_empty", e, 1), u - 1)
+                yield ("arrive", bar("halo_full", e, 1))
+                gs += 1
+
+    def weight_producer():
+        gb = 0
+        for _ in range(ntiles):
+            for _s in range(ks):
+                e, u = gb % sb, gb // sb
+                if u > 0:
+                    yield ("wait", bar("b_empty", e, 1), u - 1)
+                yield ("arrive", bar("b_full", e, 1))
+                gb += 1
+
+    def mma():
+        ga = gb = gs_base = 0
+        for it in range(ntiles):
+            released = 0
+            for s in range(ks):
+                ea, eb = ga % sa, gb % sb
+                yield ("wait", bar("a_full", ea, wpg), ga // sa)
+                keep = slot_lo(s + 1) if s + 1 < ks else q_slots
+                while released < keep:
+                    yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
+                    released += 1
+                yield ("wait", bar("b_full", eb, 1), gb // sb)
+                for i in range(n_mt):
+                    for ns in range(n_sub):
+                        acc = i * n_sub + ns
+                        if s == 0 and it > 0:
+                            yield ("wait", bar("acc_empty", acc, 4), it - 1)
+                        if s == ks - 1:
+                            yield ("arrive", bar("acc_full", acc, 1))
+                yield ("arrive", bar("a_empty", ea, 1))
+                yield ("arrive", bar("b_empty", eb, 1))
+                ga += 1
+                gb += 1
+            gs_base += q_slots
+
+    def epilogue():
+        for it in range(ntiles):
+            for i in range(n_mt):
+                for ns in range(n_sub):
+                    acc = i * n_sub + ns
+                    yield ("wait", bar("acc_full", acc, 1), it)
+                    yield ("arrive", bar("acc_empty", acc, 4))
+
+    def transform(w):
+        grp = w // wpg
+        ga = gs_base = 0
+        for _ in range(ntiles):
+            s = (grp + G - ga % G) % G
+            while s < ks:
+                gsl = ga + s
+                ea, ua = gsl % sa, gsl // sa
+                if ua > 0:
+                    yield ("wait", bar("a_empty", ea, 1), ua - 1)
+                for q in range(slot_lo(s), slot_hi(s) + 1):
+                    g = gs_base + q
+                    yield ("wait", bar("halo_full", g % ring, 1), g // ring)
+                yield ("arrive", bar("a_full", ea, wpg))
+                s += G
+            ga += ks
+            gs_base += q_slots
+
+    r = {"halo": halo_producer(), "weights": weight_producer(), "mma": mma()}
+    for w in range(4):
+        r[f"epilogue{w}"] = epilogue()
+    for w in range(8):
+        r[f"transform{w}"] = transform(w)
+    return r
+
+
+def run(plan, K, taps, ntiles, order="rr", seed=0):
+    rs = roles(plan, K, taps, ntiles)
+    names = list(rs)
+    cur = {k: None for k in names}
+    done = set()
+    rng = random.Random(seed)
+    while len(done) < len(names):
+        progress = False
+        seq = names if order == "rr" else names[::-1] if order == "rev" else rng.sample(names, len(names))
+        for k in seq:
+            if k in done:
+                continue
+            steps = 0
+            while order != "random" or steps < rng.randint(1, 4):
+                steps += 1
+                if cur[k] is None:
+                    try:
+                        cur[k] = next(rs[k])
+                    except StopIteration:
+                        done.add(k)
+                        progress = True
+                        break
+                op = cur[k]
+                if op[0] == "arrive":
+                    op[1].arrive()
+                    cur[k] = None
+                    progress = True
+                    continue
+                b, phase = op[1], op[2]
+                if b.parity_done(phase):
+                    assert b.phase == phase + 1, f"parity aliasing in {k}: waits phase {phase}, barrier at {b.phase}"
+                    cur[k] = None
+                    progress = True
+                    continue
+                break
+        assert progress, "deadlock: " + ", ".join(k for k in names if k not in done)
+
+
+def _plan(wl_or_args):
+    if isinstance(wl_or_args, workloads.Workload):
+        wl = wl_or_args
+        pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+        w_shape = (wl.cout, wl.x_shape[1]) + tuple(wl.kernel)
+        return api.plan_conv(wl.x_shape, w_shape, wl.stride, pad6, wl.dil, wl.dtype), wl.k_gemm, \
+            wl.kernel[0] * wl.kernel[1] * wl.kernel[2]
+    xs, ws, s, pad6, d, dt = wl_or_args
+    return api.plan_conv(xs, ws, s, pad6, d, dt), ws[1] * ws[2] * ws[3] * ws[4], ws[2] * ws[3] * ws[4]
+
+
+def _check_invariants(p):
+    assert p["sa"] >= p["groups"]
+    assert p["n_mt"] * p["groups"] == 4
+    assert p["n_mt"] * p["n_tile"] <= p["tmem_cols"] <= 512
+    assert p["n_sub"] * p["sub_n"] == p["n_tile"] and p["sub_n"] % 16 == 0 and 16 <= p["sub_n"] <= 256
+    assert p["smem"] <= 232448
+    assert p["TH"] * p["TW"] == 128
+    assert p["w_box"] <= 256 and p["h_ext"] <= 256 and p["kd_ext"] <= 256
+
+
+@pytest.mark.parametrize("name", sorted(workloads.WORKLOADS))
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_workload_plans_are_deadlock_and_alias_free(name, order):
+    plan, K, taps = _plan(workloads.WORKLOADS[name])
+    assert plan["applicable"] == 1
+    _check_invariants(plan)
+    run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)))
+
+
+def test_random_shapes():
+    rng = random.Random(7)
+    checked = 0
+    for _ in range(60):
+        k = rng.choice([(1, 1, 1), (3, 3, 3), (1, 3, 3), (5, 5, 5), (3, 1, 1)])
+        cin = rng.choice([1, 3, 8, 16, 37, 64, 96, 192, 256])
+        cout = rng.choice([1, 8, 16, 40, 96, 100, 192, 256, 300, 384, 512, 640, 1024])
+        xs = (rng.choice([1, 2]), cin, rng.randint(k[0], 9), rng.randint(k[1], 40), 8 * rng.randint(1, 30))
+        s = (1, rng.choice([1, 1, 2]), rng.choice([1, 1, 2]))
+        d = (1, rng.choice([1, 2]), rng.choice([1, 2]))
+        pad6 = tuple(rng.randint(0, 2) for _ in range(6))
+        ws = (cout, cin) + k
+        dt = rng.choice([torch.bfloat16, torch.float16, torch.float32])
+        try:
+            plan, K, taps = _plan((xs, ws, s, pad6, d, dt))
+        except api.Q3DError:
+            continue  # empty output: not a valid convolution
+        if not plan["applicable"]:
+            continue
+        _check_invariants(plan)
+        run(plan, K, taps, ntiles=2, order="random", seed=checked)
+        checked += 1
+    assert checked >= 30
+
+
+def test_sim_detects_aliasing_when_stages_fewer_than_groups():
+    # the checker itself: with fewer A stages than transform groups a group can
+    # pass a wait two phases early, which the model must flag
+    plan, K, taps = _plan(workloads.WORKLOADS["wan_mid_384_bf16"])
+    bad = dict(plan, sa=3)
+    with pytest.raises(AssertionError):
+        run(bad, K, taps, ntiles=3)
