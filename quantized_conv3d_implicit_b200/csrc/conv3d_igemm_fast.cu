@@ -124,15 +124,13 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, uns
                                               volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kQ3dWaitTimeoutNs) {
-        if (err) atomicOr(err, site);
-        *abort_flag = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kQ3dSleepHintNs)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kQ3dWaitTimeoutNs) {
+      if (err) atomicOr(err, site);
+      *abort_flag = 1;
+      return false;
     }
   }
 }
@@ -266,67 +264,147 @@ __device__ __forceinline__ void row_scales(float bmax0, float bmax1, float t, ui
   s1 = e1.x; i1 = e1.y;
 }
 
-// MN-major swizzled position of 8 rows (row group rg) x column kk of a
-// subtile's K slice: atom (kk/8, rg/8) of 1 KB, K-row kk%8, chunk rg%8.
-__device__ __forceinline__ uint32_t a_chunk_offset(int rg, int kk) {
+// MN-major swizzled position of the 16-byte chunk holding 8 rows (chunk
+// index rg8 within the subtile) of column kk of a subtile's K slice: atom
+// (kk/8, rg8/8) of 1 KB, K-row kk%8, chunk rg8%8 stored at (rg8 ^ kk) % 8.
+__device__ __forceinline__ uint32_t a_chunk_offset(int rg8, int kk) {
   const int kr = kk & 7;
-  return static_cast<uint32_t>(((kk >> 3) * 2 + (rg >> 3)) * 1024 + kr * 128 + (((rg & 7) ^ kr) << 4));
+  return static_cast<uint32_t>(((kk >> 3) * 2 + (rg8 >> 3)) * 1024 + kr * 128 + (((rg8 & 7) ^ kr) << 4));
+}
+
+__device__ __forceinline__ void lds128(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
+}
+__device__ __forceinline__ void lds64(uint32_t addr, uint32_t& a, uint32_t& b) {
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(addr));
+}
+__device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
+  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
+}
+
+// Read P consecutive 16-bit elements starting f elements (0 <= f < P) past a
+// (P*2)-byte aligned shared address, as P/2 packed words.  f is the same for
+// every lane of the warp, so the case split does not diverge.
+template <int P>
+__device__ __forceinline__ void load_rows(uint32_t addr, int f, uint32_t (&out)[P / 2]);
+
+template <>
+__device__ __forceinline__ void load_rows<8>(uint32_t addr, int f, uint32_t (&out)[4]) {
+  uint32_t w[8];
+  lds128(addr, w[0], w[1], w[2], w[3]);
+  if (f == 0) {
+    out[0] = w[0]; out[1] = w[1]; out[2] = w[2]; out[3] = w[3];
+    return;
+  }
+  lds128(addr + 16, w[4], w[5], w[6], w[7]);
+  const uint32_t sel = (f & 1) ? 0x5432u : 0x3210u;
+  switch (f >> 1) {
+    case 0:
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = __byte_perm(w[j], w[j + 1], sel);
+      break;
+    case 1:
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = __byte_perm(w[j + 1], w[j + 2], sel);
+      break;
+    case 2:
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = __byte_perm(w[j + 2], w[j + 3], sel);
+      break;
+    default:
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out[j] = __byte_perm(w[j + 3], w[j + 4], sel);
+      break;
+  }
+}
+
+template <>
+__device__ __forceinline__ void load_rows<4>(uint32_t addr, int f, uint32_t (&out)[2]) {
+  uint32_t w[4];
+  lds64(addr, w[0], w[1]);
+  if (f == 0) {
+    out[0] = w[0]; out[1] = w[1];
+    return;
+  }
+  lds64(addr + 8, w[2], w[3]);
+  const uint32_t sel = (f & 1) ? 0x5432u : 0x3210u;
+  if (f >> 1) {
+    out[0] = __byte_perm(w[1], w[2], sel);
+    out[1] = __byte_perm(w[2], w[3], sel);
+  } else {
+    out[0] = __byte_perm(w[0], w[1], sel);
+    out[1] = __byte_perm(w[1], w[2], sel);
+  }
+}
+
+// Store P rows (P/2 packed words) of column kk: a whole 16-byte chunk for
+// P = 8, half of one for P = 4 (rg = row group of P rows).
+template <int P>
+__device__ __forceinline__ void store_rows(uint32_t a_sub, int rg, int kk, const uint32_t (&w)[P / 2]) {
+  if constexpr (P == 8) {
+    sts128(a_sub + a_chunk_offset(rg, kk), w[0], w[1], w[2], w[3]);
+  } else {
+    sts64(a_sub + a_chunk_offset(rg >> 1, kk) + 8u * static_cast<uint32_t>(rg & 1), w[0], w[1]);
+  }
 }
 
 // ---------------------------------------------------------------------------
-// transform: one task = 8 rows (row group rg of subtile i) x 16 columns
+// transform: one task = P rows (row group rg of one subtile) x 16 columns
 // ---------------------------------------------------------------------------
-template <typename T>
-__device__ __forceinline__ void transform_task_vec(const FastParams& p, uint32_t a_sub, int rg, int kb, int thr_al,
-                                                  int delta, uint32_t halo_base, uint32_t slot_base,
-                                                  const float t, uint32_t tab) {
-  // 16 columns x 4 words (pairs of rows (2j, 2j+1))
-  uint32_t d[16][4];
+template <typename T, int P>
+__device__ __forceinline__ void transform_task_vec(const FastParams& p, uint32_t a_sub, int rg, int kb,
+                                                  uint32_t thr_addr, int delta, uint32_t halo_base,
+                                                  uint32_t slot_base, const float t, uint32_t tab) {
+  constexpr int NW = P / 2;
+  uint32_t d[16][NW];
   TapWalker wk;
   wk.init(p, kb, halo_base, slot_base);
 #pragma unroll
   for (int kk = 0; kk < 16; ++kk) {
     if (kb + kk < p.g.K) {
-      const int e = thr_al + wk.u + delta;
-      const uint32_t addr = wk.slot_addr + static_cast<uint32_t>(e & ~1) * 2u;
-      const uint32_t sel = (e & 1) ? 0x5432u : 0x3210u;
-      const uint32_t w0 = lds32(addr), w1 = lds32(addr + 4), w2 = lds32(addr + 8), w3 = lds32(addr + 12),
-                     w4 = lds32(addr + 16);
-      d[kk][0] = __byte_perm(w0, w1, sel);
-      d[kk][1] = __byte_perm(w1, w2, sel);
-      d[kk][2] = __byte_perm(w2, w3, sel);
-      d[kk][3] = __byte_perm(w3, w4, sel);
+      const int e = wk.u + delta;           // warp-uniform element offset
+      const int f = e & (P - 1);
+      uint32_t out[NW];
+      load_rows<P>(wk.slot_addr + thr_addr + static_cast<uint32_t>(e - f) * 2u, f, out);
+#pragma unroll
+      for (int j = 0; j < NW; ++j) d[kk][j] = out[j];
     } else {
-      d[kk][0] = d[kk][1] = d[kk][2] = d[kk][3] = 0u;
+#pragma unroll
+      for (int j = 0; j < NW; ++j) d[kk][j] = 0u;
     }
     if (kk < 15) wk.step(p, halo_base, slot_base);
   }
+  const int kl = kb & (kBlockK - 1);
   if (p.quant) {
-    uint32_t mx[4];
+    uint32_t mx[NW];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < NW; ++j) {
       mx[j] = Pair16<T>::maxabs(d[0][j], d[1][j]);
 #pragma unroll
       for (int kk = 2; kk < 16; ++kk) mx[j] = Pair16<T>::maxabs(mx[j], d[kk][j]);
     }
-    float sc[8], iv[8];
+    float sc[P], iv[P];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NW; ++j)
       row_scales(Pair16<T>::abs_lo(mx[j]), Pair16<T>::abs_hi(mx[j]), t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1],
                  iv[2 * j + 1]);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
+      uint32_t w[NW];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        d[kk][j] = quant_pair_bf16x2(Pair16<T>::lo(d[kk][j]), Pair16<T>::hi(d[kk][j]), iv[2 * j], iv[2 * j + 1],
-                                     sc[2 * j], sc[2 * j + 1]);
-      sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), d[kk][0], d[kk][1], d[kk][2], d[kk][3]);
+      for (int j = 0; j < NW; ++j)
+        w[j] = quant_pair_bf16x2(Pair16<T>::lo(d[kk][j]), Pair16<T>::hi(d[kk][j]), iv[2 * j], iv[2 * j + 1],
+                                 sc[2 * j], sc[2 * j + 1]);
+      store_rows<P>(a_sub, rg, kl + kk, w);
     }
   } else {
 #pragma unroll
-    for (int kk = 0; kk < 16; ++kk)
-      sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), Pair16<T>::to_bf16x2(d[kk][0]),
-             Pair16<T>::to_bf16x2(d[kk][1]), Pair16<T>::to_bf16x2(d[kk][2]), Pair16<T>::to_bf16x2(d[kk][3]));
+    for (int kk = 0; kk < 16; ++kk) {
+      uint32_t w[NW];
+#pragma unroll
+      for (int j = 0; j < NW; ++j) w[j] = Pair16<T>::to_bf16x2(d[kk][j]);
+      store_rows<P>(a_sub, rg, kl + kk, w);
+    }
   }
 }
 
@@ -343,45 +421,47 @@ __device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t addr) { return
 
 // General path (any W stride, any dtype): element loads, two passes (block
 // maxima, then quantisation) so only one column is held at a time.
-template <typename T>
+template <typename T, int P>
 __device__ __forceinline__ void transform_task_gen(const FastParams& p, uint32_t a_sub, int rg, int kb,
                                                   const int (&roff)[8], uint32_t halo_base, uint32_t slot_base,
                                                   const float t, uint32_t tab) {
   constexpr uint32_t esz = sizeof(T);
-  float sc[8], iv[8];
+  constexpr int NW = P / 2;
+  float sc[P], iv[P];
   if (p.quant) {
-    float bm[8];
+    float bm[P];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) bm[r] = 0.0f;
+    for (int r = 0; r < P; ++r) bm[r] = 0.0f;
     TapWalker wk;
     wk.init(p, kb, halo_base, slot_base);
 #pragma unroll 1
     for (int kk = 0; kk < 16; ++kk) {
       if (kb + kk < p.g.K) {
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int r = 0; r < P; ++r)
           bm[r] = fmaxf(bm[r], fabsf(lds_elem<T>(wk.slot_addr + static_cast<uint32_t>(wk.u + roff[r]) * esz)));
       }
       if (kk < 15) wk.step(p, halo_base, slot_base);
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NW; ++j)
       row_scales(bm[2 * j], bm[2 * j + 1], t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1], iv[2 * j + 1]);
   }
   TapWalker wk;
   wk.init(p, kb, halo_base, slot_base);
+  const int kl = kb & (kBlockK - 1);
 #pragma unroll 1
   for (int kk = 0; kk < 16; ++kk) {
-    float v[8];
+    float v[P];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int r = 0; r < P; ++r)
       v[r] = (kb + kk < p.g.K) ? lds_elem<T>(wk.slot_addr + static_cast<uint32_t>(wk.u + roff[r]) * esz) : 0.0f;
-    uint32_t w[4];
+    uint32_t w[NW];
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NW; ++j)
       w[j] = p.quant ? quant_pair_bf16x2(v[2 * j], v[2 * j + 1], iv[2 * j], iv[2 * j + 1], sc[2 * j], sc[2 * j + 1])
                      : pack_bf16x2(v[2 * j], v[2 * j + 1]);
-    sts128(a_sub + a_chunk_offset(rg, (kb & (kBlockK - 1)) + kk), w[0], w[1], w[2], w[3]);
+    store_rows<P>(a_sub, rg, kl + kk, w);
     if (kk < 15) wk.step(p, halo_base, slot_base);
   }
 }
@@ -606,13 +686,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpXf0) {
     // ------------------------------------------------------------ transform
+    // A warp covers one 16-column block of a K slice for 32 row groups:
+    // 8-row groups of two subtiles (n_mt >= 2) or 4-row groups of the single
+    // subtile (n_mt == 1), so the taps it walks are the same in every lane.
+    const int P = p.n_mt >= 2 ? 8 : 4;
     const int xw = warp - kWarpXf0;
     const int grp = xw / xf_warps_per_group;     // which K slices this warp works on
-    const int lw = xw % xf_warps_per_group;      // 2 warps per subtile
-    const int sub = lw >> 1;
-    const int blk = 2 * (lw & 1) + (lane >> 4);  // 16-column block within the K slice
-    const int rg = lane & 15;                    // 8-row group within the subtile
-    const int lr0 = 8 * rg;
+    const int lw = xw % xf_warps_per_group;
+    const int blk = lw & 3;                      // 16-column block within the K slice
+    const int sub = (P == 8) ? 2 * (lw >> 2) + (lane >> 4) : 0;
+    const int rg = (P == 8) ? (lane & 15) : lane;
+    const int lr0 = P * rg;                      // first row of the group within the subtile
     const int th = sub * p.TH + lr0 / p.TW;      // row of the tile
     const int tw0 = lr0 % p.TW;
     const uint32_t halo_base = base + p.off_halo;
@@ -646,6 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int w0 = halo_w0(p, tc.ow0);
       const int delta = tc.ow0 * g.sw - g.pw - w0;
       const int thr_al = th * g.sh * p.w_box + tw0 * g.sw;
+      const uint32_t thr_addr = static_cast<uint32_t>(thr_al) * 2u;
 #pragma unroll
       for (int r = 0; r < 8; ++r) roff[r] = thr_al + r * g.sw + delta;
       // first K slice of this tile that belongs to this warp's group
@@ -667,12 +752,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_sub = base + p.off_a + ea * p.a_stage_bytes + static_cast<uint32_t>(sub) * kASubBytes;
         const int kb = kBlockK * s + 16 * blk;
         if constexpr (sizeof(T) == 2) {
-          if (p.vec)
-            transform_task_vec<T>(p, a_sub, rg, kb, thr_al, delta, halo_base, gs_base, t, tab);
-          else
-            transform_task_gen<T>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          if (p.vec) {
+            if (P == 8)
+              transform_task_vec<T, 8>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, t, tab);
+            else
+              transform_task_vec<T, 4>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, t, tab);
+          } else if (P == 8) {
+            transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          } else {
+            transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          }
+        } else if (P == 8) {
+          transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
         } else {
-          transform_task_gen<T>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -758,7 +851,7 @@ static bool plan_fast(const ConvGeom& g, int dtype, FastParams& p, size_t& smem)
   }
   if (bTW == 0) return false;
   p.TW = bTW; p.TH = 128 / bTW; p.n_mt = bMT;
-  p.groups = 4 / bMT;
+  p.groups = bMT >= 4 ? 1 : 2;  // 8 transform warps; a K slice needs 2*n_mt (n_mt >= 2) or 4 warps
   p.n_owb = ceil_div(g.OW, p.TW);
   p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
   p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;

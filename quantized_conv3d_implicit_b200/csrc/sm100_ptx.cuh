@@ -58,14 +58,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended for up to hint_ns while
+// the phase is incomplete (it resumes as soon as the phase completes), so a
+// waiting warp does not take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Suspend hint for bounded waits: long enough that waiting threads sleep
+// instead of spinning, short enough that timeouts and aborts are noticed.
+constexpr uint32_t kQ3dSleepHintNs = 200000u;
+
 // Wait for the phase with the given parity to complete.  Returns false (and
 // sets bit `site` of *err) if it has not completed within the time limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned int* err, unsigned int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && global_timer_ns() - t0 > kQ3dWaitTimeoutNs) {
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kQ3dSleepHintNs)) return true;
+    if (global_timer_ns() - t0 > kQ3dWaitTimeoutNs) {
       if (err) atomicOr(err, site);
       return false;
     }
