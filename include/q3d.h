@@ -120,6 +120,39 @@ Q3D_API q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tens
                                      q3d_stream_t stream);
 
 /*
+ * conv3d_implicit_gemm_noalloc -- as conv3d_implicit_gemm_pad2 (same
+ * arguments, same kernels, same result), for callers that may not allocate
+ * device memory during the call.  The article has no counterpart to this
+ * entry point.
+ *
+ * Weights that cannot be read in place (dtype other than BF16, K not a
+ * multiple of 8, or a base that is not 16-byte aligned) are converted to
+ * BF16 [Cout, ld], ld = K rounded up to a multiple of 8, into a fixed
+ * staging area compiled into the library (16 MiB per device, reserved when
+ * the library module holding it first loads on that device), instead of a
+ * stream-ordered allocation.  Nothing there needs to start at zero: the
+ * staging kernel writes every byte the convolution reads, padding columns
+ * included.
+ *   - Limit: Cout * ld * 2 <= 16 MiB (e.g. Cout 384 with Cin 384 and a
+ *     3x3x3 kernel, or Cout 512 with Cin 512); larger staged weights are
+ *     rejected with Q3D_ERR_UNSUPPORTED_SHAPE before anything is enqueued.
+ *     BF16 weights usable in place have no limit.
+ *   - The first call on each device looks up the staging area's address
+ *     (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture begins.  A failed lookup returns
+ *     Q3D_ERR_CUDA.
+ *   - There is one staging area per device: two calls that stage weights
+ *     and may run at the same time on one device (different streams, or
+ *     different host threads) race on it and may read each other's
+ *     weights.  Calls ordered on one stream are safe.
+ */
+Q3D_API q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                        const float* act_amax, const int32_t stride[3],
+                                        const int32_t pad_lo[3], const int32_t pad_hi[3],
+                                        const int32_t dil[3], int32_t quant_act, q3d_tensor* out,
+                                        q3d_stream_t stream);
+
+/*
  * fp4_fake_quant -- out = NVFP4 fake-quantisation of x (sec. 6.4, 7.3).
  *   x     any rank 1..5, dtype F32/F16/BF16, numel % 16 == 0; consecutive
  *         groups of 16 elements in memory order form the blocks.

@@ -23,7 +23,8 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
           4: "Q3D_ERR_ARCH", 5: "Q3D_ERR_CUDA", 6: "Q3D_ERR_DEVICE_TIMEOUT", 7: "Q3D_ERR_UNSUPPORTED_SHAPE"}
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
-EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "fp4_fake_quant", "q3d_last_error",
+EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
+           "fp4_fake_quant", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_selftest_formats",
            "q3d_plan_conv")
 
@@ -61,6 +62,8 @@ def load_library(path: Optional[str] = None):
         lib.conv3d_implicit_gemm.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.conv3d_implicit_gemm_pad2.restype = ctypes.c_int
         lib.conv3d_implicit_gemm_pad2.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
+        lib.conv3d_implicit_gemm_noalloc.restype = ctypes.c_int
+        lib.conv3d_implicit_gemm_noalloc.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.fp4_fake_quant.restype = ctypes.c_int
         lib.fp4_fake_quant.argtypes = [T, vp, T, vp]
         lib.q3d_last_error.restype = ctypes.c_char_p
@@ -165,6 +168,27 @@ def conv3d_implicit_gemm(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.
     st = lib.conv3d_implicit_gemm_pad2(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
                                        arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
                                        _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
+def conv3d_implicit_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor,
+                                 bias: Optional[torch.Tensor] = None, stride=1, padding=0, dilation=1,
+                                 act_amax: Optional[torch.Tensor] = None, quant_act: bool = False,
+                                 stream=None) -> torch.Tensor:
+    """conv3d_implicit_gemm through the C entry point that allocates no
+    device memory (weights needing conversion are staged in the library's
+    fixed 16 MiB area per device).  `out` must be preallocated."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    if quant_act and (act_amax is None or act_amax.dtype != torch.float32 or act_amax.numel() != 1):
+        raise ValueError("quant_act requires a one-element float32 act_amax tensor")
+    arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    xs, ws, os_, bs = _tensor(x), _tensor(w), _tensor(out), _tensor(bias)
+    amax_ptr = act_amax.data_ptr() if quant_act else None
+    st = lib.conv3d_implicit_gemm_noalloc(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
+                                          arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
+                                          _stream_handle(stream))
     _check(lib, st)
     return out
 

@@ -113,35 +113,14 @@ q3d_status check_tensor(const q3d_tensor* t, const char* name, int ndim) {
   return Q3D_OK;
 }
 
-}  // namespace
-
-namespace q3d {
-
-EncodeTiledFn get_encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-}  // namespace q3d
-
-extern "C" {
-
-const char* q3d_last_error(void) { return g_last_error.c_str(); }
-
-int32_t q3d_version(void) { return 100; }
-
-q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
-                                     const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
-                                     const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_act,
-                                     q3d_tensor* out, q3d_stream_t stream) {
+// Host-side checks and geometry shared by the convolution entry points.
+// Returns Q3D_OK with *noop set for an empty batch or Cout == 0 (nothing to
+// enqueue); otherwise fills *g and *L (weights not yet staged).
+q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias, const float* act_amax,
+                        const int32_t stride[3], const int32_t pad_lo[3], const int32_t pad_hi[3],
+                        const int32_t dil[3], int32_t quant_act, q3d_tensor* out, q3d::ConvGeom* gp,
+                        q3d::ConvLaunch* Lp, bool* noop) {
+  *noop = false;
   q3d_status st;
   if ((st = check_tensor(x, "x", 5)) != Q3D_OK) return st;
   if ((st = check_tensor(w, "w", 5)) != Q3D_OK) return st;
@@ -176,7 +155,10 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
       out->shape[4] != o_dims[2])
     return fail(Q3D_ERR_INVALID_ARG, "out must have shape [%lld, %lld, %lld, %lld, %lld]", (long long)N,
                 (long long)Cout, (long long)o_dims[0], (long long)o_dims[1], (long long)o_dims[2]);
-  if (N == 0 || Cout == 0) return Q3D_OK;  // empty batch or no output channels: nothing to compute
+  if (N == 0 || Cout == 0) {  // empty batch or no output channels: nothing to compute
+    *noop = true;
+    return Q3D_OK;
+  }
   if (overlaps(out, x) || overlaps(out, w) || (bias && overlaps(out, bias)))
     return fail(Q3D_ERR_INVALID_ARG, "out overlaps an input tensor");
   const int64_t K = C * KD * KH * KW;
@@ -187,9 +169,8 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
 
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != Q3D_OK) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  q3d::ConvGeom g;
+  q3d::ConvGeom& g = *gp;
   g.N = (int32_t)N; g.C = (int32_t)C; g.D = (int32_t)D; g.H = (int32_t)H; g.W = (int32_t)W;
   g.Cout = (int32_t)Cout; g.KD = (int32_t)KD; g.KH = (int32_t)KH; g.KW = (int32_t)KW;
   g.sd = stride[0]; g.sh = stride[1]; g.sw = stride[2];
@@ -198,10 +179,57 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
   g.OD = (int32_t)o_dims[0]; g.OH = (int32_t)o_dims[1]; g.OW = (int32_t)o_dims[2];
   g.M = M; g.K = (int32_t)K; g.taps = (int32_t)(KD * KH * KW);
 
-  q3d::ConvLaunch L;
+  q3d::ConvLaunch& L = *Lp;
   L.x = x->data; L.bias = bias ? bias->data : nullptr; L.y = out->data;
   L.act_amax = quant_act ? act_amax : nullptr;
   L.dtype = x->dtype; L.quant = quant_act ? 1 : 0; L.err = dev->err_word; L.sm_count = dev->sm_count;
+  return Q3D_OK;
+}
+
+// The convolution kernels proper, once the BF16 weights are in place.
+cudaError_t launch_conv(const q3d::ConvGeom& g, const q3d::ConvLaunch& L, cudaStream_t s, const char** why) {
+  bool handled = false;
+  cudaError_t e = q3d::launch_conv3d_fast(g, L, s, why, &handled);
+  if (e == cudaSuccess && !handled) e = q3d::launch_conv3d_basic(g, L, s, why);
+  return e;
+}
+
+}  // namespace
+
+namespace q3d {
+
+EncodeTiledFn get_encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace q3d
+
+extern "C" {
+
+const char* q3d_last_error(void) { return g_last_error.c_str(); }
+
+int32_t q3d_version(void) { return 100; }
+
+q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                     const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
+                                     const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_act,
+                                     q3d_tensor* out, q3d_stream_t stream) {
+  q3d::ConvGeom g;
+  q3d::ConvLaunch L;
+  bool noop = false;
+  q3d_status st = prepare_conv(x, w, bias, act_amax, stride, pad_lo, pad_hi, dil, quant_act, out, &g, &L, &noop);
+  if (st != Q3D_OK || noop) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t K = g.K, Cout = g.Cout;
 
   // B operand: BF16 [Cout, ld] with a 16-byte row pitch.  BF16 weights with
   // K % 8 == 0 and a 16-byte aligned base are used in place; otherwise a
@@ -222,9 +250,7 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
   }
 
   const char* why = nullptr;
-  bool handled = false;
-  e = q3d::launch_conv3d_fast(g, L, s, &why, &handled);
-  if (e == cudaSuccess && !handled) e = q3d::launch_conv3d_basic(g, L, s, &why);
+  e = launch_conv(g, L, s, &why);
   if (scratch) cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) {
     if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
@@ -238,6 +264,45 @@ q3d_status conv3d_implicit_gemm(const q3d_tensor* x, const q3d_tensor* w, const 
                                 const int32_t dil[3], int32_t quant_act, q3d_tensor* out, q3d_stream_t stream) {
   if (!pad) return fail(Q3D_ERR_NULLPTR, "pad is NULL");
   return conv3d_implicit_gemm_pad2(x, w, bias, act_amax, stride, pad, pad, dil, quant_act, out, stream);
+}
+
+q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                        const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
+                                        const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_act,
+                                        q3d_tensor* out, q3d_stream_t stream) {
+  q3d::ConvGeom g;
+  q3d::ConvLaunch L;
+  bool noop = false;
+  q3d_status st = prepare_conv(x, w, bias, act_amax, stride, pad_lo, pad_hi, dil, quant_act, out, &g, &L, &noop);
+  if (st != Q3D_OK || noop) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (x->dtype == Q3D_BF16 && g.K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {
+    L.w_bf16 = w->data;  // usable in place, as in conv3d_implicit_gemm_pad2
+    L.w_ld = g.K;
+  } else {
+    const int64_t ld = (static_cast<int64_t>(g.K) + 7) / 8 * 8;
+    const int64_t bytes = static_cast<int64_t>(g.Cout) * ld * 2;
+    if (bytes > static_cast<int64_t>(q3d::kNoAllocStagingBytes))
+      return fail(Q3D_ERR_UNSUPPORTED_SHAPE,
+                  "staged BF16 weights need %lld bytes (Cout %d x %lld x 2) but the fixed staging area of "
+                  "conv3d_implicit_gemm_noalloc holds %lld; use conv3d_implicit_gemm_pad2",
+                  (long long)bytes, g.Cout, (long long)ld, (long long)q3d::kNoAllocStagingBytes);
+    void* area = nullptr;
+    e = q3d::noalloc_staging_area(&area);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc staging area)");
+    e = q3d::launch_stage_weights(w->data, x->dtype, g.Cout, g.K, ld, area, s);
+    if (e != cudaSuccess) return cuda_fail(e, "weight staging launch");
+    L.w_bf16 = area;
+    L.w_ld = ld;
+  }
+  const char* why = nullptr;
+  e = launch_conv(g, L, s, &why);
+  if (e != cudaSuccess) {
+    if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
+    return cuda_fail(e, "conv3d launch");
+  }
+  return Q3D_OK;
 }
 
 q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream) {

@@ -63,6 +63,13 @@ cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, flo
 cudaError_t launch_stage_weights(const void* w, int dtype, int32_t Cout, int32_t K, int64_t ld, void* w_bf16,
                                  cudaStream_t s);
 
+// Fixed device-resident staging area used by conv3d_implicit_gemm_noalloc
+// for BF16 weights (one per device, reserved when its module loads).
+constexpr size_t kNoAllocStagingBytes = static_cast<size_t>(16) << 20;
+// Device address of the current device's staging area (looked up once per
+// device with cudaGetSymbolAddress; the lookup's error is returned).
+cudaError_t noalloc_staging_area(void** out);
+
 // Plan of the specialised kernel (test hook): out[0] = applicable, then the
 // tiling and pipeline parameters in a fixed order (see q3d.h).
 bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out);
