@@ -43,6 +43,34 @@ L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+KERNEL_SOURCES = ("conv3d_igemm_fast.cu", "sm100_ptx.cuh", "nvfp4.cuh")
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary of this workload, or None when there is none or the kernel
+    sources have changed since it was captured (sha256 recorded beside it)."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", f"conv3d_igemm_fast_{workload}.md")
+    try:
+        with open(p) as f:
+            text = f.read()
+        h = hashlib.sha256()
+        for name in KERNEL_SOURCES:
+            with open(os.path.join(ROOT, "quantized_conv3d_implicit_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    fields = dict(line.split(":", 1) for line in text.splitlines()
+                  if line.startswith(("source_sha256:", "traffic_bytes_per_launch:")))
+    if fields.get("source_sha256", "").strip() != h.hexdigest():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"].strip())
+    except (KeyError, ValueError):
+        return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -253,7 +281,7 @@ def run_ours(args, world, rank, local):
         "layer_frac_of_peak": round(conv_tflops / peak, 4),
         "roofline": {
             "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(conv_tflops / peak, 4), "traffic": None,
+            "frac": round(conv_tflops / peak, 4), "traffic": profiled_traffic(wl.name),
             "kernel": "conv3d_igemm (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
         },
         "clocks": clocks,
