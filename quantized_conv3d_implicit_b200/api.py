@@ -26,7 +26,7 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_selftest_formats",
-           "q3d_plan_conv")
+           "q3d_plan_conv", "q3d_plan_conv_tmem")
 
 
 class Q3DTensor(ctypes.Structure):
@@ -74,9 +74,11 @@ def load_library(path: Optional[str] = None):
         lib.q3d_selftest_formats.restype = ctypes.c_int
         lib.q3d_selftest_formats.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
         i64x5 = ctypes.POINTER(ctypes.c_int64)
-        lib.q3d_plan_conv.restype = ctypes.c_int
-        lib.q3d_plan_conv.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32,
-                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+        for name in ("q3d_plan_conv", "q3d_plan_conv_tmem"):
+            fn = getattr(lib, name)
+            fn.restype = ctypes.c_int
+            fn.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32,
+                           ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
         if path is None:
             _lib = lib
         return lib
@@ -232,15 +234,19 @@ PLAN_FIELDS = ("applicable", "TH", "TW", "n_mt", "groups", "n_tile", "n_ntiles",
                "q_slots", "ring", "sa", "sb", "tmem_cols", "smem", "n_ohb", "n_owb", "vec", "w_box", "h_ext", "kd_ext")
 
 
-def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfloat16) -> dict:
-    """Test hook (host only): the specialised kernel's tiling/pipeline plan."""
+def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfloat16, kernel="fast") -> dict:
+    """Test hook (host only): the tiling/pipeline plan of the shared-memory
+    specialised kernel (kernel="fast") or of the tensor-memory kernel
+    (kernel="tmem", one more field: a_col0)."""
     lib = load_library()
     lo, hi = _pads(padding)
     a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
     a5 = lambda t: (ctypes.c_int64 * 5)(*[int(v) for v in t])  # noqa: E731
     out = (ctypes.c_int32 * 32)()
-    st = lib.q3d_plan_conv(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)),
-                           _DTYPES[dtype], out, 32)
+    fn = lib.q3d_plan_conv_tmem if kernel == "tmem" else lib.q3d_plan_conv
+    st = fn(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)), _DTYPES[dtype],
+            out, 32)
     _check(lib, st)
-    return dict(zip(PLAN_FIELDS, list(out)[:len(PLAN_FIELDS)]))
+    fields = PLAN_FIELDS + (("a_col0",) if kernel == "tmem" else ())
+    return dict(zip(fields, list(out)[:len(fields)]))
 

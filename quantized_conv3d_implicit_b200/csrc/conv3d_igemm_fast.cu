@@ -921,7 +921,7 @@ static bool plan_fast(const ConvGeom& g, int dtype, FastParams& p, size_t& smem)
 }
 
 bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
-  FastParams p;
+  FastParams p{};
   size_t smem = 0;
   const bool ok = plan_fast(g, dtype, p, smem);
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, p.groups, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
@@ -938,7 +938,7 @@ cudaError_t launch_conv3d_fast(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   if (kernel_choice() == 1) return cudaSuccess;
   const int esz = L.dtype == 0 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
-  FastParams p;
+  FastParams p{};
   size_t smem = 0;
   if (!plan_fast(g, L.dtype, p, smem)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;

@@ -1,0 +1,857 @@
+// conv3d_igemm_tmem.cu -- implicit-GEMM Conv3D for sm_100a with the A
+// operand (the implicit im2col matrix, fake-quantised on the fly) built in
+// tensor memory.
+//
+// GEMM view as in the Model-Optimizer "Conv3D Implicit GEMM CUDA kernel"
+// article, sec. 5.1 (rows (n, od, oh, ow), columns (c, kd, kh, kw)), with the
+// NVFP4 activation quantiser of sec. 6.3 fused into the A-operand producer.
+//
+// A tile is n_mt M-subtiles of 128 output positions (TH x TW rectangles of one
+// (n, od) plane, stacked along oh) times n_tile output channels.  Per 64-wide
+// K slice, the weights arrive by TMA in shared memory (K-major, 128B swizzle)
+// and the A slice is written by the transform warps straight into tensor
+// memory with tcgen05.st, one 32-bit column per pair of consecutive K
+// elements; tcgen05.mma then reads A from tensor memory and B from shared
+// memory.  Shared memory therefore carries only the input halo and the
+// weights, not A.
+//
+// Roles (24 warps, one persistent CTA per SM):
+//   warp 0      weight producer (TMA);
+//   warp 1      TMEM owner and MMA issuer (tcgen05.mma kind::f16, M = 128,
+//               N = n_tile in <= 256-wide instructions, K = 16 per
+//               instruction = one quantisation block);
+//   warp 2      halo producer: 5-D TMA boxes of x (zero fill outside the
+//               input = the convolution padding) into a ring of slots;
+//   warps 4-7   epilogue: tcgen05.ld, bias in FP32, rounding to the output
+//               dtype, bounds-checked NCDHW stores;
+//   warps 8-23  transform.  Warp w owns TMEM lane quadrant w % 4 (the lanes
+//               its tcgen05.st may reach) and 16-column block (w - 8) / 4 of
+//               every K slice; each thread owns one output position (a TMEM
+//               lane) of every subtile.  Per block it gathers its 16 halo
+//               values with per-CTA tables of tap offsets, takes the block
+//               maximum, derives the E4M3 scale (IEEE division), and
+//               dequantises through a per-row table of the eight BF16
+//               magnitudes q*scale (byte permutes indexed by the E2M1
+//               codes), then stores the 16 BF16 values with one tcgen05.st.
+// All waits are bounded; a timeout in any role aborts all roles.
+#include <algorithm>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <cuda_runtime.h>
+
+#include "nvfp4.cuh"
+#include "q3d_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace q3d {
+
+namespace {
+
+constexpr int kThreads = 768;
+constexpr int kWarpB = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpHalo = 2;
+constexpr int kWarpEpi0 = 4;
+constexpr int kWarpXf0 = 8;
+constexpr int kNumXfWarps = 16;
+constexpr int kBlockK = 64;
+constexpr int kMaxSmem = 232448;  // 227 KB dynamic shared memory per CTA
+constexpr int kMaxAcc = 8;
+constexpr int kMaxTaps = 343;     // 7x7x7
+constexpr uint32_t kTmemCols = 512;
+
+struct TmemParams {
+  ConvGeom g;
+  const void* bias;
+  void* y;
+  const float* act_amax;
+  unsigned int* err;
+  int quant;
+  // tiling
+  int TH, TW, n_mt;
+  int n_ohb, n_owb;
+  int n_tile, n_ntiles, n_sub, sub_n;
+  int64_t num_tiles;
+  int ks;
+  // halo staging
+  int align;
+  int w_box, h_ext, kd_ext, c_slot, q_slots, chan_elems;
+  uint32_t chan_bytes, slot_bytes, slot_tx;
+  int ring;
+  // pipelines
+  int sa, sb;
+  uint32_t b_stage_bytes;
+  int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
+  int dk_c, dk_phi;       // 64 = dk_c * taps + dk_phi
+  uint32_t off_b, off_halo, off_tab, off_phase, off_bar;
+};
+
+struct TileCoord {
+  int n, od, oh0, ow0, nt;
+};
+
+// Output-channel tile fastest, then the frame od, then the spatial blocks:
+// tiles running concurrently share two of their three input frames in L2.
+__device__ __forceinline__ TileCoord decode_tile(const TmemParams& p, int64_t t) {
+  TileCoord c;
+  c.nt = static_cast<int>(t % p.n_ntiles); t /= p.n_ntiles;
+  c.od = static_cast<int>(t % p.g.OD); t /= p.g.OD;
+  const int owb = static_cast<int>(t % p.n_owb); t /= p.n_owb;
+  const int ohb = static_cast<int>(t % p.n_ohb);
+  c.n = static_cast<int>(t / p.n_ohb);
+  c.oh0 = ohb * p.TH * p.n_mt;
+  c.ow0 = owb * p.TW;
+  return c;
+}
+
+__device__ __forceinline__ int floor_div(int a, int b) { return (a >= 0) ? a / b : -((-a + b - 1) / b); }
+
+// First input column of a tile's halo: the leftmost tap rounded down to a
+// 16-byte boundary (the TMA start-coordinate rule).
+__device__ __forceinline__ int halo_w0(const TmemParams& p, int ow0) {
+  return floor_div(ow0 * p.g.sw - p.g.pw, p.align) * p.align;
+}
+
+// Lowest / highest halo slot holding a column of K slice s.
+__device__ __forceinline__ int slot_lo(const TmemParams& p, int s) { return ((kBlockK * s) / p.g.taps) / p.c_slot; }
+__device__ __forceinline__ int slot_hi(const TmemParams& p, int s) {
+  return (min(kBlockK * s + kBlockK - 1, p.g.K - 1) / p.g.taps) / p.c_slot;
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, unsigned int* err, unsigned int site,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kQ3dSleepHintNs)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kQ3dWaitTimeoutNs) {
+      if (err) atomicOr(err, site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, int& a, int& b, int& c, int& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
+}
+__device__ __forceinline__ void ld_shared_v2f(uint32_t addr, float& a, float& b) {
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "r"(addr));
+}
+
+// E2M1 codes (round to nearest even, saturating) of four non-negative
+// values, one per nibble of the low 16 bits (a0 lowest).
+__device__ __forceinline__ uint32_t e2m1_codes4(float a0, float a1, float a2, float a3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1;\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "mov.b16 h, {q0, q1};\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cvt_bf16x2(float hi, float lo) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t maxabs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t maxabs_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Per-element views of a packed pair of 16-bit inputs.
+template <typename T>
+struct Half2;
+template <>
+struct Half2<__nv_bfloat16> {
+  static __device__ __forceinline__ float abs_lo(uint32_t w) { return __uint_as_float((w << 16) & 0x7FFFFFFFu); }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) { return __uint_as_float(w & 0x7FFF0000u); }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_bf16x2(a, b); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
+};
+template <>
+struct Half2<__half> {
+  static __device__ __forceinline__ float abs_lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0x7FFFu)));
+  }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>((w >> 16) & 0x7FFFu)));
+  }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_f16x2(a, b); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) {
+    return cvt_bf16x2(__half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))),
+                      __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu))));
+  }
+};
+
+// Dequantisation table of one row's block: the BF16 bit patterns of q*scale
+// for the eight E2M1 magnitudes q in code order {0, .5, 1, 1.5, 2, 3, 4, 6},
+// split into low bytes (lo_a = codes 0-3, lo_b = codes 4-7) and high bytes.
+// Each product is the binary32 product rounded to BF16; multiplying by a
+// power of two commutes with both roundings, so every entry follows from
+// BF16(scale) and BF16(binary32(1.5 * scale)) by adding to the exponent field.
+struct DqTable {
+  uint32_t lo_a, lo_b, hi_a, hi_b;
+};
+__device__ __forceinline__ DqTable dq_table(float scale) {
+  const uint32_t p = cvt_bf16x2(__fmul_rn(1.5f, scale), scale);  // lo: BF16(s), hi: BF16(1.5 s)
+  const uint32_t e01 = (p << 16) - 0x00800000u;                  // {0, s/2}
+  const uint32_t e45 = p + 0x00800080u;                          // {2s, 3s}
+  const uint32_t e67 = p + 0x01000100u;                          // {4s, 6s}
+  DqTable t;
+  t.lo_a = __byte_perm(e01, p, 0x6420);
+  t.hi_a = __byte_perm(e01, p, 0x7531);
+  t.lo_b = __byte_perm(e45, e67, 0x6420);
+  t.hi_b = __byte_perm(e45, e67, 0x7531);
+  return t;
+}
+
+// Four quantised BF16 values (two packed words) from four scaled magnitudes
+// a = |v| / scale, with the signs of the inputs (sign bits at 15 and 31 of
+// sgn01 and sgn23).
+__device__ __forceinline__ void dq4(const DqTable& t, float a0, float a1, float a2, float a3, uint32_t sgn01,
+                                    uint32_t sgn23, uint32_t& o01, uint32_t& o23) {
+  const uint32_t sel = e2m1_codes4(a0, a1, a2, a3);
+  const uint32_t lo = __byte_perm(t.lo_a, t.lo_b, sel);
+  const uint32_t hi = __byte_perm(t.hi_a, t.hi_b, sel);
+  o01 = __byte_perm(lo, hi, 0x5140) | (sgn01 & 0x80008000u);
+  o23 = __byte_perm(lo, hi, 0x7362) | (sgn23 & 0x80008000u);
+}
+
+// (scale, 1/scale) of a row's block from its |v| maximum: IEEE bmax / (6 g),
+// clamp to 448, E4M3 code, then the per-CTA table indexed by the code.
+__device__ __forceinline__ void block_scale(float bmax, float t6g, uint32_t tab, float& s, float& inv) {
+  const float r = fminf(__fdiv_rn(bmax, t6g), 448.0f);  // NaN (0/0) also becomes 448
+  uint16_t code;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(code) : "f"(0.0f), "f"(r));
+  ld_shared_v2f(tab + (code & 0x7Fu) * 8u, s, inv);
+}
+
+// One row x one 16-column block: the 16 BF16 values of A as 8 packed words.
+// addr0: shared address of the row's element for the block's first column
+// in channel c0; off[j]: byte offset of column j from addr0 (tap offset,
+// plus the distance to channel c0 + 1 for the columns past the channel end).
+// nvalid < 16 only in a partial last block (columns >= K read as zero).
+template <typename T>
+__device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], int nvalid, bool quant, float t6g,
+                                          uint32_t tab, uint32_t (&out)[8]) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t r[16];
+    if (nvalid >= 16) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = ld_shared_u16(addr0 + static_cast<uint32_t>(off[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = j < nvalid ? ld_shared_u16(addr0 + static_cast<uint32_t>(off[j])) : 0u;
+    }
+    uint32_t pk[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pk[i] = __byte_perm(r[2 * i], r[2 * i + 1], 0x5410);
+    if (!quant) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = Half2<T>::to_bf16x2(pk[i]);
+      return;
+    }
+    uint32_t m01 = Half2<T>::maxabs(pk[0], pk[1]), m23 = Half2<T>::maxabs(pk[2], pk[3]);
+    uint32_t m45 = Half2<T>::maxabs(pk[4], pk[5]), m67 = Half2<T>::maxabs(pk[6], pk[7]);
+    m01 = Half2<T>::maxabs(m01, m23);
+    m45 = Half2<T>::maxabs(m45, m67);
+    m01 = Half2<T>::maxabs(m01, m45);
+    const float bmax = fmaxf(Half2<T>::abs_lo(m01), Half2<T>::abs_hi(m01));
+    float s, inv;
+    block_scale(bmax, t6g, tab, s, inv);
+    const DqTable dt = dq_table(s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w0 = pk[2 * i], w1 = pk[2 * i + 1];
+      dq4(dt, __fmul_rn(Half2<T>::abs_lo(w0), inv), __fmul_rn(Half2<T>::abs_hi(w0), inv),
+          __fmul_rn(Half2<T>::abs_lo(w1), inv), __fmul_rn(Half2<T>::abs_hi(w1), inv), w0, w1, out[2 * i],
+          out[2 * i + 1]);
+    }
+  } else {
+    float v[16];
+    if (nvalid >= 16) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(ld_shared_u32(addr0 + static_cast<uint32_t>(off[j])));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        v[j] = j < nvalid ? __uint_as_float(ld_shared_u32(addr0 + static_cast<uint32_t>(off[j]))) : 0.0f;
+    }
+    if (!quant) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = cvt_bf16x2(v[2 * i + 1], v[2 * i]);
+      return;
+    }
+    float bmax = fabsf(v[0]);
+#pragma unroll
+    for (int j = 1; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
+    float s, inv;
+    block_scale(bmax, t6g, tab, s, inv);
+    const DqTable dt = dq_table(s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = 4 * i;
+      // sign bits of (v[j], v[j+1]) and (v[j+2], v[j+3]) at bits 15 and 31
+      const uint32_t s01 = __byte_perm(__float_as_uint(v[j]), __float_as_uint(v[j + 1]), 0x7632);
+      const uint32_t s23 = __byte_perm(__float_as_uint(v[j + 2]), __float_as_uint(v[j + 3]), 0x7632);
+      dq4(dt, __fmul_rn(fabsf(v[j]), inv), __fmul_rn(fabsf(v[j + 1]), inv), __fmul_rn(fabsf(v[j + 2]), inv),
+          __fmul_rn(fabsf(v[j + 3]), inv), s01, s23, out[2 * i], out[2 * i + 1]);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
+                             const __grid_constant__ CUtensorMap tmap_w) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+
+  const uint32_t bar_halo_full = base + p.off_bar;
+  const uint32_t bar_halo_empty = bar_halo_full + 8u * p.ring;
+  const uint32_t bar_b_full = bar_halo_empty + 8u * p.ring;
+  const uint32_t bar_b_empty = bar_b_full + 8u * p.sb;
+  const uint32_t bar_a_full = bar_b_empty + 8u * p.sb;
+  const uint32_t bar_a_empty = bar_a_full + 8u * p.sa;
+  const uint32_t bar_acc_full = bar_a_empty + 8u * p.sa;
+  const uint32_t bar_acc_empty = bar_acc_full + 8u * kMaxAcc;
+  const uint32_t bar_drain = bar_acc_empty + 8u * kMaxAcc;
+  const uint32_t bar_end = bar_drain + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + (bar_end - base));
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + (bar_end - base) + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const ConvGeom& g = p.g;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.ring; ++i) {
+      mbar_init(bar_halo_full + 8u * i, 1);
+      mbar_init(bar_halo_empty + 8u * i, 1);
+    }
+    for (int i = 0; i < p.sb; ++i) {
+      mbar_init(bar_b_full + 8u * i, 1);
+      mbar_init(bar_b_empty + 8u * i, 1);
+    }
+    for (int i = 0; i < p.sa; ++i) {
+      mbar_init(bar_a_full + 8u * i, kNumXfWarps);
+      mbar_init(bar_a_empty + 8u * i, 1);
+    }
+    for (int i = 0; i < kMaxAcc; ++i) {
+      mbar_init(bar_acc_full + 8u * i, 1);
+      mbar_init(bar_acc_empty + 8u * i, 4);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kWarpB) {
+    // ------------------------------------------------------------ weight producer
+    if (lane == 0) {
+      uint32_t gb = 0;
+      int64_t last = -1;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        for (int s = 0; s < p.ks; ++s, ++gb) {
+          const uint32_t e = gb % p.sb, u = gb / p.sb;
+          if (u > 0 && !wait_or_abort(bar_b_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteProducerEmpty, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_b_full + 8u * e, p.b_stage_bytes);
+          for (int i = 0; i < p.n_sub; ++i)
+            tma_load_2d(base + p.off_b + e * p.b_stage_bytes + static_cast<uint32_t>(i * p.sub_n) * 128u, &tmap_w,
+                        bar_b_full + 8u * e, kBlockK * s, tc.nt * p.n_tile + i * p.sub_n);
+          last = gb;
+        }
+      }
+      if (!ok && last >= 0)
+        mbar_wait(bar_b_full + 8u * static_cast<uint32_t>(last % p.sb), static_cast<uint32_t>(last / p.sb) & 1u, p.err,
+                  kSiteDrain);
+    }
+  } else if (warp == kWarpHalo) {
+    // ------------------------------------------------------------ halo producer
+    if (lane == 0) {
+      uint32_t gs = 0;
+      int64_t last = -1;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
+        const TileCoord tc = decode_tile(p, t);
+        const int w0 = halo_w0(p, tc.ow0);
+        const int h0 = tc.oh0 * g.sh - g.ph;
+        const int d0 = tc.od * g.sd - g.pd;
+        for (int q = 0; q < p.q_slots; ++q, ++gs) {
+          const uint32_t e = gs % p.ring, u = gs / p.ring;
+          if (u > 0 && !wait_or_abort(bar_halo_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteHaloEmpty, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar_halo_full + 8u * e, p.slot_tx);
+          tma_load_5d(base + p.off_halo + e * p.slot_bytes, &tmap_x, bar_halo_full + 8u * e, w0, h0, d0,
+                      q * p.c_slot, tc.n);
+          last = gs;
+        }
+      }
+      if (!ok && last >= 0)
+        mbar_wait(bar_halo_full + 8u * static_cast<uint32_t>(last % p.ring),
+                  static_cast<uint32_t>(last / p.ring) & 1u, p.err, kSiteDrain);
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
+      uint32_t ga = 0, gb = 0, it = 0, gs_base = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+        int released = 0;
+        for (int s = 0; ok && s < p.ks; ++s, ++ga, ++gb) {
+          const uint32_t ea = ga % p.sa, eb = gb % p.sb;
+          if (!wait_or_abort(bar_a_full + 8u * ea, (ga / p.sa) & 1u, p.err, kSiteAStageFull, abort_flag)) {
+            ok = false;
+            break;
+          }
+          // Slices are complete in order up to s, and no later slice reads a
+          // halo slot below the first one slice s+1 needs: hand those back.
+          const int keep = (s + 1 < p.ks) ? slot_lo(p, s + 1) : p.q_slots;
+          for (; released < keep; ++released)
+            mbar_arrive(bar_halo_empty + 8u * ((gs_base + static_cast<uint32_t>(released)) % p.ring));
+          if (!wait_or_abort(bar_b_full + 8u * eb, (gb / p.sb) & 1u, p.err, kSiteTmaFull, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_stage = tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(p.n_mt * 32);
+          const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
+          for (int i = 0; ok && i < p.n_mt; ++i) {
+            const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
+            for (int ns = 0; ns < p.n_sub; ++ns) {
+              const int acc = i * p.n_sub + ns;
+              if (s == 0 && it > 0) {
+                if (!wait_or_abort(bar_acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+              const uint64_t bsub = bdesc + static_cast<uint64_t>(ns * p.sub_n * 8);
+#pragma unroll
+              for (int j = 0; j < kBlockK / 16; ++j)
+                umma_bf16_ts(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
+                             (s > 0 || j > 0) ? 1u : 0u);
+              if (s == p.ks - 1) umma_commit(bar_acc_full + 8u * acc);
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar_a_empty + 8u * ea);
+          umma_commit(bar_b_empty + 8u * eb);
+        }
+        gs_base += static_cast<uint32_t>(p.q_slots);
+      }
+      if (!ok) {
+        umma_commit(bar_drain);
+        mbar_wait(bar_drain, 0, p.err, kSiteDrain);
+      }
+    }
+  } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    const int qw = warp - kWarpEpi0;  // == warp % 4: TMEM lanes 32*qw..
+    const int lr = qw * 32 + lane;    // row within a subtile
+    const int th_l = lr / p.TW, tw_l = lr % p.TW;
+    const int S_hw = g.OH * g.OW;
+    const int64_t S = static_cast<int64_t>(g.OD) * S_hw;
+    T* y = static_cast<T*>(p.y);
+    const T* bias = static_cast<const T*>(p.bias);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+      const TileCoord tc = decode_tile(p, t);
+      const int ow = tc.ow0 + tw_l;
+      for (int i = 0; ok && i < p.n_mt; ++i) {
+        const int oh = tc.oh0 + i * p.TH + th_l;
+        const bool valid = oh < g.OH && ow < g.OW;
+        const int64_t ybase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
+                              static_cast<int64_t>(oh) * g.OW + ow;
+        for (int ns = 0; ns < p.n_sub; ++ns) {
+          const int acc = i * p.n_sub + ns;
+          if (!wait_or_abort(bar_acc_full + 8u * acc, it & 1u, p.err, kSiteAccFull, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int co0 = tc.nt * p.n_tile + ns * p.sub_n;
+          const uint32_t taddr =
+              tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+          for (int c0 = 0; c0 < p.sub_n; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
+            tmem_wait_ld();
+            if (valid) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int co = co0 + c0 + j;
+                if (co < g.Cout) {
+                  float f = __uint_as_float(v[j]);
+                  if (bias) f = __fadd_rn(f, DTypeOps<T>::to_f32(bias[co]));
+                  y[ybase + static_cast<int64_t>(co) * S] = DTypeOps<T>::from_f32(f);
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_acc_empty + 8u * acc);
+        }
+      }
+    }
+  } else if (warp >= kWarpXf0) {
+    // ------------------------------------------------------------ transform
+    constexpr uint32_t esz = sizeof(T);
+    const int xw = warp - kWarpXf0;
+    const int quad = warp & 3;                 // TMEM lanes 32*quad..+31
+    const int blk = xw >> 2;                   // 16-column block of every K slice
+    const int row = quad * 32 + lane;          // output position within a subtile
+    const int th = row / p.TW, tw = row % p.TW;
+    const uint32_t halo_base = base + p.off_halo;
+    const uint32_t tab = base + p.off_tab;
+    const uint32_t phase_tab = base + p.off_phase;
+    const int xf_tid = threadIdx.x - kWarpXf0 * 32;
+
+    // Per-CTA tables: (scale, 1/scale) for every non-negative E4M3 code, and
+    // for every block phase phi (column index of the block's first column
+    // within its channel) the byte offsets of the 16 taps from the first
+    // tap's channel origin, ignoring the channel step (added per block).
+    float t6g = 0.0f;
+    {
+      const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f};
+      t6g = G.t;
+      if (p.quant && xf_tid < 128) {
+        uint32_t h2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
+        const float s8 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+        float s = __fmul_rn(s8, G.g);
+        if (s < 1e-5f) s = 1.0f;
+        float* e = reinterpret_cast<float*>(smem + p.off_tab + xf_tid * 8);
+        e[0] = s;
+        e[1] = __frcp_rn(s);
+      }
+      int* ph = reinterpret_cast<int*>(smem + p.off_phase);
+      for (int i = xf_tid; i < g.taps * 16; i += kNumXfWarps * 32) {
+        int t = (i >> 4) + (i & 15);
+        if (t >= g.taps) t -= g.taps;  // taps >= 16: at most one channel step per block
+        const int kw = t % g.KW, r = t / g.KW;
+        const int kh = r % g.KH, kd = r / g.KH;
+        ph[i] = (kd * g.dd * p.h_ext * p.w_box + kh * g.dh * p.w_box + kw * g.dw) * static_cast<int>(esz);
+      }
+      named_bar_sync(1, kNumXfWarps * 32);
+    }
+
+    const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
+    uint32_t gs_base = 0;  // global slot counter at the start of the tile
+    uint32_t ga = 0;       // global K-slice counter at the start of the tile
+    bool ok = true;
+    for (int64_t tt = blockIdx.x; ok && tt < p.num_tiles; tt += gridDim.x) {
+      const TileCoord tc = decode_tile(p, tt);
+      const int w0 = halo_w0(p, tc.ow0);
+      const int delta = tc.ow0 * g.sw - g.pw - w0;
+      // byte offset of this thread's output position in subtile 0, and the
+      // step to the same position in the next subtile (TH rows further down)
+      const uint32_t thr0 = static_cast<uint32_t>((th * g.sh * p.w_box + tw * g.sw + delta) * static_cast<int>(esz));
+      const uint32_t thr_step = static_cast<uint32_t>(p.TH * g.sh * p.w_box * static_cast<int>(esz));
+      // block state: first column k0, its channel c0 = (q0 slot, cs0 within
+      // the slot) and phase phi = k0 - c0 * taps
+      int k0 = 16 * blk;
+      int c0 = k0 / g.taps;
+      int phi = k0 - c0 * g.taps;
+      int q0 = c0 / p.c_slot;
+      int cs0 = c0 - q0 * p.c_slot;
+      for (int s = 0; s < p.ks; ++s) {
+        const uint32_t gslice = ga + static_cast<uint32_t>(s);
+        const uint32_t ea = gslice % p.sa, ua = gslice / p.sa;
+        if (ua > 0 && !wait_or_abort(bar_a_empty + 8u * ea, (ua - 1u) & 1u, p.err, kSiteMmaDone, abort_flag)) {
+          ok = false;
+          break;
+        }
+        for (int q = slot_lo(p, s), qh = slot_hi(p, s); ok && q <= qh; ++q) {
+          const uint32_t gsl = gs_base + static_cast<uint32_t>(q);
+          ok = wait_or_abort(bar_halo_full + 8u * (gsl % p.ring), (gsl / p.ring) & 1u, p.err, kSiteHaloFull,
+                             abort_flag);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
+                               ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(blk * 8);
+        const int nvalid = g.K - k0;
+        if (nvalid <= 0) {
+          // a block entirely past K: zeros (the weights there are zero-filled too)
+          uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          for (int i = 0; i < p.n_mt; ++i) tmem_st8(a_col + static_cast<uint32_t>(i * 32), z);
+        } else {
+          // channel origins of c0 and c0 + 1 in the halo ring
+          const uint32_t e0 = (gs_base + static_cast<uint32_t>(q0)) % static_cast<uint32_t>(p.ring);
+          const uint32_t org0 = halo_base + e0 * p.slot_bytes + static_cast<uint32_t>(cs0) * p.chan_bytes;
+          uint32_t org1;
+          if (cs0 + 1 < p.c_slot) {
+            org1 = org0 + p.chan_bytes;
+          } else {
+            const uint32_t e1 = (gs_base + static_cast<uint32_t>(q0 + 1)) % static_cast<uint32_t>(p.ring);
+            org1 = halo_base + e1 * p.slot_bytes;
+          }
+          const int step = static_cast<int>(org1 - org0);
+          const int split = g.taps - phi;  // columns j >= split belong to channel c0 + 1
+          int off[16];
+          const uint32_t prow = phase_tab + static_cast<uint32_t>(phi * 64);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) ld_shared_v4(prow + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) off[j] += (j >= split) ? step : 0;
+          for (int i = 0; i < p.n_mt; ++i) {
+            uint32_t w[8];
+            row_block<T>(org0 + thr0 + static_cast<uint32_t>(i) * thr_step, off, nvalid, p.quant != 0, t6g, tab, w);
+            tmem_st8(a_col + static_cast<uint32_t>(i * 32), w);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_a_full + 8u * ea);
+        // next slice: the block moves 64 columns on
+        k0 += kBlockK;
+        phi += p.dk_phi;
+        int dc = p.dk_c;
+        if (phi >= g.taps) {
+          phi -= g.taps;
+          ++dc;
+        }
+        cs0 += dc;
+        while (cs0 >= p.c_slot) {
+          cs0 -= p.c_slot;
+          ++q0;
+        }
+      }
+      if (!ok) break;
+      gs_base += static_cast<uint32_t>(p.q_slots);
+      ga += static_cast<uint32_t>(p.ks);
+    }
+  }
+
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+template <typename T>
+cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
+                              size_t smem, cudaStream_t s) {
+  auto kern = conv3d_igemm_tmem_kernel<T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
+  return cudaGetLastError();
+}
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+// Tiling and pipeline plan of the tensor-memory kernel (pure host
+// arithmetic).  Returns false when the kernel does not apply: fewer than 16
+// taps (a 16-column block would span more than two channels), rows of x not
+// a multiple of 16 bytes (TMA stride rule), or no plan that fits.
+static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem) {
+  const int esz = dtype == 0 ? 4 : 2;
+  const int align = 16 / esz;
+  if ((static_cast<int64_t>(g.W) * esz) % 16 != 0) return false;
+  if (g.taps < 16 || g.taps > kMaxTaps) return false;
+  memset(&p, 0, sizeof(p));
+  p.g = g;
+  p.align = align;
+
+  // output channels per tile: all of Cout up to 448 (448 + two 32-column A
+  // stages fill the 512 TMEM columns), else tiles of at most 256
+  int n_ntiles = 1, n_tile = (g.Cout + 15) / 16 * 16;
+  if (n_tile > 448) {
+    n_ntiles = ceil_div(g.Cout, 256);
+    n_tile = (ceil_div(g.Cout, n_ntiles) + 15) / 16 * 16;
+  }
+  const int n_sub = ceil_div(n_tile, 256);
+  const int sub_n = (ceil_div(n_tile, n_sub) + 15) / 16 * 16;
+  n_tile = sub_n * n_sub;
+  p.n_tile = n_tile; p.n_ntiles = n_ntiles; p.n_sub = n_sub; p.sub_n = sub_n;
+  auto a_col0_of = [&](int mt) { return (mt * n_tile + 31) / 32 * 32; };
+  auto stages_of = [&](int mt) { return (static_cast<int>(kTmemCols) - a_col0_of(mt)) / (mt * 32); };
+
+  // tile shape: subtile TH x TW = 128, n_mt subtiles stacked along oh; at
+  // least two A stages must fit next to the accumulators
+  const int kd_ext = (g.KD - 1) * g.dd + 1;
+  double best = 1e30;
+  int bTW = 0, bMT = 0;
+  for (int mt = 4; mt >= 1; mt /= 2) {
+    if (mt * n_sub > kMaxAcc || stages_of(mt) < 2) continue;
+    for (int TW = 128; TW >= 8; TW /= 2) {
+      const int TH = 128 / TW, rows = TH * mt;
+      const int h_ext = (rows - 1) * g.sh + (g.KH - 1) * g.dh + 1;
+      const int w_ext = (TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
+      const int w_box = (w_ext + 2 * (align - 1)) / align * align;
+      if (w_box > 256 || h_ext > 256 || kd_ext > 256) continue;
+      const double waste = (double)(ceil_div(g.OH, rows) * rows) * (ceil_div(g.OW, TW) * TW) / ((double)g.OH * g.OW);
+      const double halo = (double)h_ext * w_box / (128.0 * mt);
+      // fewer subtiles per tile cost weight bandwidth: about 8% per halving
+      const double score = waste * (1.0 + 0.01 * halo) * (1.0 + 0.08 * (mt >= 4 ? 0 : mt == 2 ? 1 : 2));
+      if (score < best - 1e-9) { best = score; bTW = TW; bMT = mt; }
+    }
+  }
+  if (bTW == 0) return false;
+  p.TW = bTW; p.TH = 128 / bTW; p.n_mt = bMT;
+  p.a_col0 = a_col0_of(bMT);
+  p.sa = std::min(4, stages_of(bMT));
+  p.n_owb = ceil_div(g.OW, p.TW);
+  p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
+  p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;
+  const int w_ext = (p.TW - 1) * g.sw + (g.KW - 1) * g.dw + 1;
+  p.w_box = (w_ext + 2 * (align - 1)) / align * align;
+  p.kd_ext = kd_ext;
+  p.chan_elems = p.kd_ext * p.h_ext * p.w_box;
+  p.chan_bytes = static_cast<uint32_t>(p.chan_elems * esz);
+  p.ks = ceil_div(g.K, kBlockK);
+  p.num_tiles = static_cast<int64_t>(g.N) * g.OD * p.n_ohb * p.n_owb * n_ntiles;
+  p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
+  p.dk_c = kBlockK / g.taps;
+  p.dk_phi = kBlockK - p.dk_c * g.taps;
+
+  const int chan_bytes = static_cast<int>(p.chan_bytes);
+  const int phase_bytes = g.taps * 64;
+  // Halo ring: the MMA thread hands a slot back once every slice that reads
+  // it is complete, while the transform may run up to sa slices ahead of the
+  // MMA, so the ring holds the slots of sa consecutive slices (+2 so the
+  // producer can run ahead).
+  for (int target = 10240; target >= 1; target = (target > chan_bytes ? target / 2 : 0)) {
+    p.c_slot = std::max(1, std::min(std::min(256, g.C), target / chan_bytes));
+    p.q_slots = ceil_div(g.C, p.c_slot);
+    p.slot_tx = static_cast<uint32_t>(p.c_slot) * p.chan_bytes;
+    p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
+    int span = 1;
+    for (int s0 = 0; s0 < p.ks; ++s0) {
+      const int lo = ((kBlockK * s0) / g.taps) / p.c_slot;
+      const int hi = (std::min(kBlockK * (s0 + p.sa) - 1, g.K - 1) / g.taps) / p.c_slot;
+      span = std::max(span, hi - lo + 1);
+    }
+    const int r = span + 2;
+    for (int b = 8; b >= 2; --b) {
+      const int nbar = 2 * r + 2 * b + 2 * p.sa + 2 * kMaxAcc + 1;
+      const int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
+                        64 /* pad after the halo ring */ + 1024 /* scale table */ + phase_bytes + nbar * 8 + 16;
+      if (total <= kMaxSmem) {
+        p.sb = b; p.ring = r;
+        p.off_b = 0;
+        p.off_halo = p.off_b + b * p.b_stage_bytes;
+        p.off_tab = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
+        p.off_phase = p.off_tab + 1024u;
+        p.off_bar = p.off_phase + static_cast<uint32_t>(phase_bytes);
+        smem = static_cast<size_t>(total);
+        return true;
+      }
+    }
+    if (p.c_slot == 1) break;
+  }
+  return false;
+}
+
+bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
+  TmemParams p{};
+  size_t smem = 0;
+  const bool ok = plan_tmem(g, dtype, p, smem);
+  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 1, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
+                       p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
+                       static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0};
+  const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
+  for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
+  return ok;
+}
+
+cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
+                               bool* handled) {
+  *handled = false;
+  const int esz = L.dtype == 0 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
+  TmemParams p{};
+  size_t smem = 0;
+  if (!plan_tmem(g, L.dtype, p, smem)) return cudaSuccess;
+  p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
+
+  EncodeTiledFn encode = get_encode_tiled();
+  if (!encode) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }
+  CUtensorMap tmap_x, tmap_w;
+  {
+    const CUtensorMapDataType dt = L.dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                   : L.dtype == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const cuuint64_t dims[5] = {(cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.D, (cuuint64_t)g.C, (cuuint64_t)g.N};
+    const cuuint64_t st[4] = {(cuuint64_t)g.W * esz, (cuuint64_t)g.H * g.W * esz, (cuuint64_t)g.D * g.H * g.W * esz,
+                              (cuuint64_t)g.C * g.D * g.H * g.W * esz};
+    const cuuint32_t box[5] = {(cuuint32_t)p.w_box, (cuuint32_t)p.h_ext, (cuuint32_t)p.kd_ext, (cuuint32_t)p.c_slot, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    CUresult cr = encode(&tmap_x, dt, 5, const_cast<void*>(L.x), dims, st, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaSuccess;  // shape the TMA unit cannot describe: another kernel
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)g.K, (cuuint64_t)g.Cout};
+    const cuuint64_t st[1] = {(cuuint64_t)L.w_ld * 2u};
+    const cuuint32_t box[2] = {(cuuint32_t)kBlockK, (cuuint32_t)p.sub_n};
+    const cuuint32_t es[2] = {1, 1};
+    CUresult cr = encode(&tmap_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(L.w_bf16), dims, st, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) { *why = "weight tensor map rejected"; return cudaErrorInvalidValue; }
+  }
+  const int64_t grid64 = std::min<int64_t>(p.num_tiles, L.sm_count);
+  *handled = true;
+  switch (L.dtype) {
+    case 0: return launch_tmem_typed<float>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+    case 1: return launch_tmem_typed<__half>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+    default: return launch_tmem_typed<__nv_bfloat16>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+  }
+}
+
+}  // namespace q3d

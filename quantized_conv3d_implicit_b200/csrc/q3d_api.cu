@@ -23,6 +23,8 @@ namespace q3d {
 cudaError_t launch_conv3d_basic(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why);
 cudaError_t launch_conv3d_fast(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
                                bool* handled);
+cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
+                               bool* handled);
 }  // namespace q3d
 
 namespace {
@@ -186,12 +188,24 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
   return Q3D_OK;
 }
 
-// The convolution kernels proper, once the BF16 weights are in place.
+// The convolution kernels proper, once the BF16 weights are in place: the
+// tensor-memory kernel where it applies, else the shared-memory specialised
+// kernel, else the general one.  Q3D_KERNEL=tmem|fast|basic starts the chain
+// at that kernel (all three compute the same result).
 cudaError_t launch_conv(const q3d::ConvGeom& g, const q3d::ConvLaunch& L, cudaStream_t s, const char** why) {
+  const char* kc = getenv("Q3D_KERNEL");
+  const int first = (kc && !strcmp(kc, "basic")) ? 2 : (kc && !strcmp(kc, "fast")) ? 1 : 0;
   bool handled = false;
-  cudaError_t e = q3d::launch_conv3d_fast(g, L, s, why, &handled);
-  if (e == cudaSuccess && !handled) e = q3d::launch_conv3d_basic(g, L, s, why);
-  return e;
+  cudaError_t e = cudaSuccess;
+  if (first <= 0) {
+    e = q3d::launch_conv3d_tmem(g, L, s, why, &handled);
+    if (e != cudaSuccess || handled) return e;
+  }
+  if (first <= 1) {
+    e = q3d::launch_conv3d_fast(g, L, s, why, &handled);
+    if (e != cudaSuccess || handled) return e;
+  }
+  return q3d::launch_conv3d_basic(g, L, s, why);
 }
 
 }  // namespace
@@ -359,13 +373,14 @@ q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* 
   return Q3D_OK;
 }
 
-q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
-                         const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
-                         int32_t* plan, int32_t plan_len) {
+// Geometry of a planning request (host only); Q3D_OK or an argument error.
+static q3d_status plan_geom(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                            const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
+                            int32_t* plan, q3d::ConvGeom* gp) {
   if (!x_shape || !w_shape || !stride || !pad_lo || !pad_hi || !dil || !plan)
     return fail(Q3D_ERR_NULLPTR, "NULL pointer");
   if (!dtype_ok(dtype)) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "dtype");
-  q3d::ConvGeom g;
+  q3d::ConvGeom& g = *gp;
   const int64_t k_dims[3] = {w_shape[2], w_shape[3], w_shape[4]};
   int64_t o_dims[3];
   for (int i = 0; i < 3; ++i) {
@@ -386,7 +401,26 @@ q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], con
   g.M = x_shape[0] * o_dims[0] * o_dims[1] * o_dims[2];
   g.K = (int32_t)(x_shape[1] * k_dims[0] * k_dims[1] * k_dims[2]);
   g.taps = (int32_t)(k_dims[0] * k_dims[1] * k_dims[2]);
+  return Q3D_OK;
+}
+
+q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                         const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
+                         int32_t* plan, int32_t plan_len) {
+  q3d::ConvGeom g;
+  const q3d_status st = plan_geom(x_shape, w_shape, stride, pad_lo, pad_hi, dil, dtype, plan, &g);
+  if (st != Q3D_OK) return st;
   q3d::plan_conv3d_fast(g, dtype, plan, plan_len);
+  return Q3D_OK;
+}
+
+q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                              const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
+                              int32_t* plan, int32_t plan_len) {
+  q3d::ConvGeom g;
+  const q3d_status st = plan_geom(x_shape, w_shape, stride, pad_lo, pad_hi, dil, dtype, plan, &g);
+  if (st != Q3D_OK) return st;
+  q3d::plan_conv3d_tmem(g, dtype, plan, plan_len);
   return Q3D_OK;
 }
 

@@ -73,6 +73,9 @@ cudaError_t noalloc_staging_area(void** out);
 // Plan of the specialised kernel (test hook): out[0] = applicable, then the
 // tiling and pipeline parameters in a fixed order (see q3d.h).
 bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out);
+// The same for the tensor-memory kernel (groups = 1, TMEM columns = 512,
+// vectorised reads = 0; one more entry: the first TMEM column of A).
+bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out);
 
 // The implicit-GEMM convolution; returns a CUDA error or cudaSuccess, and a
 // short reason in *why when it rejects the problem before launching.

@@ -18,14 +18,16 @@ from _parity import assert_conv_close, bits, to_np_f32
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["auto", "basic"])
+@pytest.fixture(params=["auto", "fast", "basic"])
 def kernel(request, monkeypatch):
-    """Run a test with the library's default kernel choice and again with the
-    general-purpose kernel forced (both must meet the same bar)."""
-    if request.param == "basic":
-        monkeypatch.setenv("Q3D_KERNEL", "basic")
-    else:
+    """Run a test with the library's default kernel choice (the tensor-memory
+    kernel where it applies), with the shared-memory specialised kernel
+    forced, and with the general-purpose kernel forced: all must meet the
+    same bar."""
+    if request.param == "auto":
         monkeypatch.delenv("Q3D_KERNEL", raising=False)
+    else:
+        monkeypatch.setenv("Q3D_KERNEL", request.param)
     return request.param
 
 
@@ -56,6 +58,13 @@ SHAPES = [
     ((1, 4, 5, 8, 8), 16, (3, 3, 3), (2, 3, 1), (0, 1, 2), (1, 0, 0), (2, 1, 3)),      # mixed everything
     ((1, 7, 3, 3, 3), 5, (3, 3, 3), (1, 1, 1), (0, 0, 0), (0, 0, 0), (1, 1, 1)),       # 1x1x1 output, K=189
     ((3, 16, 2, 5, 7), 40, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # batch 3, M=210
+    # rows of x a multiple of 16 bytes (TMA-fed kernels), with ragged tiles
+    ((1, 5, 4, 9, 16), 24, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1)),     # K=135: partial block
+    ((1, 6, 6, 13, 24), 33, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 2, 2)),    # dilation
+    ((2, 5, 5, 9, 32), 20, (3, 3, 3), (1, 2, 2), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # stride 2
+    ((1, 3, 7, 9, 16), 8, (5, 5, 5), (1, 1, 1), (2, 2, 2), (2, 2, 2), (1, 1, 1)),      # 5x5x5, K=375
+    ((1, 8, 3, 6, 8), 500, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # two N tiles
+    ((1, 20, 3, 21, 40), 200, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1)),  # K=540, N=208
 ]
 
 
@@ -72,11 +81,13 @@ def test_conv_small_shapes(cuda_ok, kernel, case, quant, dtype):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("quant", [False, True])
-def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, quant, dtype):
+@pytest.mark.parametrize("width", [11, 16])
+def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, quant, dtype, width):
     # one-hot weights: y[:, co] = A[:, k(co)], a single nonzero product per
     # output, so the FP32 accumulator holds the BF16 operand exactly and the
-    # whole im2col row (quantised or not) is reproduced bit for bit
-    xs, k = (1, 5, 4, 9, 11), (3, 3, 3)
+    # whole im2col row (quantised or not) is reproduced bit for bit; W = 16
+    # reaches the TMA-fed kernels, W = 11 the general one
+    xs, k = (1, 5, 4, 9, width), (3, 3, 3)
     K = 5 * 27
     g = torch.Generator().manual_seed(3)
     x = (torch.randn(xs, generator=g) * 3).to(dtype)

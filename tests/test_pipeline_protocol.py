@@ -36,7 +36,7 @@ class Bar:
         return (self.phase & 1) != (phase & 1)
 
 
-def roles(plan, K, taps, ntiles):
+def roles(plan, K, taps, ntiles, kernel="fast"):
     bars = {}
 
     def bar(name, i, count):
@@ -47,7 +47,8 @@ def roles(plan, K, taps, ntiles):
 
     ks, q_slots, ring, sa, sb, G = (plan[k] for k in ("ks", "q_slots", "ring", "sa", "sb", "groups"))
     n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
-    wpg = 8 // G
+    n_xf = 16 if kernel == "tmem" else 8   # transform warps; the tensor-memory kernel has one group
+    wpg = n_xf // G
 
     def slot_lo(s):
         return ((64 * s) // taps) // c_slot
@@ -129,13 +130,13 @@ def roles(plan, K, taps, ntiles):
     r = {"halo": halo_producer(), "weights": weight_producer(), "mma": mma()}
     for w in range(4):
         r[f"epilogue{w}"] = epilogue()
-    for w in range(8):
+    for w in range(n_xf):
         r[f"transform{w}"] = transform(w)
     return r
 
 
-def run(plan, K, taps, ntiles, order="rr", seed=0):
-    rs = roles(plan, K, taps, ntiles)
+def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast"):
+    rs = roles(plan, K, taps, ntiles, kernel)
     names = list(rs)
     cur = {k: None for k in names}
     done = set()
@@ -172,15 +173,16 @@ def run(plan, K, taps, ntiles, order="rr", seed=0):
         assert progress, "deadlock: " + ", ".join(k for k in names if k not in done)
 
 
-def _plan(wl_or_args):
+def _plan(wl_or_args, kernel="fast"):
     if isinstance(wl_or_args, workloads.Workload):
         wl = wl_or_args
         pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
         w_shape = (wl.cout, wl.x_shape[1]) + tuple(wl.kernel)
-        return api.plan_conv(wl.x_shape, w_shape, wl.stride, pad6, wl.dil, wl.dtype), wl.k_gemm, \
+        return api.plan_conv(wl.x_shape, w_shape, wl.stride, pad6, wl.dil, wl.dtype, kernel=kernel), wl.k_gemm, \
             wl.kernel[0] * wl.kernel[1] * wl.kernel[2]
     xs, ws, s, pad6, d, dt = wl_or_args
-    return api.plan_conv(xs, ws, s, pad6, d, dt), ws[1] * ws[2] * ws[3] * ws[4], ws[2] * ws[3] * ws[4]
+    return api.plan_conv(xs, ws, s, pad6, d, dt, kernel=kernel), ws[1] * ws[2] * ws[3] * ws[4], \
+        ws[2] * ws[3] * ws[4]
 
 
 def _check_invariants(p):
@@ -235,3 +237,56 @@ def test_sim_detects_aliasing_when_stages_fewer_than_groups():
     bad = dict(plan, sa=plan["groups"] - 1)
     with pytest.raises(AssertionError):
         run(bad, K, taps, ntiles=3)
+
+
+def _check_tmem_invariants(p, taps):
+    assert p["groups"] == 1 and p["tmem_cols"] == 512 and taps >= 16
+    # accumulators [0, n_mt*n_tile), then sa A stages of n_mt * 32 columns
+    assert p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
+    assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512 and p["sa"] >= 2
+    assert p["n_mt"] * p["n_sub"] <= 8
+    assert p["n_sub"] * p["sub_n"] == p["n_tile"] and p["sub_n"] % 16 == 0 and 16 <= p["sub_n"] <= 256
+    assert p["smem"] <= 232448 and p["TH"] * p["TW"] == 128
+    assert p["w_box"] <= 256 and p["h_ext"] <= 256 and p["kd_ext"] <= 256
+
+
+@pytest.mark.parametrize("name", sorted(workloads.WORKLOADS))
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_tmem_kernel_plans_are_deadlock_and_alias_free(name, order):
+    plan, K, taps = _plan(workloads.WORKLOADS[name], kernel="tmem")
+    if taps < 16:
+        assert plan["applicable"] == 0
+        return
+    assert plan["applicable"] == 1
+    _check_tmem_invariants(plan, taps)
+    run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)), kernel="tmem")
+
+
+def test_tmem_kernel_random_shapes():
+    rng = random.Random(11)
+    checked = 0
+    for _ in range(80):
+        k = rng.choice([(3, 3, 3), (5, 5, 5), (3, 3, 2), (1, 5, 5), (2, 3, 3)])
+        cin = rng.choice([1, 3, 8, 16, 37, 64, 96, 192, 256])
+        cout = rng.choice([1, 8, 16, 40, 96, 100, 192, 256, 300, 384, 448, 512, 640, 1024])
+        xs = (rng.choice([1, 2]), cin, rng.randint(k[0], 9), rng.randint(k[1], 40), 8 * rng.randint(1, 30))
+        s = (1, rng.choice([1, 1, 2]), rng.choice([1, 1, 2]))
+        d = (1, rng.choice([1, 2]), rng.choice([1, 2]))
+        pad6 = tuple(rng.randint(0, 2) for _ in range(6))
+        ws = (cout, cin) + k
+        dt = rng.choice([torch.bfloat16, torch.float16, torch.float32])
+        try:
+            plan, K, taps = _plan((xs, ws, s, pad6, d, dt), kernel="tmem")
+        except api.Q3DError:
+            continue  # empty output: not a valid convolution
+        if not plan["applicable"]:
+            continue
+        _check_tmem_invariants(plan, taps)
+        run(plan, K, taps, ntiles=2, order="random", seed=checked, kernel="tmem")
+        checked += 1
+    assert checked >= 40
+
+
+def test_tmem_kernel_declines_fewer_than_16_taps():
+    plan, _, _ = _plan(((1, 64, 4, 16, 16), (64, 64, 1, 3, 3), 1, 1, 1, torch.bfloat16), kernel="tmem")
+    assert plan["applicable"] == 0 and plan["TW"] == 0
