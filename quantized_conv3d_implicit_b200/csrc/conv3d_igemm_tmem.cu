@@ -113,12 +113,6 @@ __device__ __forceinline__ int halo_w0(const TmemParams& p, int ow0) {
   return floor_div(ow0 * p.g.sw - p.g.pw, p.align) * p.align;
 }
 
-// Lowest / highest halo slot holding a column of K slice s.
-__device__ __forceinline__ int slot_lo(const TmemParams& p, int s) { return ((kBlockK * s) / p.g.taps) / p.c_slot; }
-__device__ __forceinline__ int slot_hi(const TmemParams& p, int s) {
-  return (min(kBlockK * s + kBlockK - 1, p.g.K - 1) / p.g.taps) / p.c_slot;
-}
-
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, unsigned int* err, unsigned int site,
                                               volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -353,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.ring; ++i) {
       mbar_init(bar_halo_full + 8u * i, 1);
-      mbar_init(bar_halo_empty + 8u * i, 1);
+      mbar_init(bar_halo_empty + 8u * i, kNumXfWarps);  // every transform warp hands the slot back
     }
     for (int i = 0; i < p.sb; ++i) {
       mbar_init(bar_b_full + 8u * i, 1);
@@ -437,21 +431,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
-      uint32_t ga = 0, gb = 0, it = 0, gs_base = 0;
+      uint32_t ga = 0, gb = 0, it = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
-        int released = 0;
         for (int s = 0; ok && s < p.ks; ++s, ++ga, ++gb) {
           const uint32_t ea = ga % p.sa, eb = gb % p.sb;
           if (!wait_or_abort(bar_a_full + 8u * ea, (ga / p.sa) & 1u, p.err, kSiteAStageFull, abort_flag)) {
             ok = false;
             break;
           }
-          // Slices are complete in order up to s, and no later slice reads a
-          // halo slot below the first one slice s+1 needs: hand those back.
-          const int keep = (s + 1 < p.ks) ? slot_lo(p, s + 1) : p.q_slots;
-          for (; released < keep; ++released)
-            mbar_arrive(bar_halo_empty + 8u * ((gs_base + static_cast<uint32_t>(released)) % p.ring));
           if (!wait_or_abort(bar_b_full + 8u * eb, (gb / p.sb) & 1u, p.err, kSiteTmaFull, abort_flag)) {
             ok = false;
             break;
@@ -483,7 +471,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(bar_a_empty + 8u * ea);
           umma_commit(bar_b_empty + 8u * eb);
         }
-        gs_base += static_cast<uint32_t>(p.q_slots);
       }
       if (!ok) {
         umma_commit(bar_drain);
@@ -602,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int phi = k0 - c0 * g.taps;
       int q0 = c0 / p.c_slot;
       int cs0 = c0 - q0 * p.c_slot;
+      int released = 0;  // halo slots of this tile this warp has handed back
       for (int s = 0; s < p.ks; ++s) {
         const uint32_t gslice = ga + static_cast<uint32_t>(s);
         const uint32_t ea = gslice % p.sa, ua = gslice / p.sa;
@@ -609,16 +597,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        for (int q = slot_lo(p, s), qh = slot_hi(p, s); ok && q <= qh; ++q) {
-          const uint32_t gsl = gs_base + static_cast<uint32_t>(q);
-          ok = wait_or_abort(bar_halo_full + 8u * (gsl % p.ring), (gsl / p.ring) & 1u, p.err, kSiteHaloFull,
-                             abort_flag);
+        const int nvalid = g.K - k0;
+        const int split = g.taps - phi;  // columns j >= split belong to channel c0 + 1
+        if (nvalid > 0) {
+          // the halo slot of channel c0, and the next slot when the block's
+          // tail reaches channel c0 + 1 and that channel starts the next slot
+          const int nslots = (split < min(16, nvalid) && cs0 + 1 == p.c_slot) ? 2 : 1;
+          for (int q = q0; ok && q < q0 + nslots; ++q) {
+            const uint32_t gsl = gs_base + static_cast<uint32_t>(q);
+            ok = wait_or_abort(bar_halo_full + 8u * (gsl % p.ring), (gsl / p.ring) & 1u, p.err, kSiteHaloFull,
+                               abort_flag);
+          }
         }
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
                                ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(blk * 8);
-        const int nvalid = g.K - k0;
         if (nvalid <= 0) {
           // a block entirely past K: zeros (the weights there are zero-filled too)
           uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
@@ -635,7 +629,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             org1 = halo_base + e1 * p.slot_bytes;
           }
           const int step = static_cast<int>(org1 - org0);
-          const int split = g.taps - phi;  // columns j >= split belong to channel c0 + 1
           int off[16];
           const uint32_t prow = phase_tab + static_cast<uint32_t>(phi * 64);
 #pragma unroll
@@ -651,7 +644,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar_a_full + 8u * ea);
         // next slice: the block moves 64 columns on
         k0 += kBlockK;
         phi += p.dk_phi;
@@ -664,6 +656,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (cs0 >= p.c_slot) {
           cs0 -= p.c_slot;
           ++q0;
+        }
+        if (lane == 0) {
+          mbar_arrive(bar_a_full + 8u * ea);
+          // Later blocks of this warp start at slot q0 or above: hand the
+          // slots below back (a slot is free once all transform warps have).
+          const int keep = (s + 1 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
+          for (; released < keep; ++released)
+            mbar_arrive(bar_halo_empty + 8u * ((gs_base + static_cast<uint32_t>(released)) % p.ring));
         }
       }
       if (!ok) break;
@@ -760,10 +760,10 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
 
   const int chan_bytes = static_cast<int>(p.chan_bytes);
   const int phase_bytes = g.taps * 64;
-  // Halo ring: the MMA thread hands a slot back once every slice that reads
-  // it is complete, while the transform may run up to sa slices ahead of the
-  // MMA, so the ring holds the slots of sa consecutive slices (+2 so the
-  // producer can run ahead).
+  // Halo ring: the transform warps hand a slot back as soon as they are past
+  // it, so the ring only has to hold one slice's slots for progress; it is
+  // sized for sa slices plus two, and any shared memory left after the
+  // weight stages buys further slots (more halo loads in flight).
   for (int target = 10240; target >= 1; target = (target > chan_bytes ? target / 2 : 0)) {
     p.c_slot = std::max(1, std::min(std::min(256, g.C), target / chan_bytes));
     p.q_slots = ceil_div(g.C, p.c_slot);
@@ -775,12 +775,17 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
       const int hi = (std::min(kBlockK * (s0 + p.sa) - 1, g.K - 1) / g.taps) / p.c_slot;
       span = std::max(span, hi - lo + 1);
     }
-    const int r = span + 2;
     for (int b = 8; b >= 2; --b) {
+      int r = span + 2;
       const int nbar = 2 * r + 2 * b + 2 * p.sa + 2 * kMaxAcc + 1;
-      const int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
+      int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
                         64 /* pad after the halo ring */ + 1024 /* scale table */ + phase_bytes + nbar * 8 + 16;
       if (total <= kMaxSmem) {
+        const int extra = std::min(32 - r, (kMaxSmem - total) / (static_cast<int>(p.slot_bytes) + 16));
+        if (extra > 0) {
+          r += extra;
+          total += extra * (static_cast<int>(p.slot_bytes) + 16);
+        }
         p.sb = b; p.ring = r;
         p.off_b = 0;
         p.off_halo = p.off_b + b * p.b_stage_bytes;

@@ -26,7 +26,9 @@ class Bar:
     def __init__(self, count):
         self.count, self.pending, self.phase = count, count, 0
 
-    def arrive(self):
+    def arrive(self, phase=None):
+        # an arrival meant for a given phase must not land in an earlier one
+        assert phase is None or phase == self.phase, f"arrival for phase {phase} while at {self.phase}"
         self.pending -= 1
         if self.pending == 0:
             self.phase += 1
@@ -49,6 +51,10 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
     n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
     n_xf = 16 if kernel == "tmem" else 8   # transform warps; the tensor-memory kernel has one group
     wpg = n_xf // G
+    # who hands halo slots back: the MMA thread (shared-memory kernel) or
+    # every transform warp once it is past the slot (tensor-memory kernel)
+    xf_release = kernel == "tmem"
+    halo_empty_count = n_xf if xf_release else 1
 
     def slot_lo(s):
         return ((64 * s) // taps) // c_slot
@@ -62,7 +68,7 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
             for _q in range(q_slots):
                 e, u = gs % ring, gs // ring
                 if u > 0:
-                    yield ("wait", bar("halo_empty", e, 1), u - 1)
+                    yield ("wait", bar("halo_empty", e, halo_empty_count), u - 1)
                 yield ("arrive", bar("halo_full", e, 1))
                 gs += 1
 
@@ -84,7 +90,7 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
                 ea, eb = ga % sa, gb % sb
                 yield ("wait", bar("a_full", ea, wpg), ga // sa)
                 keep = slot_lo(s + 1) if s + 1 < ks else q_slots
-                while released < keep:
+                while not xf_release and released < keep:
                     yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
                     released += 1
                 yield ("wait", bar("b_full", eb, 1), gb // sb)
@@ -111,18 +117,43 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
 
     def transform(w):
         grp = w // wpg
+        blk = w >> 2   # tensor-memory kernel: 16-column block of every slice
         ga = gs_base = 0
         for _ in range(ntiles):
             s = (grp + G - ga % G) % G
+            released = 0
             while s < ks:
                 gsl = ga + s
                 ea, ua = gsl % sa, gsl // sa
                 if ua > 0:
                     yield ("wait", bar("a_empty", ea, 1), ua - 1)
-                for q in range(slot_lo(s), slot_hi(s) + 1):
+                if xf_release:
+                    # only the slots this warp's block reads
+                    k0 = 64 * s + 16 * blk
+                    qs = []
+                    if k0 < K:
+                        c0, phi = divmod(k0, taps)
+                        q0, cs0 = divmod(c0, c_slot)
+                        split, nvalid = taps - phi, K - k0
+                        qs = [q0, q0 + 1] if (split < min(16, nvalid) and cs0 + 1 == c_slot) else [q0]
+                else:
+                    qs = range(slot_lo(s), slot_hi(s) + 1)
+                for q in qs:
                     g = gs_base + q
                     yield ("wait", bar("halo_full", g % ring, 1), g // ring)
                 yield ("arrive", bar("a_full", ea, wpg))
+                if xf_release:
+                    # the tensor-memory kernel's warps hand back the slots below
+                    # their next block's slot (phase = use of the ring entry)
+                    if s + 1 < ks:
+                        k0n = 64 * (s + 1) + 16 * blk
+                        keep = min((k0n // taps) // c_slot, q_slots)
+                    else:
+                        keep = q_slots
+                    while released < keep:
+                        g = gs_base + released
+                        yield ("arrive", bar("halo_empty", g % ring, halo_empty_count), g // ring)
+                        released += 1
                 s += G
             ga += ks
             gs_base += q_slots
@@ -159,7 +190,7 @@ def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast"):
                         break
                 op = cur[k]
                 if op[0] == "arrive":
-                    op[1].arrive()
+                    op[1].arrive(op[2] if len(op) > 2 else None)
                     cur[k] = None
                     progress = True
                     continue
