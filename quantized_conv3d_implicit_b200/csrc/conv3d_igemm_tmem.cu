@@ -113,6 +113,20 @@ __device__ __forceinline__ int halo_w0(const TmemParams& p, int ow0) {
   return floor_div(ow0 * p.g.sw - p.g.pw, p.align) * p.align;
 }
 
+// Position in a ring of n pipeline entries: the entry, and the parity of the
+// pass over the ring (the barrier phase that a use of the entry completes).
+// Advanced by one compare per step, so no pipeline loop divides.
+struct RingPos {
+  uint32_t e, ph;
+  __device__ __forceinline__ void next(uint32_t n) {
+    if (++e == n) {
+      e = 0;
+      ph ^= 1u;
+    }
+  }
+};
+__device__ __forceinline__ RingPos ring_pos(uint32_t g, uint32_t n) { return RingPos{g % n, (g / n) & 1u}; }
+
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, unsigned int* err, unsigned int site,
                                               volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -379,13 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ weight producer
     if (lane == 0) {
       uint32_t gb = 0;
-      int64_t last = -1;
-      bool ok = true;
+      RingPos bp{0u, 0u}, last{0u, 0u};
+      bool ok = true, any = false;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
-        for (int s = 0; s < p.ks; ++s, ++gb) {
-          const uint32_t e = gb % p.sb, u = gb / p.sb;
-          if (u > 0 && !wait_or_abort(bar_b_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteProducerEmpty, abort_flag)) {
+        for (int s = 0; s < p.ks; ++s, ++gb, bp.next(static_cast<uint32_t>(p.sb))) {
+          const uint32_t e = bp.e;
+          if (gb >= static_cast<uint32_t>(p.sb) &&
+              !wait_or_abort(bar_b_empty + 8u * e, bp.ph ^ 1u, p.err, kSiteProducerEmpty, abort_flag)) {
             ok = false;
             break;
           }
@@ -393,54 +408,55 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < p.n_sub; ++i)
             tma_load_2d(base + p.off_b + e * p.b_stage_bytes + static_cast<uint32_t>(i * p.sub_n) * 128u, &tmap_w,
                         bar_b_full + 8u * e, kBlockK * s, tc.nt * p.n_tile + i * p.sub_n);
-          last = gb;
+          last = bp;
+          any = true;
         }
       }
-      if (!ok && last >= 0)
-        mbar_wait(bar_b_full + 8u * static_cast<uint32_t>(last % p.sb), static_cast<uint32_t>(last / p.sb) & 1u, p.err,
-                  kSiteDrain);
+      if (!ok && any) mbar_wait(bar_b_full + 8u * last.e, last.ph, p.err, kSiteDrain);
     }
   } else if (warp == kWarpHalo) {
     // ------------------------------------------------------------ halo producer
     if (lane == 0) {
       uint32_t gs = 0;
-      int64_t last = -1;
-      bool ok = true;
+      RingPos hp{0u, 0u}, last{0u, 0u};
+      bool ok = true, any = false;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
         const int w0 = halo_w0(p, tc.ow0);
         const int h0 = tc.oh0 * g.sh - g.ph;
         const int d0 = tc.od * g.sd - g.pd;
-        for (int q = 0; q < p.q_slots; ++q, ++gs) {
-          const uint32_t e = gs % p.ring, u = gs / p.ring;
-          if (u > 0 && !wait_or_abort(bar_halo_empty + 8u * e, (u - 1u) & 1u, p.err, kSiteHaloEmpty, abort_flag)) {
+        for (int q = 0; q < p.q_slots; ++q, ++gs, hp.next(static_cast<uint32_t>(p.ring))) {
+          const uint32_t e = hp.e;
+          if (gs >= static_cast<uint32_t>(p.ring) &&
+              !wait_or_abort(bar_halo_empty + 8u * e, hp.ph ^ 1u, p.err, kSiteHaloEmpty, abort_flag)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(bar_halo_full + 8u * e, p.slot_tx);
           tma_load_5d(base + p.off_halo + e * p.slot_bytes, &tmap_x, bar_halo_full + 8u * e, w0, h0, d0,
                       q * p.c_slot, tc.n);
-          last = gs;
+          last = hp;
+          any = true;
         }
       }
-      if (!ok && last >= 0)
-        mbar_wait(bar_halo_full + 8u * static_cast<uint32_t>(last % p.ring),
-                  static_cast<uint32_t>(last / p.ring) & 1u, p.err, kSiteDrain);
+      if (!ok && any) mbar_wait(bar_halo_full + 8u * last.e, last.ph, p.err, kSiteDrain);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
-      uint32_t ga = 0, gb = 0, it = 0;
+      uint32_t it = 0;
+      RingPos ap{0u, 0u}, bp{0u, 0u};
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
-        for (int s = 0; ok && s < p.ks; ++s, ++ga, ++gb) {
-          const uint32_t ea = ga % p.sa, eb = gb % p.sb;
-          if (!wait_or_abort(bar_a_full + 8u * ea, (ga / p.sa) & 1u, p.err, kSiteAStageFull, abort_flag)) {
+        for (int s = 0; ok && s < p.ks;
+             ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
+          const uint32_t ea = ap.e, eb = bp.e;
+          if (!wait_or_abort(bar_a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag)) {
             ok = false;
             break;
           }
-          if (!wait_or_abort(bar_b_full + 8u * eb, (gb / p.sb) & 1u, p.err, kSiteTmaFull, abort_flag)) {
+          if (!wait_or_abort(bar_b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag)) {
             ok = false;
             break;
           }
@@ -571,8 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
-    uint32_t gs_base = 0;  // global slot counter at the start of the tile
-    uint32_t ga = 0;       // global K-slice counter at the start of the tile
+    uint32_t gs_base = 0;       // global halo slot counter at the start of the tile
+    uint32_t gslice = 0;        // global K-slice counter
+    RingPos as{0u, 0u};         // A stage of the current slice
+    RingPos hr{0u, 0u};         // next halo slot this warp hands back
+    const uint32_t ring = static_cast<uint32_t>(p.ring);
     bool ok = true;
     for (int64_t tt = blockIdx.x; ok && tt < p.num_tiles; tt += gridDim.x) {
       const TileCoord tc = decode_tile(p, tt);
@@ -589,25 +608,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       int phi = k0 - c0 * g.taps;
       int q0 = c0 / p.c_slot;
       int cs0 = c0 - q0 * p.c_slot;
+      RingPos h0 = ring_pos(gs_base + static_cast<uint32_t>(q0), ring);  // ring entry of slot q0
       int released = 0;  // halo slots of this tile this warp has handed back
-      for (int s = 0; s < p.ks; ++s) {
-        const uint32_t gslice = ga + static_cast<uint32_t>(s);
-        const uint32_t ea = gslice % p.sa, ua = gslice / p.sa;
-        if (ua > 0 && !wait_or_abort(bar_a_empty + 8u * ea, (ua - 1u) & 1u, p.err, kSiteMmaDone, abort_flag)) {
+      for (int s = 0; s < p.ks; ++s, ++gslice, as.next(static_cast<uint32_t>(p.sa))) {
+        const uint32_t ea = as.e;
+        if (gslice >= static_cast<uint32_t>(p.sa) &&
+            !wait_or_abort(bar_a_empty + 8u * ea, as.ph ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
           ok = false;
           break;
         }
+        RingPos h1 = h0;  // ring entry of slot q0 + 1
+        h1.next(ring);
         const int nvalid = g.K - k0;
         const int split = g.taps - phi;  // columns j >= split belong to channel c0 + 1
         if (nvalid > 0) {
           // the halo slot of channel c0, and the next slot when the block's
           // tail reaches channel c0 + 1 and that channel starts the next slot
-          const int nslots = (split < min(16, nvalid) && cs0 + 1 == p.c_slot) ? 2 : 1;
-          for (int q = q0; ok && q < q0 + nslots; ++q) {
-            const uint32_t gsl = gs_base + static_cast<uint32_t>(q);
-            ok = wait_or_abort(bar_halo_full + 8u * (gsl % p.ring), (gsl / p.ring) & 1u, p.err, kSiteHaloFull,
-                               abort_flag);
-          }
+          ok = wait_or_abort(bar_halo_full + 8u * h0.e, h0.ph, p.err, kSiteHaloFull, abort_flag);
+          if (ok && split < min(16, nvalid) && cs0 + 1 == p.c_slot)
+            ok = wait_or_abort(bar_halo_full + 8u * h1.e, h1.ph, p.err, kSiteHaloFull, abort_flag);
         }
         if (!ok) break;
         tc_fence_after();
@@ -619,15 +638,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < p.n_mt; ++i) tmem_st8(a_col + static_cast<uint32_t>(i * 32), z);
         } else {
           // channel origins of c0 and c0 + 1 in the halo ring
-          const uint32_t e0 = (gs_base + static_cast<uint32_t>(q0)) % static_cast<uint32_t>(p.ring);
-          const uint32_t org0 = halo_base + e0 * p.slot_bytes + static_cast<uint32_t>(cs0) * p.chan_bytes;
-          uint32_t org1;
-          if (cs0 + 1 < p.c_slot) {
-            org1 = org0 + p.chan_bytes;
-          } else {
-            const uint32_t e1 = (gs_base + static_cast<uint32_t>(q0 + 1)) % static_cast<uint32_t>(p.ring);
-            org1 = halo_base + e1 * p.slot_bytes;
-          }
+          const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0) * p.chan_bytes;
+          const uint32_t org1 = (cs0 + 1 < p.c_slot) ? org0 + p.chan_bytes : halo_base + h1.e * p.slot_bytes;
           const int step = static_cast<int>(org1 - org0);
           int off[16];
           const uint32_t prow = phase_tab + static_cast<uint32_t>(phi * 64);
@@ -656,19 +668,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (cs0 >= p.c_slot) {
           cs0 -= p.c_slot;
           ++q0;
+          h0.next(ring);
         }
         if (lane == 0) {
           mbar_arrive(bar_a_full + 8u * ea);
           // Later blocks of this warp start at slot q0 or above: hand the
           // slots below back (a slot is free once all transform warps have).
           const int keep = (s + 1 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
-          for (; released < keep; ++released)
-            mbar_arrive(bar_halo_empty + 8u * ((gs_base + static_cast<uint32_t>(released)) % p.ring));
+          for (; released < keep; ++released, hr.next(ring)) mbar_arrive(bar_halo_empty + 8u * hr.e);
         }
       }
       if (!ok) break;
       gs_base += static_cast<uint32_t>(p.q_slots);
-      ga += static_cast<uint32_t>(p.ks);
     }
   }
 
