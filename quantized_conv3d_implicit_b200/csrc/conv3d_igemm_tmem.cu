@@ -83,7 +83,7 @@ struct TmemParams {
   int sa, sb;
   uint32_t b_stage_bytes;
   int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
-  int dk_c, dk_phi;       // 64 = dk_c * taps + dk_phi
+  int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   uint32_t off_b, off_halo, off_tab, off_phase, off_bar;
 };
 
@@ -368,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_b_empty + 8u * i, 1);
     }
     for (int i = 0; i < p.sa; ++i) {
-      mbar_init(bar_a_full + 8u * i, kNumXfWarps);
+      mbar_init(bar_a_full + 8u * i, kNumXfWarps / 2);  // the 8 warps of the slice's group
       mbar_init(bar_a_empty + 8u * i, 1);
     }
     for (int i = 0; i < kMaxAcc; ++i) {
@@ -546,10 +546,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpXf0) {
     // ------------------------------------------------------------ transform
+    // Two groups of 8 warps take the K slices of alternate global index;
+    // within a group, warp w owns TMEM lane quadrant w % 4 (the lanes its
+    // tcgen05.st may reach) and two adjacent 16-column blocks b0, b0 + 1 of
+    // each of its slices, for every subtile.
     constexpr uint32_t esz = sizeof(T);
     const int xw = warp - kWarpXf0;
     const int quad = warp & 3;                 // TMEM lanes 32*quad..+31
-    const int blk = xw >> 2;                   // 16-column block of every K slice
+    const int grp = xw >> 3;                   // global slices of this parity
+    const int b0 = ((xw >> 2) & 1) * 2;        // first of the warp's two blocks
     const int row = quad * 32 + lane;          // output position within a subtile
     const int th = row / p.TW, tw = row % p.TW;
     const uint32_t halo_base = base + p.off_halo;
@@ -558,9 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int xf_tid = threadIdx.x - kWarpXf0 * 32;
 
     // Per-CTA tables: (scale, 1/scale) for every non-negative E4M3 code, and
-    // for every block phase phi (column index of the block's first column
-    // within its channel) the byte offsets of the 16 taps from the first
-    // tap's channel origin, ignoring the channel step (added per block).
+    // for every block phase phi (column of the block's first element within
+    // its channel) the byte offsets of the block's 16 taps from that
+    // channel's origin, the columns past the channel end taken in the next
+    // channel as if it followed contiguously (chan_bytes further on).
     float t6g = 0.0f;
     {
       const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f};
@@ -578,20 +584,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       int* ph = reinterpret_cast<int*>(smem + p.off_phase);
       for (int i = xf_tid; i < g.taps * 16; i += kNumXfWarps * 32) {
         int t = (i >> 4) + (i & 15);
-        if (t >= g.taps) t -= g.taps;  // taps >= 16: at most one channel step per block
+        int chan = 0;
+        if (t >= g.taps) {  // taps >= 16: at most one channel step per block
+          t -= g.taps;
+          chan = static_cast<int>(p.chan_bytes);
+        }
         const int kw = t % g.KW, r = t / g.KW;
         const int kh = r % g.KH, kd = r / g.KH;
-        ph[i] = (kd * g.dd * p.h_ext * p.w_box + kh * g.dh * p.w_box + kw * g.dw) * static_cast<int>(esz);
+        ph[i] = (kd * g.dd * p.h_ext * p.w_box + kh * g.dh * p.w_box + kw * g.dw) * static_cast<int>(esz) + chan;
       }
       named_bar_sync(1, kNumXfWarps * 32);
     }
 
     const uint32_t lane_field = static_cast<uint32_t>(quad * 32) << 16;
-    uint32_t gs_base = 0;       // global halo slot counter at the start of the tile
-    uint32_t gslice = 0;        // global K-slice counter
-    RingPos as{0u, 0u};         // A stage of the current slice
-    RingPos hr{0u, 0u};         // next halo slot this warp hands back
     const uint32_t ring = static_cast<uint32_t>(p.ring);
+    const int cb = static_cast<int>(p.chan_bytes);
+    uint32_t gs_base = 0;                 // global halo slot counter at the start of the tile
+    uint32_t ga = 0;                      // global K-slice counter at the start of the tile
+    uint32_t gslice = static_cast<uint32_t>(grp);  // global index of this group's next slice
+    RingPos as{static_cast<uint32_t>(grp) % static_cast<uint32_t>(p.sa), 0u};  // its A stage
+    RingPos hr{0u, 0u};                   // next halo slot this warp hands back
     bool ok = true;
     for (int64_t tt = blockIdx.x; ok && tt < p.num_tiles; tt += gridDim.x) {
       const TileCoord tc = decode_tile(p, tt);
@@ -601,65 +613,88 @@ __global__ void __launch_bounds__(kThreads, 1)
       // step to the same position in the next subtile (TH rows further down)
       const uint32_t thr0 = static_cast<uint32_t>((th * g.sh * p.w_box + tw * g.sw + delta) * static_cast<int>(esz));
       const uint32_t thr_step = static_cast<uint32_t>(p.TH * g.sh * p.w_box * static_cast<int>(esz));
-      // block state: first column k0, its channel c0 = (q0 slot, cs0 within
-      // the slot) and phase phi = k0 - c0 * taps
-      int k0 = 16 * blk;
+      // first slice of this tile that belongs to the group, and the state of
+      // block b0 there: first column k0, its channel c0 = (slot q0, cs0
+      // within the slot), phase phi = k0 - c0 * taps, ring entry h0 of q0
+      int s = static_cast<int>((gslice - ga) & 0x7FFFFFFFu);
+      int k0 = kBlockK * s + 16 * b0;
       int c0 = k0 / g.taps;
       int phi = k0 - c0 * g.taps;
       int q0 = c0 / p.c_slot;
       int cs0 = c0 - q0 * p.c_slot;
-      RingPos h0 = ring_pos(gs_base + static_cast<uint32_t>(q0), ring);  // ring entry of slot q0
+      RingPos h0 = ring_pos(gs_base + static_cast<uint32_t>(q0), ring);
       int released = 0;  // halo slots of this tile this warp has handed back
-      for (int s = 0; s < p.ks; ++s, ++gslice, as.next(static_cast<uint32_t>(p.sa))) {
+      for (; s < p.ks; s += 2, gslice += 2, as.next(static_cast<uint32_t>(p.sa)), as.next(static_cast<uint32_t>(p.sa))) {
         const uint32_t ea = as.e;
         if (gslice >= static_cast<uint32_t>(p.sa) &&
             !wait_or_abort(bar_a_empty + 8u * ea, as.ph ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
           ok = false;
           break;
         }
-        RingPos h1 = h0;  // ring entry of slot q0 + 1
-        h1.next(ring);
-        const int nvalid = g.K - k0;
-        const int split = g.taps - phi;  // columns j >= split belong to channel c0 + 1
-        if (nvalid > 0) {
-          // the halo slot of channel c0, and the next slot when the block's
-          // tail reaches channel c0 + 1 and that channel starts the next slot
-          ok = wait_or_abort(bar_halo_full + 8u * h0.e, h0.ph, p.err, kSiteHaloFull, abort_flag);
-          if (ok && split < min(16, nvalid) && cs0 + 1 == p.c_slot)
-            ok = wait_or_abort(bar_halo_full + 8u * h1.e, h1.ph, p.err, kSiteHaloFull, abort_flag);
+        // block b0 + 1 starts 16 columns on (taps >= 16: at most one channel on)
+        int phi1 = phi + 16, cs1 = cs0, q1 = q0;
+        RingPos h1 = h0;
+        if (phi1 >= g.taps) {
+          phi1 -= g.taps;
+          if (++cs1 == p.c_slot) {
+            cs1 = 0;
+            ++q1;
+            h1.next(ring);
+          }
+        }
+        const int nv0 = g.K - k0, nv1 = nv0 - 16;
+        const int split0 = g.taps - phi, split1 = g.taps - phi1;  // columns j >= split are in the next channel
+        const bool cross0 = split0 < min(16, nv0) && cs0 + 1 == p.c_slot;  // next channel starts the next slot
+        const bool cross1 = split1 < min(16, nv1) && cs1 + 1 == p.c_slot;
+        // halo slots the two blocks read: q0 .. q_last
+        if (nv0 > 0) {
+          const int q_last = nv1 > 0 ? q1 + (cross1 ? 1 : 0) : q0 + (cross0 ? 1 : 0);
+          RingPos hw = h0;
+          for (int q = q0; ok && q <= q_last; ++q, hw.next(ring))
+            ok = wait_or_abort(bar_halo_full + 8u * hw.e, hw.ph, p.err, kSiteHaloFull, abort_flag);
         }
         if (!ok) break;
         tc_fence_after();
         const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
-                               ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(blk * 8);
-        if (nvalid <= 0) {
-          // a block entirely past K: zeros (the weights there are zero-filled too)
-          uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          for (int i = 0; i < p.n_mt; ++i) tmem_st8(a_col + static_cast<uint32_t>(i * 32), z);
-        } else {
-          // channel origins of c0 and c0 + 1 in the halo ring
-          const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0) * p.chan_bytes;
-          const uint32_t org1 = (cs0 + 1 < p.c_slot) ? org0 + p.chan_bytes : halo_base + h1.e * p.slot_bytes;
-          const int step = static_cast<int>(org1 - org0);
+                               ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
+#pragma unroll 1
+        for (int bb = 0; bb < 2; ++bb) {
+          const int nv = bb ? nv1 : nv0;
+          const uint32_t colb = a_col + 8u * static_cast<uint32_t>(bb);
+          if (nv <= 0) {
+            // a block entirely past K: zeros (the weights there are zero-filled too)
+            uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            for (int i = 0; i < p.n_mt; ++i) tmem_st8(colb + static_cast<uint32_t>(i * 32), z);
+            continue;
+          }
+          const int phb = bb ? phi1 : phi, csb = bb ? cs1 : cs0, splitb = bb ? split1 : split0;
+          const RingPos hb = bb ? h1 : h0;
+          const uint32_t org = halo_base + hb.e * p.slot_bytes + static_cast<uint32_t>(csb * cb);
           int off[16];
-          const uint32_t prow = phase_tab + static_cast<uint32_t>(phi * 64);
+          const uint32_t prow = phase_tab + static_cast<uint32_t>(phb * 64);
 #pragma unroll
           for (int j = 0; j < 16; j += 4) ld_shared_v4(prow + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
+          if (bb ? cross1 : cross0) {
+            // the next channel opens the next ring slot: move its columns there
+            RingPos hn = hb;
+            hn.next(ring);
+            const int adj = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org) - cb;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) off[j] += (j >= split) ? step : 0;
+            for (int j = 0; j < 16; ++j) off[j] += (j >= splitb) ? adj : 0;
+          }
           for (int i = 0; i < p.n_mt; ++i) {
             uint32_t w[8];
-            row_block<T>(org0 + thr0 + static_cast<uint32_t>(i) * thr_step, off, nvalid, p.quant != 0, t6g, tab, w);
-            tmem_st8(a_col + static_cast<uint32_t>(i * 32), w);
+            row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, p.quant != 0, t6g, tab, w);
+            tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
           }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        // next slice: the block moves 64 columns on
-        k0 += kBlockK;
-        phi += p.dk_phi;
-        int dc = p.dk_c;
+        // this warp's next slice is two on: its blocks move 128 columns
+        k0 += 2 * kBlockK;
+        phi += p.dk2_phi;
+        int dc = p.dk2_c;
         if (phi >= g.taps) {
           phi -= g.taps;
           ++dc;
@@ -674,12 +709,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar_a_full + 8u * ea);
           // Later blocks of this warp start at slot q0 or above: hand the
           // slots below back (a slot is free once all transform warps have).
-          const int keep = (s + 1 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
+          const int keep = (s + 2 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
           for (; released < keep; ++released, hr.next(ring)) mbar_arrive(bar_halo_empty + 8u * hr.e);
         }
       }
       if (!ok) break;
+      if (lane == 0)  // a tile with no slice for this group (ks == 1) still hands its slots back
+        for (; released < p.q_slots; ++released, hr.next(ring)) mbar_arrive(bar_halo_empty + 8u * hr.e);
       gs_base += static_cast<uint32_t>(p.q_slots);
+      ga += static_cast<uint32_t>(p.ks);
     }
   }
 
@@ -766,8 +804,8 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   p.ks = ceil_div(g.K, kBlockK);
   p.num_tiles = static_cast<int64_t>(g.N) * g.OD * p.n_ohb * p.n_owb * n_ntiles;
   p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
-  p.dk_c = kBlockK / g.taps;
-  p.dk_phi = kBlockK - p.dk_c * g.taps;
+  p.dk2_c = 2 * kBlockK / g.taps;
+  p.dk2_phi = 2 * kBlockK - p.dk2_c * g.taps;
 
   const int chan_bytes = static_cast<int>(p.chan_bytes);
   const int phase_bytes = g.taps * 64;
@@ -816,7 +854,7 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   TmemParams p{};
   size_t smem = 0;
   const bool ok = plan_tmem(g, dtype, p, smem);
-  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 1, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
+  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));

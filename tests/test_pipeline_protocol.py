@@ -88,7 +88,7 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
             released = 0
             for s in range(ks):
                 ea, eb = ga % sa, gb % sb
-                yield ("wait", bar("a_full", ea, wpg), ga // sa)
+                yield ("wait", bar("a_full", ea, 8 if kernel == "tmem" else wpg), ga // sa)
                 keep = slot_lo(s + 1) if s + 1 < ks else q_slots
                 while not xf_release and released < keep:
                     yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
@@ -158,11 +158,61 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
             ga += ks
             gs_base += q_slots
 
+    def transform_tmem(w):
+        # tensor-memory kernel: group w >> 3 takes the global slices of its
+        # parity; warp w handles blocks b0, b0 + 1 of each, waits for the halo
+        # slots those read and hands back the slots below its next pair
+        grp, b0 = w >> 3, ((w >> 2) & 1) * 2
+        gs_base = ga = 0
+        gslice = grp
+        hr = 0  # next global slot to hand back
+        for _ in range(ntiles):
+            s = gslice - ga
+            released = 0
+            while s < ks:
+                ea, ua = gslice % sa, gslice // sa
+                if gslice >= sa:
+                    yield ("wait", bar("a_empty", ea, 1), ua - 1)
+                k0 = 64 * s + 16 * b0
+                if k0 < K:
+                    c0, phi = divmod(k0, taps)
+                    q0, cs0 = divmod(c0, c_slot)
+                    phi1, cs1, q1 = phi + 16, cs0, q0
+                    if phi1 >= taps:
+                        phi1 -= taps
+                        cs1 += 1
+                        if cs1 == c_slot:
+                            cs1, q1 = 0, q1 + 1
+                    nv0, nv1 = K - k0, K - k0 - 16
+                    cross0 = (taps - phi) < min(16, nv0) and cs0 + 1 == c_slot
+                    cross1 = (taps - phi1) < min(16, nv1) and cs1 + 1 == c_slot
+                    q_last = q1 + int(cross1) if nv1 > 0 else q0 + int(cross0)
+                    for q in range(q0, q_last + 1):
+                        g = gs_base + q
+                        yield ("wait", bar("halo_full", g % ring, 1), g // ring)
+                yield ("arrive", bar("a_full", ea, 8))
+                if s + 2 < ks:
+                    keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot, q_slots)
+                else:
+                    keep = q_slots
+                while released < keep:
+                    yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
+                    released += 1
+                    hr += 1
+                s += 2
+                gslice += 2
+            while released < q_slots:
+                yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
+                released += 1
+                hr += 1
+            gs_base += q_slots
+            ga += ks
+
     r = {"halo": halo_producer(), "weights": weight_producer(), "mma": mma()}
     for w in range(4):
         r[f"epilogue{w}"] = epilogue()
     for w in range(n_xf):
-        r[f"transform{w}"] = transform(w)
+        r[f"transform{w}"] = transform_tmem(w) if kernel == "tmem" else transform(w)
     return r
 
 
@@ -271,7 +321,7 @@ def test_sim_detects_aliasing_when_stages_fewer_than_groups():
 
 
 def _check_tmem_invariants(p, taps):
-    assert p["groups"] == 1 and p["tmem_cols"] == 512 and taps >= 16
+    assert p["groups"] == 2 and p["tmem_cols"] == 512 and taps >= 16
     # accumulators [0, n_mt*n_tile), then sa A stages of n_mt * 32 columns
     assert p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
     assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512 and p["sa"] >= 2
