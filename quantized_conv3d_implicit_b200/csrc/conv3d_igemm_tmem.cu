@@ -195,8 +195,9 @@ template <typename T>
 struct Half2;
 template <>
 struct Half2<__nv_bfloat16> {
-  static __device__ __forceinline__ float abs_lo(uint32_t w) { return __uint_as_float((w << 16) & 0x7FFFFFFFu); }
-  static __device__ __forceinline__ float abs_hi(uint32_t w) { return __uint_as_float(w & 0x7FFF0000u); }
+  // |x| as an operand modifier of the consuming multiply or max
+  static __device__ __forceinline__ float abs_lo(uint32_t w) { return fabsf(__uint_as_float(w << 16)); }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) { return fabsf(__uint_as_float(w & 0xFFFF0000u)); }
   static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_bf16x2(a, b); }
   static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
 };
