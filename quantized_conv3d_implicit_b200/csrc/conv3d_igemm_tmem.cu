@@ -333,7 +333,56 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
   }
 }
 
+// Two rows (the same output position in two subtiles) of one full 16-column
+// block of a 16-bit input, sharing the tap offsets: the two load, maximum,
+// scale and dequantisation chains are interleaved so each hides the other's
+// latency.  Same results as two row_block calls.
 template <typename T>
+__device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, const int (&off)[16], bool quant,
+                                             float t6g, uint32_t tab, uint32_t (&out_a)[8], uint32_t (&out_b)[8]) {
+  static_assert(sizeof(T) == 2, "16-bit inputs only");
+  uint32_t pa[8], pb[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t a0 = ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i]));
+    const uint32_t b0 = ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i]));
+    const uint32_t a1 = ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i + 1]));
+    const uint32_t b1 = ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i + 1]));
+    pa[i] = __byte_perm(a0, a1, 0x5410);
+    pb[i] = __byte_perm(b0, b1, 0x5410);
+  }
+  if (!quant) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      out_a[i] = Half2<T>::to_bf16x2(pa[i]);
+      out_b[i] = Half2<T>::to_bf16x2(pb[i]);
+    }
+    return;
+  }
+  uint32_t ma = Half2<T>::maxabs(Half2<T>::maxabs(pa[0], pa[1]), Half2<T>::maxabs(pa[2], pa[3]));
+  uint32_t mb = Half2<T>::maxabs(Half2<T>::maxabs(pb[0], pb[1]), Half2<T>::maxabs(pb[2], pb[3]));
+  ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
+  mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
+  float sa, ia, sb, ib;
+  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), t6g, tab, sa, ia);
+  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), t6g, tab, sb, ib);
+  const DqTable da = dq_table(sa), db = dq_table(sb);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a0 = pa[2 * i], a1 = pa[2 * i + 1], b0 = pb[2 * i], b1 = pb[2 * i + 1];
+    dq4(da, __fmul_rn(Half2<T>::abs_lo(a0), ia), __fmul_rn(Half2<T>::abs_hi(a0), ia),
+        __fmul_rn(Half2<T>::abs_lo(a1), ia), __fmul_rn(Half2<T>::abs_hi(a1), ia), a0, a1, out_a[2 * i],
+        out_a[2 * i + 1]);
+    dq4(db, __fmul_rn(Half2<T>::abs_lo(b0), ib), __fmul_rn(Half2<T>::abs_hi(b0), ib),
+        __fmul_rn(Half2<T>::abs_lo(b1), ib), __fmul_rn(Half2<T>::abs_hi(b1), ib), b0, b1, out_b[2 * i],
+        out_b[2 * i + 1]);
+  }
+}
+
+// kPairs: the tile has at least two M-subtiles, built in interleaved pairs
+// (a separate instantiation, so single-subtile tiles keep their register
+// allocation).
+template <typename T, bool kPairs>
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
                              const __grid_constant__ CUtensorMap tmap_w) {
@@ -683,7 +732,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) off[j] += (j >= splitb) ? adj : 0;
           }
-          for (int i = 0; i < p.n_mt; ++i) {
+          int i = 0;
+          if constexpr (kPairs && sizeof(T) == 2) {
+            // full blocks, subtiles in pairs: interleaved chains
+            if (nv >= 16)
+              for (; i + 1 < p.n_mt; i += 2) {
+                uint32_t wa[8], wb[8];
+                const uint32_t ra = org + thr0 + static_cast<uint32_t>(i) * thr_step;
+                row_block_x2<T>(ra, ra + thr_step, off, p.quant != 0, t6g, tab, wa, wb);
+                tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
+                tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
+              }
+          }
+          for (; i < p.n_mt; ++i) {
             uint32_t w[8];
             row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, p.quant != 0, t6g, tab, w);
             tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
@@ -732,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <typename T>
 cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                               size_t smem, cudaStream_t s) {
-  auto kern = conv3d_igemm_tmem_kernel<T>;
+  auto kern = p.n_mt >= 2 ? conv3d_igemm_tmem_kernel<T, true> : conv3d_igemm_tmem_kernel<T, false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
