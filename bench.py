@@ -43,7 +43,7 @@ L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-KERNEL_SOURCES = ("conv3d_igemm_fast.cu", "sm100_ptx.cuh", "nvfp4.cuh")
+KERNEL_SOURCES = ("conv3d_igemm_tmem.cu", "sm100_ptx.cuh", "nvfp4.cuh")
 
 
 def profiled_traffic(workload: str):
@@ -51,7 +51,7 @@ def profiled_traffic(workload: str):
     summary of this workload, or None when there is none or the kernel
     sources have changed since it was captured (sha256 recorded beside it)."""
     import hashlib
-    p = os.path.join(ROOT, "profiles", f"conv3d_igemm_fast_{workload}.md")
+    p = os.path.join(ROOT, "profiles", f"conv3d_igemm_tmem_{workload}.md")
     try:
         with open(p) as f:
             text = f.read()
@@ -282,7 +282,7 @@ def run_ours(args, world, rank, local):
         "roofline": {
             "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(conv_tflops / peak, 4), "traffic": profiled_traffic(wl.name),
-            "kernel": "conv3d_igemm (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
+            "kernel": "conv3d_igemm_tmem (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
         },
         "clocks": clocks,
         "e2e": e2e,
