@@ -84,6 +84,8 @@ struct TmemParams {
   uint32_t b_stage_bytes;
   int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
   int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
+  int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
+  int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
   uint32_t off_b, off_halo, off_tab, off_phase, off_bar;
 };
 
@@ -633,12 +635,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int* ph = reinterpret_cast<int*>(smem + p.off_phase);
       for (int i = xf_tid; i < g.taps * 16; i += kNumXfWarps * 32) {
-        int t = (i >> 4) + (i & 15);
-        int chan = 0;
-        if (t >= g.taps) {  // taps >= 16: at most one channel step per block
-          t -= g.taps;
-          chan = static_cast<int>(p.chan_bytes);
-        }
+        const int tt = (i >> 4) + (i & 15);
+        const int nch = tt / g.taps;  // channels past the block's first one
+        const int t = tt - nch * g.taps;
+        const int chan = nch * static_cast<int>(p.chan_bytes);
         const int kw = t % g.KW, r = t / g.KW;
         const int kh = r % g.KH, kd = r / g.KH;
         ph[i] = (kd * g.dd * p.h_ext * p.w_box + kh * g.dh * p.w_box + kw * g.dw) * static_cast<int>(esz) + chan;
@@ -681,21 +681,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // block b0 + 1 starts 16 columns on (taps >= 16: at most one channel on)
-        int phi1 = phi + 16, cs1 = cs0, q1 = q0;
+        // block b0 + 1 starts 16 columns on
+        int phi1 = phi + p.dk16_phi, cs1 = cs0 + p.dk16_c, q1 = q0;
         RingPos h1 = h0;
         if (phi1 >= g.taps) {
           phi1 -= g.taps;
-          if (++cs1 == p.c_slot) {
-            cs1 = 0;
-            ++q1;
-            h1.next(ring);
-          }
+          ++cs1;
+        }
+        while (cs1 >= p.c_slot) {
+          cs1 -= p.c_slot;
+          ++q1;
+          h1.next(ring);
         }
         const int nv0 = g.K - k0, nv1 = nv0 - 16;
         const int split0 = g.taps - phi, split1 = g.taps - phi1;  // columns j >= split are in the next channel
-        const bool cross0 = split0 < min(16, nv0) && cs0 + 1 == p.c_slot;  // next channel starts the next slot
-        const bool cross1 = split1 < min(16, nv1) && cs1 + 1 == p.c_slot;
+        // the block's second channel opens the next slot (never with slot-aligned blocks)
+        const bool cross0 = !p.slot_aligned && split0 < min(16, nv0) && cs0 + 1 == p.c_slot;
+        const bool cross1 = !p.slot_aligned && split1 < min(16, nv1) && cs1 + 1 == p.c_slot;
         // halo slots the two blocks read: q0 .. q_last
         if (nv0 > 0) {
           const int q_last = nv1 > 0 ? q1 + (cross1 ? 1 : 0) : q0 + (cross0 ? 1 : 0);
@@ -805,23 +807,24 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 }  // namespace
 
 // Tiling and pipeline plan of the tensor-memory kernel (pure host
-// arithmetic).  Returns false when the kernel does not apply: fewer than 16
-// taps (a 16-column block would span more than two channels), rows of x not
-// a multiple of 16 bytes (TMA stride rule), or no plan that fits.
+// arithmetic).  Returns false when the kernel does not apply: rows of x not
+// a multiple of 16 bytes (TMA stride rule), more than 343 taps, or no plan
+// that fits.
 static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem) {
   const int esz = dtype == 0 ? 4 : 2;
   const int align = 16 / esz;
   if ((static_cast<int64_t>(g.W) * esz) % 16 != 0) return false;
-  if (g.taps < 16 || g.taps > kMaxTaps) return false;
+  if (g.taps > kMaxTaps) return false;
   memset(&p, 0, sizeof(p));
   p.g = g;
   p.align = align;
 
   // output channels per tile: all of Cout up to 448 (448 + two 32-column A
-  // stages fill the 512 TMEM columns), else tiles of at most 256
+  // stages fill the 512 TMEM columns), else the fewest equal tiles of at
+  // most 448 (each N-tile rebuilds the A operand)
   int n_ntiles = 1, n_tile = (g.Cout + 15) / 16 * 16;
   if (n_tile > 448) {
-    n_ntiles = ceil_div(g.Cout, 256);
+    n_ntiles = ceil_div(g.Cout, 448);
     n_tile = (ceil_div(g.Cout, n_ntiles) + 15) / 16 * 16;
   }
   const int n_sub = ceil_div(n_tile, 256);
@@ -868,6 +871,19 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
   p.dk2_c = 2 * kBlockK / g.taps;
   p.dk2_phi = 2 * kBlockK - p.dk2_c * g.taps;
+  p.dk16_c = 16 / g.taps;
+  p.dk16_phi = 16 - p.dk16_c * g.taps;
+  // Fewer than 16 taps: a block spans several channels, so slots hold a
+  // multiple of cm channels (c_slot * taps a multiple of 16) and no block
+  // straddles two slots.  From 16 taps on a block spans at most two
+  // channels and may straddle; the transform then moves the second
+  // channel's columns to the next slot.
+  int cm = 1;
+  if (g.taps < 16) {
+    int a = g.taps, b = 16;
+    while (b) { const int r = a % b; a = b; b = r; }
+    cm = 16 / a;
+  }
 
   const int chan_bytes = static_cast<int>(p.chan_bytes);
   const int phase_bytes = g.taps * 64;
@@ -877,34 +893,40 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   // weight stages buys further slots (more halo loads in flight).
   for (int target = 10240; target >= 1; target = (target > chan_bytes ? target / 2 : 0)) {
     p.c_slot = std::max(1, std::min(std::min(256, g.C), target / chan_bytes));
+    if (cm > 1) p.c_slot = std::min(256 / cm * cm, (p.c_slot + cm - 1) / cm * cm);
+    p.slot_aligned = (p.c_slot * g.taps) % 16 == 0 ? 1 : 0;
     p.q_slots = ceil_div(g.C, p.c_slot);
     p.slot_tx = static_cast<uint32_t>(p.c_slot) * p.chan_bytes;
     p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
-    int span = 1;
-    for (int s0 = 0; s0 < p.ks; ++s0) {
-      const int lo = ((kBlockK * s0) / g.taps) / p.c_slot;
-      const int hi = (std::min(kBlockK * (s0 + p.sa) - 1, g.K - 1) / g.taps) / p.c_slot;
-      span = std::max(span, hi - lo + 1);
-    }
-    for (int b = 8; b >= 2; --b) {
-      int r = span + 2;
-      const int nbar = 2 * r + 2 * b + 2 * p.sa + 2 * kMaxAcc + 1;
-      int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
-                        64 /* pad after the halo ring */ + 1024 /* scale table */ + phase_bytes + nbar * 8 + 16;
-      if (total <= kMaxSmem) {
-        const int extra = std::min(32 - r, (kMaxSmem - total) / (static_cast<int>(p.slot_bytes) + 16));
-        if (extra > 0) {
-          r += extra;
-          total += extra * (static_cast<int>(p.slot_bytes) + 16);
+    // fewer A stages shrink the halo window the ring must cover
+    const int sa_max = std::min(4, stages_of(bMT));
+    for (int a = sa_max; a >= 2; --a) {
+      int span = 1;
+      for (int s0 = 0; s0 < p.ks; ++s0) {
+        const int lo = ((kBlockK * s0) / g.taps) / p.c_slot;
+        const int hi = (std::min(kBlockK * (s0 + a) - 1, g.K - 1) / g.taps) / p.c_slot;
+        span = std::max(span, hi - lo + 1);
+      }
+      for (int b = 8; b >= 2; --b) {
+        int r = span + 2;
+        const int nbar = 2 * r + 2 * b + 2 * a + 2 * kMaxAcc + 1;
+        int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
+                    64 /* pad after the halo ring */ + 1024 /* scale table */ + phase_bytes + nbar * 8 + 16;
+        if (total <= kMaxSmem) {
+          const int extra = std::min(32 - r, (kMaxSmem - total) / (static_cast<int>(p.slot_bytes) + 16));
+          if (extra > 0) {
+            r += extra;
+            total += extra * (static_cast<int>(p.slot_bytes) + 16);
+          }
+          p.sa = a; p.sb = b; p.ring = r;
+          p.off_b = 0;
+          p.off_halo = p.off_b + b * p.b_stage_bytes;
+          p.off_tab = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
+          p.off_phase = p.off_tab + 1024u;
+          p.off_bar = p.off_phase + static_cast<uint32_t>(phase_bytes);
+          smem = static_cast<size_t>(total);
+          return true;
         }
-        p.sb = b; p.ring = r;
-        p.off_b = 0;
-        p.off_halo = p.off_b + b * p.b_stage_bytes;
-        p.off_tab = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
-        p.off_phase = p.off_tab + 1024u;
-        p.off_bar = p.off_phase + static_cast<uint32_t>(phase_bytes);
-        smem = static_cast<size_t>(total);
-        return true;
       }
     }
     if (p.c_slot == 1) break;

@@ -177,15 +177,12 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
                 if k0 < K:
                     c0, phi = divmod(k0, taps)
                     q0, cs0 = divmod(c0, c_slot)
-                    phi1, cs1, q1 = phi + 16, cs0, q0
-                    if phi1 >= taps:
-                        phi1 -= taps
-                        cs1 += 1
-                        if cs1 == c_slot:
-                            cs1, q1 = 0, q1 + 1
+                    c1, phi1 = divmod(k0 + 16, taps)
+                    q1, cs1 = divmod(c1, c_slot)
                     nv0, nv1 = K - k0, K - k0 - 16
-                    cross0 = (taps - phi) < min(16, nv0) and cs0 + 1 == c_slot
-                    cross1 = (taps - phi1) < min(16, nv1) and cs1 + 1 == c_slot
+                    aligned = (c_slot * taps) % 16 == 0   # no block straddles two slots
+                    cross0 = not aligned and (taps - phi) < min(16, nv0) and cs0 + 1 == c_slot
+                    cross1 = not aligned and (taps - phi1) < min(16, nv1) and cs1 + 1 == c_slot
                     q_last = q1 + int(cross1) if nv1 > 0 else q0 + int(cross0)
                     for q in range(q0, q_last + 1):
                         g = gs_base + q
@@ -321,7 +318,10 @@ def test_sim_detects_aliasing_when_stages_fewer_than_groups():
 
 
 def _check_tmem_invariants(p, taps):
-    assert p["groups"] == 2 and p["tmem_cols"] == 512 and taps >= 16
+    assert p["groups"] == 2 and p["tmem_cols"] == 512
+    if taps < 16:
+        # a block spans several channels: slots must hold whole blocks
+        assert (p["c_slot"] * taps) % 16 == 0
     # accumulators [0, n_mt*n_tile), then sa A stages of n_mt * 32 columns
     assert p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
     assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512 and p["sa"] >= 2
@@ -335,9 +335,6 @@ def _check_tmem_invariants(p, taps):
 @pytest.mark.parametrize("order", ["rr", "rev", "random"])
 def test_tmem_kernel_plans_are_deadlock_and_alias_free(name, order):
     plan, K, taps = _plan(workloads.WORKLOADS[name], kernel="tmem")
-    if taps < 16:
-        assert plan["applicable"] == 0
-        return
     assert plan["applicable"] == 1
     _check_tmem_invariants(plan, taps)
     run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)), kernel="tmem")
@@ -347,7 +344,8 @@ def test_tmem_kernel_random_shapes():
     rng = random.Random(11)
     checked = 0
     for _ in range(80):
-        k = rng.choice([(3, 3, 3), (5, 5, 5), (3, 3, 2), (1, 5, 5), (2, 3, 3)])
+        k = rng.choice([(3, 3, 3), (5, 5, 5), (3, 3, 2), (1, 5, 5), (2, 3, 3), (1, 1, 1), (1, 3, 3), (3, 1, 1),
+                        (2, 2, 2), (1, 2, 2)])
         cin = rng.choice([1, 3, 8, 16, 37, 64, 96, 192, 256])
         cout = rng.choice([1, 8, 16, 40, 96, 100, 192, 256, 300, 384, 448, 512, 640, 1024])
         xs = (rng.choice([1, 2]), cin, rng.randint(k[0], 9), rng.randint(k[1], 40), 8 * rng.randint(1, 30))
@@ -368,6 +366,15 @@ def test_tmem_kernel_random_shapes():
     assert checked >= 40
 
 
-def test_tmem_kernel_declines_fewer_than_16_taps():
-    plan, _, _ = _plan(((1, 64, 4, 16, 16), (64, 64, 1, 3, 3), 1, 1, 1, torch.bfloat16), kernel="tmem")
+@pytest.mark.parametrize("kshape", [(1, 1, 1), (1, 3, 3), (3, 1, 1), (2, 2, 2)])
+def test_tmem_kernel_plans_blocks_within_one_slot_below_16_taps(kshape):
+    taps = kshape[0] * kshape[1] * kshape[2]
+    plan, K, _ = _plan(((1, 64, 4, 16, 16), (64, 64) + kshape, 1, 0, 1, torch.bfloat16), kernel="tmem")
+    assert plan["applicable"] == 1
+    assert (plan["c_slot"] * taps) % 16 == 0
+    run(plan, K, taps, ntiles=2, order="rr", kernel="tmem")
+
+
+def test_tmem_kernel_declines_unaligned_rows():
+    plan, _, _ = _plan(((1, 8, 4, 16, 12), (8, 8, 3, 3, 3), 1, 1, 1, torch.bfloat16), kernel="tmem")
     assert plan["applicable"] == 0 and plan["TW"] == 0
