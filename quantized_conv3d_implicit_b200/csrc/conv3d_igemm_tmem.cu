@@ -381,6 +381,63 @@ __device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, c
   }
 }
 
+// Two full 16-column blocks of one row (a transform warp's pair b0, b0 + 1
+// in a single-subtile tile) of a 16-bit input, each with its own channel
+// origin and phase-table row; the two chains are interleaved.  Each block's
+// tap offsets are read just before its gathers to keep register use low.
+// Same results as two row_block calls.
+template <typename T>
+__device__ __forceinline__ void row_block_2b(uint32_t addr_a, uint32_t prow_a, uint32_t addr_b, uint32_t prow_b,
+                                             bool quant, float t6g, uint32_t tab, uint32_t (&out_a)[8],
+                                             uint32_t (&out_b)[8]) {
+  static_assert(sizeof(T) == 2, "16-bit inputs only");
+  uint32_t pa[8], pb[8];
+  {
+    int off[16];
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) ld_shared_v4(prow_a + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      pa[i] = __byte_perm(ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i])),
+                          ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i + 1])), 0x5410);
+  }
+  {
+    int off[16];
+#pragma unroll
+    for (int j = 0; j < 16; j += 4) ld_shared_v4(prow_b + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      pb[i] = __byte_perm(ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i])),
+                          ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i + 1])), 0x5410);
+  }
+  if (!quant) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      out_a[i] = Half2<T>::to_bf16x2(pa[i]);
+      out_b[i] = Half2<T>::to_bf16x2(pb[i]);
+    }
+    return;
+  }
+  uint32_t ma = Half2<T>::maxabs(Half2<T>::maxabs(pa[0], pa[1]), Half2<T>::maxabs(pa[2], pa[3]));
+  uint32_t mb = Half2<T>::maxabs(Half2<T>::maxabs(pb[0], pb[1]), Half2<T>::maxabs(pb[2], pb[3]));
+  ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
+  mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
+  float sa, ia, sb, ib;
+  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), t6g, tab, sa, ia);
+  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), t6g, tab, sb, ib);
+  const DqTable da = dq_table(sa), db = dq_table(sb);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t a0 = pa[2 * i], a1 = pa[2 * i + 1], b0 = pb[2 * i], b1 = pb[2 * i + 1];
+    dq4(da, __fmul_rn(Half2<T>::abs_lo(a0), ia), __fmul_rn(Half2<T>::abs_hi(a0), ia),
+        __fmul_rn(Half2<T>::abs_lo(a1), ia), __fmul_rn(Half2<T>::abs_hi(a1), ia), a0, a1, out_a[2 * i],
+        out_a[2 * i + 1]);
+    dq4(db, __fmul_rn(Half2<T>::abs_lo(b0), ib), __fmul_rn(Half2<T>::abs_hi(b0), ib),
+        __fmul_rn(Half2<T>::abs_lo(b1), ib), __fmul_rn(Half2<T>::abs_hi(b1), ib), b0, b1, out_b[2 * i],
+        out_b[2 * i + 1]);
+  }
+}
+
 // kPairs: the tile has at least two M-subtiles, built in interleaved pairs
 // (a separate instantiation, so single-subtile tiles keep their register
 // allocation).
@@ -709,8 +766,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
                                ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
+        bool pair_done = false;
+        if constexpr (!kPairs && sizeof(T) == 2) {
+          // single subtile, both blocks full and within their slots: one interleaved pass
+          if (nv0 >= 32 && !cross0 && !cross1) {
+            uint32_t wa[8], wb[8];
+            row_block_2b<T>(halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0,
+                            phase_tab + static_cast<uint32_t>(phi * 64),
+                            halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb) + thr0,
+                            phase_tab + static_cast<uint32_t>(phi1 * 64), p.quant != 0, t6g, tab, wa, wb);
+            tmem_st8(a_col, wa);
+            tmem_st8(a_col + 8u, wb);
+            pair_done = true;
+          }
+        }
 #pragma unroll 1
-        for (int bb = 0; bb < 2; ++bb) {
+        for (int bb = 0; bb < 2 && !pair_done; ++bb) {
           const int nv = bb ? nv1 : nv0;
           const uint32_t colb = a_col + 8u * static_cast<uint32_t>(bb);
           if (nv <= 0) {
