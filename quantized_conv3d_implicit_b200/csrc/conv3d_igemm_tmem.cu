@@ -438,6 +438,74 @@ __device__ __forceinline__ void row_block_2b(uint32_t addr_a, uint32_t prow_a, u
   }
 }
 
+struct MmaBars {
+  uint32_t a_full, b_full, a_empty, b_empty, acc_full, acc_empty, drain;
+};
+
+// The MMA issuer: per K slice, wait for the A stage and the weight stage,
+// issue n_mt x n_sub x 4 tcgen05.mma (A from TMEM, B from shared memory,
+// K = 16 each), commit the accumulators after the tile's last slice and the
+// two stages after every slice.  NMT / NSUB fix the subtile and N-part
+// counts at compile time (0: taken from the plan), so the common shapes
+// issue straight-line code.
+template <int NMT, int NSUB>
+__device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t base, uint32_t tmem_base,
+                                               const MmaBars& b, volatile int* abort_flag) {
+  const int n_mt = NMT ? NMT : p.n_mt;
+  const int n_sub = NSUB ? NSUB : p.n_sub;
+  const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
+  const uint32_t sub_cols = static_cast<uint32_t>(p.sub_n);
+  const uint32_t tile_cols = static_cast<uint32_t>(p.n_tile);
+  const uint64_t bsub_step = static_cast<uint64_t>(p.sub_n * 8);  // descriptor units of 16 B
+  uint32_t it = 0;
+  RingPos ap{0u, 0u}, bp{0u, 0u};
+  bool ok = true;
+  for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+    for (int s = 0; ok && s < p.ks; ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
+      const uint32_t ea = ap.e, eb = bp.e;
+      if (!wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) ||
+          !wait_or_abort(b.b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a_stage = tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(n_mt * 32);
+      const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
+      const bool first = (s == 0), last = (s == p.ks - 1);
+#pragma unroll
+      for (int i = 0; i < (NMT ? NMT : 4); ++i) {
+        if (!NMT && i >= n_mt) break;
+#pragma unroll
+        for (int ns = 0; ns < (NSUB ? NSUB : 2); ++ns) {
+          if (!NSUB && ns >= n_sub) break;
+          const int acc = i * n_sub + ns;
+          if (first && it > 0 && ok) {
+            ok = wait_or_abort(b.acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag);
+            tc_fence_after();
+          }
+          if (ok) {
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i) * tile_cols + static_cast<uint32_t>(ns) * sub_cols;
+            const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
+            const uint64_t bsub = bdesc + static_cast<uint64_t>(ns) * bsub_step;
+#pragma unroll
+            for (int j = 0; j < kBlockK / 16; ++j)
+              umma_bf16_ts(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
+                           (first && j == 0) ? 0u : 1u);
+            if (last) umma_commit(b.acc_full + 8u * acc);
+          }
+        }
+      }
+      if (!ok) break;
+      umma_commit(b.a_empty + 8u * ea);
+      umma_commit(b.b_empty + 8u * eb);
+    }
+  }
+  if (!ok) {
+    umma_commit(b.drain);
+    mbar_wait(b.drain, 0, p.err, kSiteDrain);
+  }
+}
+
 // kPairs: the tile has at least two M-subtiles, built in interleaved pairs
 // (a separate instantiation, so single-subtile tiles keep their register
 // allocation).
@@ -553,53 +621,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
-      uint32_t it = 0;
-      RingPos ap{0u, 0u}, bp{0u, 0u};
-      bool ok = true;
-      for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
-        for (int s = 0; ok && s < p.ks;
-             ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
-          const uint32_t ea = ap.e, eb = bp.e;
-          if (!wait_or_abort(bar_a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag)) {
-            ok = false;
-            break;
-          }
-          if (!wait_or_abort(bar_b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_stage = tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(p.n_mt * 32);
-          const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
-          for (int i = 0; ok && i < p.n_mt; ++i) {
-            const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
-            for (int ns = 0; ns < p.n_sub; ++ns) {
-              const int acc = i * p.n_sub + ns;
-              if (s == 0 && it > 0) {
-                if (!wait_or_abort(bar_acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-              }
-              const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
-              const uint64_t bsub = bdesc + static_cast<uint64_t>(ns * p.sub_n * 8);
-#pragma unroll
-              for (int j = 0; j < kBlockK / 16; ++j)
-                umma_bf16_ts(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
-                             (s > 0 || j > 0) ? 1u : 0u);
-              if (s == p.ks - 1) umma_commit(bar_acc_full + 8u * acc);
-            }
-          }
-          if (!ok) break;
-          umma_commit(bar_a_empty + 8u * ea);
-          umma_commit(bar_b_empty + 8u * eb);
-        }
-      }
-      if (!ok) {
-        umma_commit(bar_drain);
-        mbar_wait(bar_drain, 0, p.err, kSiteDrain);
+      const MmaBars bars{bar_a_full, bar_b_full, bar_a_empty, bar_b_empty, bar_acc_full, bar_acc_empty, bar_drain};
+      switch (p.n_mt * 4 + p.n_sub) {  // straight-line issue for the common shapes
+        case 1 * 4 + 1: mma_issue_loop<1, 1>(p, base, tmem_base, bars, abort_flag); break;
+        case 1 * 4 + 2: mma_issue_loop<1, 2>(p, base, tmem_base, bars, abort_flag); break;
+        case 2 * 4 + 1: mma_issue_loop<2, 1>(p, base, tmem_base, bars, abort_flag); break;
+        case 2 * 4 + 2: mma_issue_loop<2, 2>(p, base, tmem_base, bars, abort_flag); break;
+        default: mma_issue_loop<0, 0>(p, base, tmem_base, bars, abort_flag); break;
       }
     }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
