@@ -65,6 +65,7 @@ SHAPES = [
     ((1, 3, 7, 9, 16), 8, (5, 5, 5), (1, 1, 1), (2, 2, 2), (2, 2, 2), (1, 1, 1)),      # 5x5x5, K=375
     ((1, 8, 3, 6, 8), 500, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # two N tiles
     ((1, 20, 3, 21, 40), 200, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1)),  # K=540, N=208
+    ((1, 8, 3, 8, 32), 192, (3, 3, 3), (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1)),     # 2 subtiles, 2 A stages
 ]
 
 
