@@ -442,12 +442,14 @@ struct MmaBars {
   uint32_t a_full, b_full, a_empty, b_empty, acc_full, acc_empty, drain;
 };
 
-// The MMA issuer: per K slice, wait for the A stage and the weight stage,
-// issue n_mt x n_sub x 4 tcgen05.mma (A from TMEM, B from shared memory,
-// K = 16 each), commit the accumulators after the tile's last slice and the
-// two stages after every slice.  NMT / NSUB fix the subtile and N-part
-// counts at compile time (0: taken from the plan), so the common shapes
-// issue straight-line code.
+// The MMA issuer, run by a whole warp: per K slice, wait for the A stage and
+// the weight stage, issue n_mt x n_sub x 4 tcgen05.mma (A from TMEM, B from
+// shared memory, K = 16 each), commit the accumulators after the tile's last
+// slice and the two stages after every slice.  Every lane computes the same
+// operands and one elected lane issues, so the operands are warp-uniform;
+// wait results are combined over the warp so all lanes take the same path.
+// NMT / NSUB fix the subtile and N-part counts at compile time (0: taken from
+// the plan), so the common shapes issue straight-line code.
 template <int NMT, int NSUB>
 __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t base, uint32_t tmem_base,
                                                const MmaBars& b, volatile int* abort_flag) {
@@ -463,8 +465,9 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
   for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
     for (int s = 0; ok && s < p.ks; ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
       const uint32_t ea = ap.e, eb = bp.e;
-      if (!wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) ||
-          !wait_or_abort(b.b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag)) {
+      ok = wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) &&
+           wait_or_abort(b.b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
@@ -480,7 +483,8 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
           if (!NSUB && ns >= n_sub) break;
           const int acc = i * n_sub + ns;
           if (first && it > 0 && ok) {
-            ok = wait_or_abort(b.acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag);
+            ok = __all_sync(0xffffffffu,
+                            wait_or_abort(b.acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag));
             tc_fence_after();
           }
           if (ok) {
@@ -489,19 +493,19 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
             const uint64_t bsub = bdesc + static_cast<uint64_t>(ns) * bsub_step;
 #pragma unroll
             for (int j = 0; j < kBlockK / 16; ++j)
-              umma_bf16_ts(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
-                           (first && j == 0) ? 0u : 1u);
-            if (last) umma_commit(b.acc_full + 8u * acc);
+              umma_bf16_ts_elect(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
+                                 (first && j == 0) ? 0u : 1u);
+            if (last) umma_commit_elect(b.acc_full + 8u * acc);
           }
         }
       }
       if (!ok) break;
-      umma_commit(b.a_empty + 8u * ea);
-      umma_commit(b.b_empty + 8u * eb);
+      umma_commit_elect(b.a_empty + 8u * ea);
+      umma_commit_elect(b.b_empty + 8u * eb);
     }
   }
   if (!ok) {
-    umma_commit(b.drain);
+    umma_commit_elect(b.drain);
     mbar_wait(b.drain, 0, p.err, kSiteDrain);
   }
 }
@@ -619,16 +623,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok && any) mbar_wait(bar_halo_full + 8u * last.e, last.ph, p.err, kSiteDrain);
     }
   } else if (warp == kWarpMma) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (whole warp)
+    {
       const MmaBars bars{bar_a_full, bar_b_full, bar_a_empty, bar_b_empty, bar_acc_full, bar_acc_empty, bar_drain};
+      const uint32_t tb = __shfl_sync(0xffffffffu, tmem_base, 0);
       switch (p.n_mt * 4 + p.n_sub) {  // straight-line issue for the common shapes
-        case 1 * 4 + 1: mma_issue_loop<1, 1>(p, base, tmem_base, bars, abort_flag); break;
-        case 1 * 4 + 2: mma_issue_loop<1, 2>(p, base, tmem_base, bars, abort_flag); break;
-        case 2 * 4 + 1: mma_issue_loop<2, 1>(p, base, tmem_base, bars, abort_flag); break;
-        case 2 * 4 + 2: mma_issue_loop<2, 2>(p, base, tmem_base, bars, abort_flag); break;
-        default: mma_issue_loop<0, 0>(p, base, tmem_base, bars, abort_flag); break;
+        case 1 * 4 + 1: mma_issue_loop<1, 1>(p, base, tb, bars, abort_flag); break;
+        case 1 * 4 + 2: mma_issue_loop<1, 2>(p, base, tb, bars, abort_flag); break;
+        case 2 * 4 + 1: mma_issue_loop<2, 1>(p, base, tb, bars, abort_flag); break;
+        case 2 * 4 + 2: mma_issue_loop<2, 2>(p, base, tb, bars, abort_flag); break;
+        default: mma_issue_loop<0, 0>(p, base, tb, bars, abort_flag); break;
       }
+      __syncwarp();
     }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ------------------------------------------------------------ epilogue
