@@ -187,6 +187,18 @@ Q3D_API int32_t q3d_version(void);
 Q3D_API q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream);
 
 /*
+ * q3d_selftest_ratio -- TEST HOOK, not part of the convolution path.
+ * Applies the device step that feeds the E4M3 block-scale rounding
+ * (Model-Optimizer "Conv3D Implicit GEMM CUDA kernel", sec. 6.2: the block
+ * maximum over 6 g, clamped to 448) to n pairs: out[i] = min(RN(bmax[i] /
+ * t[i]), 448), a NaN quotient giving 448.  The device computes it as every
+ * quantiser in this library does.  All pointers are device pointers of n
+ * binary32 values; enqueued on `stream`.  Q3D_ERR_NULLPTR / _INVALID_ARG
+ * (n < 0) before anything is enqueued.
+ */
+Q3D_API q3d_status q3d_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, q3d_stream_t stream);
+
+/*
  * q3d_plan_conv -- TEST HOOK (host only, no CUDA call): the tiling and
  * pipeline plan the specialised sm_100a kernel would use for a convolution of
  * this geometry and dtype.  plan[0..plan_len) receives, in order: applicable

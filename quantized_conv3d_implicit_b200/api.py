@@ -25,7 +25,7 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "q3d_last_error",
-           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats",
+           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats", "q3d_selftest_ratio",
            "q3d_plan_conv", "q3d_plan_conv_tmem")
 
 
@@ -73,6 +73,8 @@ def load_library(path: Optional[str] = None):
         lib.q3d_version.restype = ctypes.c_int32
         lib.q3d_selftest_formats.restype = ctypes.c_int
         lib.q3d_selftest_formats.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
+        lib.q3d_selftest_ratio.restype = ctypes.c_int
+        lib.q3d_selftest_ratio.argtypes = [vp, vp, ctypes.c_int64, vp, vp]
         i64x5 = ctypes.POINTER(ctypes.c_int64)
         for name in ("q3d_plan_conv", "q3d_plan_conv_tmem"):
             fn = getattr(lib, name)
@@ -228,6 +230,18 @@ def selftest_formats(v: torch.Tensor, stream=None):
     st = lib.q3d_selftest_formats(v.data_ptr(), v.numel(), e2m1.data_ptr(), e4m3.data_ptr(), _stream_handle(stream))
     _check(lib, st)
     return e2m1, e4m3
+
+
+def selftest_ratio(bmax: torch.Tensor, t: torch.Tensor, stream=None) -> torch.Tensor:
+    """Test hook: the device's min(bmax / t, 448) of the block-scale step."""
+    lib = load_library()
+    for v in (bmax, t):
+        assert v.dtype == torch.float32 and v.is_cuda and v.is_contiguous()
+    assert bmax.shape == t.shape
+    out = torch.empty_like(bmax)
+    st = lib.q3d_selftest_ratio(bmax.data_ptr(), t.data_ptr(), bmax.numel(), out.data_ptr(), _stream_handle(stream))
+    _check(lib, st)
+    return out
 
 
 PLAN_FIELDS = ("applicable", "TH", "TW", "n_mt", "groups", "n_tile", "n_ntiles", "n_sub", "sub_n", "ks", "c_slot",

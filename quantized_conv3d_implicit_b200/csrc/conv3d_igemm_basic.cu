@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int id0 = od * g.sd - g.pd, ih0 = oh * g.sh - g.ph, iw0 = ow * g.sw - g.pw;
   const T* xn = static_cast<const T*>(p.x) + static_cast<int64_t>(nb) * g.C * g.D * g.H * g.W;
-  Nvfp4Global G{0.0f, 0.0f};
+  Nvfp4Global G{0.0f, 0.0f, 0.0f};
   if (p.quant) G = nvfp4_global(__ldg(p.act_amax));
   const int khw = g.KH * g.KW;
   const uint32_t idesc = umma_idesc_bf16_f32(kBlockM, static_cast<uint32_t>(p.n_tile));

@@ -248,13 +248,13 @@ __device__ __forceinline__ uint32_t quant_pair_bf16x2(float v0, float v1, float 
   return pack_bf16x2(__fmul_rn(q0, s0), __fmul_rn(q1, s1));
 }
 
-// Scales of two rows from their block maxima: IEEE bmax / (6 g), clamp to
-// 448, E4M3 rounding of both rows in one conversion, then (scale, 1/scale)
-// from the per-CTA table indexed by the E4M3 code.
-__device__ __forceinline__ void row_scales(float bmax0, float bmax1, float t, uint32_t tab,
+// Scales of two rows from their block maxima: the correctly rounded
+// bmax / (6 g) clamped to 448, E4M3 rounding of both rows in one conversion,
+// then (scale, 1/scale) from the per-CTA table indexed by the E4M3 code.
+__device__ __forceinline__ void row_scales(float bmax0, float bmax1, const Nvfp4Global& G, uint32_t tab,
                                            float& s0, float& i0, float& s1, float& i1) {
-  const float r0 = fminf(__fdiv_rn(bmax0, t), 448.0f);
-  const float r1 = fminf(__fdiv_rn(bmax1, t), 448.0f);
+  const float r0 = nvfp4_ratio(bmax0, G.t, G.rt);
+  const float r1 = nvfp4_ratio(bmax1, G.t, G.rt);
   uint16_t codes;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(codes) : "f"(r1), "f"(r0));
   float2 e0, e1;
@@ -354,7 +354,7 @@ __device__ __forceinline__ void store_rows(uint32_t a_sub, int rg, int kk, const
 template <typename T, int P>
 __device__ __forceinline__ void transform_task_vec(const FastParams& p, uint32_t a_sub, int rg, int kb,
                                                   uint32_t thr_addr, int delta, uint32_t halo_base,
-                                                  uint32_t slot_base, const float t, uint32_t tab) {
+                                                  uint32_t slot_base, const Nvfp4Global& G, uint32_t tab) {
   constexpr int NW = P / 2;
   uint32_t d[16][NW];
   TapWalker wk;
@@ -386,7 +386,7 @@ __device__ __forceinline__ void transform_task_vec(const FastParams& p, uint32_t
     float sc[P], iv[P];
 #pragma unroll
     for (int j = 0; j < NW; ++j)
-      row_scales(Pair16<T>::abs_lo(mx[j]), Pair16<T>::abs_hi(mx[j]), t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1],
+      row_scales(Pair16<T>::abs_lo(mx[j]), Pair16<T>::abs_hi(mx[j]), G, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1],
                  iv[2 * j + 1]);
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
@@ -424,7 +424,7 @@ __device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t addr) { return
 template <typename T, int P>
 __device__ __forceinline__ void transform_task_gen(const FastParams& p, uint32_t a_sub, int rg, int kb,
                                                   const int (&roff)[8], uint32_t halo_base, uint32_t slot_base,
-                                                  const float t, uint32_t tab) {
+                                                  const Nvfp4Global& G, uint32_t tab) {
   constexpr uint32_t esz = sizeof(T);
   constexpr int NW = P / 2;
   float sc[P], iv[P];
@@ -445,7 +445,7 @@ __device__ __forceinline__ void transform_task_gen(const FastParams& p, uint32_t
     }
 #pragma unroll
     for (int j = 0; j < NW; ++j)
-      row_scales(bm[2 * j], bm[2 * j + 1], t, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1], iv[2 * j + 1]);
+      row_scales(bm[2 * j], bm[2 * j + 1], G, tab, sc[2 * j], iv[2 * j], sc[2 * j + 1], iv[2 * j + 1]);
   }
   TapWalker wk;
   wk.init(p, kb, halo_base, slot_base);
@@ -704,10 +704,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int xf_tid = threadIdx.x - kWarpXf0 * 32;
 
     // per-CTA table of (scale, 1/scale) for every non-negative E4M3 code
-    float t = 0.0f;
+    const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
     {
-      const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f};
-      t = G.t;
       if (p.quant && xf_tid < 128) {
         uint32_t h2;
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
@@ -754,18 +752,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (sizeof(T) == 2) {
           if (p.vec) {
             if (P == 8)
-              transform_task_vec<T, 8>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, t, tab);
+              transform_task_vec<T, 8>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, G, tab);
             else
-              transform_task_vec<T, 4>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, t, tab);
+              transform_task_vec<T, 4>(p, a_sub, rg, kb, thr_addr, delta, halo_base, gs_base, G, tab);
           } else if (P == 8) {
-            transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+            transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, G, tab);
           } else {
-            transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+            transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, G, tab);
           }
         } else if (P == 8) {
-          transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          transform_task_gen<T, 8>(p, a_sub, rg, kb, roff, halo_base, gs_base, G, tab);
         } else {
-          transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, t, tab);
+          transform_task_gen<T, 4>(p, a_sub, rg, kb, roff, halo_base, gs_base, G, tab);
         }
         fence_proxy_async_smem();
         __syncwarp();

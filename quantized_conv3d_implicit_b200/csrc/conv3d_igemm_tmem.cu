@@ -252,10 +252,11 @@ __device__ __forceinline__ void dq4(const DqTable& t, float a0, float a1, float 
   o23 = __byte_perm(lo, hi, 0x7362) | (sgn23 & 0x80008000u);
 }
 
-// (scale, 1/scale) of a row's block from its |v| maximum: IEEE bmax / (6 g),
-// clamp to 448, E4M3 code, then the per-CTA table indexed by the code.
-__device__ __forceinline__ void block_scale(float bmax, float t6g, uint32_t tab, float& s, float& inv) {
-  const float r = fminf(__fdiv_rn(bmax, t6g), 448.0f);  // NaN (0/0) also becomes 448
+// (scale, 1/scale) of a row's block from its |v| maximum: the correctly
+// rounded bmax / (6 g) clamped to 448, E4M3 code, then the per-CTA table
+// indexed by the code.
+__device__ __forceinline__ void block_scale(float bmax, const Nvfp4Global& G, uint32_t tab, float& s, float& inv) {
+  const float r = nvfp4_ratio(bmax, G.t, G.rt);
   uint16_t code;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(code) : "f"(0.0f), "f"(r));
   ld_shared_v2f(tab + (code & 0x7Fu) * 8u, s, inv);
@@ -267,7 +268,7 @@ __device__ __forceinline__ void block_scale(float bmax, float t6g, uint32_t tab,
 // plus the distance to channel c0 + 1 for the columns past the channel end).
 // nvalid < 16 only in a partial last block (columns >= K read as zero).
 template <typename T>
-__device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], int nvalid, bool quant, float t6g,
+__device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], int nvalid, bool quant, const Nvfp4Global& G,
                                           uint32_t tab, uint32_t (&out)[8]) {
   if constexpr (sizeof(T) == 2) {
     uint32_t r[16];
@@ -293,7 +294,7 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
     m01 = Half2<T>::maxabs(m01, m45);
     const float bmax = fmaxf(Half2<T>::abs_lo(m01), Half2<T>::abs_hi(m01));
     float s, inv;
-    block_scale(bmax, t6g, tab, s, inv);
+    block_scale(bmax, G, tab, s, inv);
     const DqTable dt = dq_table(s);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -321,7 +322,7 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
 #pragma unroll
     for (int j = 1; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
     float s, inv;
-    block_scale(bmax, t6g, tab, s, inv);
+    block_scale(bmax, G, tab, s, inv);
     const DqTable dt = dq_table(s);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -341,7 +342,7 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
 // latency.  Same results as two row_block calls.
 template <typename T>
 __device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, const int (&off)[16], bool quant,
-                                             float t6g, uint32_t tab, uint32_t (&out_a)[8], uint32_t (&out_b)[8]) {
+                                             const Nvfp4Global& G, uint32_t tab, uint32_t (&out_a)[8], uint32_t (&out_b)[8]) {
   static_assert(sizeof(T) == 2, "16-bit inputs only");
   uint32_t pa[8], pb[8];
 #pragma unroll
@@ -366,8 +367,8 @@ __device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, c
   ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
   mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
   float sa, ia, sb, ib;
-  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), t6g, tab, sa, ia);
-  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), t6g, tab, sb, ib);
+  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), G, tab, sa, ia);
+  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), G, tab, sb, ib);
   const DqTable da = dq_table(sa), db = dq_table(sb);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -388,7 +389,7 @@ __device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, c
 // Same results as two row_block calls.
 template <typename T>
 __device__ __forceinline__ void row_block_2b(uint32_t addr_a, uint32_t prow_a, uint32_t addr_b, uint32_t prow_b,
-                                             bool quant, float t6g, uint32_t tab, uint32_t (&out_a)[8],
+                                             bool quant, const Nvfp4Global& G, uint32_t tab, uint32_t (&out_a)[8],
                                              uint32_t (&out_b)[8]) {
   static_assert(sizeof(T) == 2, "16-bit inputs only");
   uint32_t pa[8], pb[8];
@@ -423,8 +424,8 @@ __device__ __forceinline__ void row_block_2b(uint32_t addr_a, uint32_t prow_a, u
   ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
   mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
   float sa, ia, sb, ib;
-  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), t6g, tab, sa, ia);
-  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), t6g, tab, sb, ib);
+  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), G, tab, sa, ia);
+  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), G, tab, sb, ib);
   const DqTable da = dq_table(sa), db = dq_table(sb);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -710,10 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // its channel) the byte offsets of the block's 16 taps from that
     // channel's origin, the columns past the channel end taken in the next
     // channel as if it followed contiguously (chan_bytes further on).
-    float t6g = 0.0f;
+    const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
     {
-      const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f};
-      t6g = G.t;
       if (p.quant && xf_tid < 128) {
         uint32_t h2;
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
@@ -808,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             row_block_2b<T>(halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0,
                             phase_tab + static_cast<uint32_t>(phi * 64),
                             halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb) + thr0,
-                            phase_tab + static_cast<uint32_t>(phi1 * 64), p.quant != 0, t6g, tab, wa, wb);
+                            phase_tab + static_cast<uint32_t>(phi1 * 64), p.quant != 0, G, tab, wa, wb);
             tmem_st8(a_col, wa);
             tmem_st8(a_col + 8u, wb);
             pair_done = true;
@@ -846,14 +845,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (; i + 1 < p.n_mt; i += 2) {
                 uint32_t wa[8], wb[8];
                 const uint32_t ra = org + thr0 + static_cast<uint32_t>(i) * thr_step;
-                row_block_x2<T>(ra, ra + thr_step, off, p.quant != 0, t6g, tab, wa, wb);
+                row_block_x2<T>(ra, ra + thr_step, off, p.quant != 0, G, tab, wa, wb);
                 tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
                 tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
               }
           }
           for (; i < p.n_mt; ++i) {
             uint32_t w[8];
-            row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, p.quant != 0, t6g, tab, w);
+            row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, p.quant != 0, G, tab, w);
             tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
           }
         }

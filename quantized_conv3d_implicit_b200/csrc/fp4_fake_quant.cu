@@ -119,6 +119,14 @@ __global__ void selftest_formats_kernel(const float* __restrict__ in, int64_t n,
   e4m3[i] = e4m3_round_trip(fabsf(v));
 }
 
+__global__ void selftest_ratio_kernel(const float* __restrict__ bmax, const float* __restrict__ t, int64_t n,
+                                      float* __restrict__ out) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float ti = t[i];
+  out[i] = nvfp4_ratio(bmax[i], ti, __frcp_rn(ti));
+}
+
 template <typename T>
 cudaError_t launch_fq_typed(const void* x, void* y, int64_t numel, const float* amax, cudaStream_t s, int sm_count) {
   const int64_t nblocks = numel / 16;
@@ -151,6 +159,14 @@ cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, flo
   const int threads = 256;
   const int64_t grid = (n + threads - 1) / threads;
   selftest_formats_kernel<<<static_cast<unsigned>(grid), threads, 0, s>>>(in, n, e2m1, e4m3);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t grid = (n + threads - 1) / threads;
+  selftest_ratio_kernel<<<static_cast<unsigned>(grid), threads, 0, s>>>(bmax, t, n, out);
   return cudaGetLastError();
 }
 

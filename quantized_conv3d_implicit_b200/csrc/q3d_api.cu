@@ -373,6 +373,17 @@ q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* 
   return Q3D_OK;
 }
 
+q3d_status q3d_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, q3d_stream_t stream) {
+  if (!bmax || !t || !out) return fail(Q3D_ERR_NULLPTR, "NULL pointer");
+  if (n < 0) return fail(Q3D_ERR_INVALID_ARG, "n < 0");
+  DeviceInfo* dev = nullptr;
+  q3d_status st;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaError_t e = q3d::launch_selftest_ratio(bmax, t, n, out, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
+  return Q3D_OK;
+}
+
 // Geometry of a planning request (host only); Q3D_OK or an argument error.
 static q3d_status plan_geom(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
                             const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,

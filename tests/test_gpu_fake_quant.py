@@ -36,6 +36,55 @@ def test_device_format_conversions_match_oracle(cuda_ok):
     assert np.array_equal(e4.cpu().numpy().view(np.uint32), oracle.e4m3(np.abs(v)).view(np.uint32))
 
 
+def _ratio_divisors():
+    """6 g for a spread of act_amax: powers of two, mantissas next to 1 and 2,
+    log-uniform values, and the smallest amax for which the ratio decides
+    anything (below it every block scale falls back to 1.0)."""
+    rng = np.random.default_rng(3)
+    t = [2.0 ** e for e in (-22, -10, -3, 0, 1, 5, 20)]
+    t += [np.float32(1.0).view(np.uint32) + d for d in (1, 2, 3)]
+    t += [np.float32(2.0).view(np.uint32) - d for d in (1, 2, 3)]
+    t = [np.uint32(v).view(np.float32) if isinstance(v, (int, np.integer)) else v for v in t]
+    t += list(np.exp(rng.uniform(np.log(1.4e-7), np.log(1e6), 40)))
+    t += [6.0 * (6e-5 / 2688.0), 6.0 * (448.0 / 2688.0), 6.0 * (1.0 / 2688.0)]
+    return np.array(t, np.float32)
+
+
+def _ratio_ref(a, t):
+    with np.errstate(all="ignore"):
+        r = a / t  # IEEE binary32 division, correctly rounded
+    return np.where(np.isnan(r), np.float32(448.0), np.minimum(r, np.float32(448.0))).astype(np.float32)
+
+
+def test_device_scale_ratio_is_correctly_rounded(cuda_ok):
+    """The block maximum over 6 g that feeds the E4M3 scale rounding equals
+    the correctly rounded binary32 quotient (clamped to 448) for every
+    non-negative finite BF16 maximum over a spread of divisors, for random
+    binary32 maxima, and in the degenerate cases amax = 0 and 0 / t.  Near
+    binary32 underflow (quotients below 2^-64) only the E4M3 decision is
+    fixed: E4M3 rounds everything below 2^-10 to zero, so there both values
+    must lie below 2^-10."""
+    bf = (np.arange(0, 0x7F80, dtype=np.uint32) << 16).view(np.float32)  # all finite bf16 >= 0
+    t = _ratio_divisors()
+    a = np.tile(bf, t.size)
+    tt = np.repeat(t, bf.size)
+    rng = np.random.default_rng(4)
+    ar = rng.integers(0, 0x7F800000, 1_000_000, dtype=np.uint32).view(np.float32)  # any finite binary32
+    tr = np.exp(rng.uniform(np.log(1.4e-7), np.log(1e6), ar.size)).astype(np.float32)
+    # maxima whose quotient lands where it decides the E4M3 code (2^-11 .. 2^10)
+    td = np.exp(rng.uniform(np.log(1.4e-7), np.log(1e6), 2_000_000)).astype(np.float32)
+    ad = (td.astype(np.float64) * np.exp2(rng.uniform(-11, 10, td.size))).astype(np.float32)
+    a = np.concatenate([a, ar, ad, np.array([0.0, 1.0, 3e38, 0.0], np.float32)])
+    tt = np.concatenate([tt, tr, td, np.array([0.0, 0.0, 0.0, 1.0], np.float32)])
+    out = api.selftest_ratio(torch.from_numpy(a).cuda(), torch.from_numpy(tt).cuda()).cpu().numpy()
+    ref = _ratio_ref(a, tt)
+    tiny = ref < np.float32(2.0 ** -64)
+    assert np.all(out[tiny] < np.float32(2.0 ** -10)) and np.all(out[tiny] >= 0)
+    assert np.count_nonzero((ref >= np.float32(2.0 ** -10)) & (ref < np.float32(448.0))) > 1_500_000
+    bad = np.flatnonzero((out.view(np.uint32) != ref.view(np.uint32)) & ~tiny)
+    assert bad.size == 0, (bad.size, a[bad[:5]], tt[bad[:5]], out[bad[:5]], ref[bad[:5]])
+
+
 def _blocks(seed, nblocks, dtype):
     g = torch.Generator().manual_seed(seed)
     x = torch.randn(nblocks, 16, generator=g)
