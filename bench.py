@@ -247,10 +247,19 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
     tflops = world * wl.flops * args.steps / (total_ms * 1e-3) / 1e12
 
+    # the global amax that feeds the quantiser (device reduction, outside the
+    # step): L2 flushed before every launch, so x streams from HBM
+    amax_us = time_act_amax(base["x"], stream, dev, args.steps)
+    big = torch.empty(256 << 20, dtype=torch.bfloat16, device=dev).normal_()  # 512 MiB, > 4x L2
+    amax_big_us = time_act_amax(big, stream, dev, args.steps)
+    big_bytes = big.numel() * big.element_size()
+    del big
+
     # end-to-end through the public API with pinned host buffers
     e2e = run_e2e(args, wl, base, stream, dev, world, step_fn=None)
 
     peaks, peaks_src = load_peaks()
+    x_bytes = base["x"].numel() * base["x"].element_size()
     conv_tflops = wl.flops / (conv_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]
     launches_per_step = 2 + (0 if (wl.dtype == torch.bfloat16 and wl.k_gemm % 8 == 0) else 1)
@@ -283,6 +292,16 @@ def run_ours(args, world, rank, local):
             "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(conv_tflops / peak, 4), "traffic": profiled_traffic(wl.name),
             "kernel": "conv3d_igemm_tmem (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
+        },
+        "act_amax": {
+            "us": round(amax_us, 2), "bytes": x_bytes, "bound": "hbm",
+            "achieved": round(x_bytes / (amax_us * 1e-6) / 1e9, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(x_bytes / (amax_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "kernel": "act_amax_kernel", "l2": "flushed (256 MiB write) before each launch",
+            "peak_source": f"{peaks_src} hbm_gbs",
+            "large_input": {"bytes": big_bytes, "us": round(amax_big_us, 2),
+                            "achieved": round(big_bytes / (amax_big_us * 1e-6) / 1e9, 1),
+                            "frac": round(big_bytes / (amax_big_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)},
         },
         "clocks": clocks,
         "e2e": e2e,
@@ -431,6 +450,30 @@ def run_reference(args, world, rank, local):
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
+
+
+def time_act_amax(x, stream, dev, steps):
+    """Mean device time (us) of q3d_act_amax on x (memset of the output word
+    + one kernel), CUDA events on the launching stream, L2 flushed before
+    each launch."""
+    import torch
+
+    from quantized_conv3d_implicit_b200 import api
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = torch.empty(1, dtype=torch.float32, device=dev)
+    n = max(10, min(steps, 100))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for _ in range(3):
+        api.act_amax(x, out=out, stream=stream)
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        api.act_amax(x, out=out, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if api.check_device_error(stream) != 0:
+        raise RuntimeError("device error in act_amax")
+    return statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
 
 
 def main(argv=None):

@@ -164,6 +164,23 @@ Q3D_API q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_t
  */
 Q3D_API q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream);
 
+/*
+ * q3d_act_amax -- *amax = max |x| over every element of x, the global amax
+ * that conv3d_implicit_gemm(quant_act) and fp4_fake_quant take.  The article
+ * feeds its quantiser this scalar: its usage example (sec. 7.2) passes
+ * x.abs().max(), and the quantised inference path (sec. 8.3) gets it from
+ * the input quantizer.
+ *   x     any rank 1..5, dtype F32/F16/BF16, numel >= 0, any alignment.
+ *   amax  device pointer to one float (4-byte aligned, not inside x),
+ *         written with the binary32 value of the largest |x[i]| (exact: the
+ *         value of an input element, widened to binary32); 0 when x is
+ *         empty.  It can be passed straight on as act_amax / amax.
+ * Enqueues a 4-byte memset of *amax and one streaming kernel on `stream`.
+ * NaN in x: the result is unspecified (a NaN).  Q3D_ERR_NULLPTR /
+ * _INVALID_ARG / _UNSUPPORTED_DTYPE before anything is enqueued.
+ */
+Q3D_API q3d_status q3d_act_amax(const q3d_tensor* x, float* amax, q3d_stream_t stream);
+
 /* Message for the last non-OK status returned on this host thread ("" if
  * none).  The pointer stays valid until the next call on this thread. */
 Q3D_API const char* q3d_last_error(void);

@@ -60,6 +60,8 @@ def _load():
             lib.oracle_fq_block.argtypes = [vp, ctypes.c_int, f32, vp]
             lib.oracle_fp4_fake_quant.restype = ctypes.c_int
             lib.oracle_fp4_fake_quant.argtypes = [vp, i64, f32, vp]
+            lib.oracle_act_amax.restype = f32
+            lib.oracle_act_amax.argtypes = [vp, i64]
             lib.oracle_round_to_dtype_bits.restype = None
             lib.oracle_round_to_dtype_bits.argtypes = [vp, i64, ctypes.c_int, vp]
             lib.oracle_out_dim.restype = i64
@@ -141,6 +143,14 @@ def fp4_fake_quant(x, amax: float) -> np.ndarray:
     rc = lib.oracle_fp4_fake_quant(_ptr(x), x.size, float(np.float32(amax)), _ptr(out))
     assert rc == 0
     return out
+
+
+def act_amax(x) -> np.float32:
+    """max |x| over the fp32 values of x (0 for an empty x): the global amax
+    of sec. 7.2 / 8.3, as one binary32 value."""
+    lib = _load()
+    x = _f32(x)
+    return np.float32(lib.oracle_act_amax(_ptr(x), x.size))
 
 
 def fp4_fake_quant_bits(x, amax: float, dtype: str) -> np.ndarray:

@@ -196,6 +196,20 @@ int oracle_fp4_fake_quant(const float* x, int64_t numel, float amax, float* out)
     return 0;
 }
 
+/* The global amax the quantiser takes (sec. 7.2 passes x.abs().max(); the
+ * sec. 8.3 inference path gets it from the input quantizer): the largest
+ * |x[i]| over the fp32 values of x, 0 for an empty x.  A plain scan; the
+ * maximum of magnitudes involves no rounding. */
+float oracle_act_amax(const float* x, int64_t numel)
+{
+    float m = 0.0f;
+    for (int64_t i = 0; i < numel; ++i) {
+        const float a = fabsf(x[i]);
+        if (a > m) m = a;
+    }
+    return m;
+}
+
 /* Round an fp32 array to the storage dtype (0 = fp32, 1 = fp16, 2 = bf16);
  * bits receives the raw pattern (16-bit types) or the binary32 pattern. */
 void oracle_round_to_dtype_bits(const float* v, int64_t n, int dtype, void* bits)

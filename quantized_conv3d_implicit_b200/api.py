@@ -24,7 +24,7 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
-           "fp4_fake_quant", "q3d_last_error",
+           "fp4_fake_quant", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_selftest_formats", "q3d_selftest_ratio",
            "q3d_plan_conv", "q3d_plan_conv_tmem")
 
@@ -66,6 +66,8 @@ def load_library(path: Optional[str] = None):
         lib.conv3d_implicit_gemm_noalloc.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.fp4_fake_quant.restype = ctypes.c_int
         lib.fp4_fake_quant.argtypes = [T, vp, T, vp]
+        lib.q3d_act_amax.restype = ctypes.c_int
+        lib.q3d_act_amax.argtypes = [T, vp, vp]
         lib.q3d_last_error.restype = ctypes.c_char_p
         lib.q3d_last_error.argtypes = []
         lib.q3d_check_device_error.restype = ctypes.c_int
@@ -207,6 +209,20 @@ def fp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: Optional[torch.Tens
         raise ValueError("amax must be a one-element float32 tensor")
     xs, os_ = _tensor(x), _tensor(out)
     st = lib.fp4_fake_quant(_ref(xs), amax.data_ptr(), _ref(os_), _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
+def act_amax(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """max |x| over all elements as a one-element float32 device tensor (0 for
+    an empty x), computed on the device by libq3d; pass it on as act_amax."""
+    lib = load_library()
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    if out.dtype != torch.float32 or out.numel() != 1:
+        raise ValueError("out must be a one-element float32 tensor")
+    xs = _tensor(x if x.dim() > 0 else x.reshape(1))
+    st = lib.q3d_act_amax(_ref(xs), out.data_ptr(), _stream_handle(stream))
     _check(lib, st)
     return out
 

@@ -342,6 +342,25 @@ q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* ou
   return Q3D_OK;
 }
 
+q3d_status q3d_act_amax(const q3d_tensor* x, float* amax, q3d_stream_t stream) {
+  if (!x) return fail(Q3D_ERR_NULLPTR, "x is NULL");
+  if (!amax) return fail(Q3D_ERR_NULLPTR, "amax is NULL");
+  if (x->ndim < 1 || x->ndim > 5) return fail(Q3D_ERR_INVALID_ARG, "x must have rank 1..5");
+  q3d_status st;
+  if ((st = check_tensor(x, "x", x->ndim)) != Q3D_OK) return st;
+  const int64_t n = numel(x);
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(amax), x0 = reinterpret_cast<uintptr_t>(x->data);
+  const uintptr_t x1 = x0 + static_cast<uintptr_t>(n * dtype_size(x->dtype));
+  if (a0 + sizeof(float) > x0 && a0 < x1) return fail(Q3D_ERR_INVALID_ARG, "amax lies inside x");
+  if (a0 % sizeof(float) != 0) return fail(Q3D_ERR_INVALID_ARG, "amax is not 4-byte aligned");
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaError_t e = q3d::launch_act_amax(x->data, x->dtype, n, amax, reinterpret_cast<cudaStream_t>(stream),
+                                       dev->sm_count);
+  if (e != cudaSuccess) return cuda_fail(e, "act_amax launch");
+  return Q3D_OK;
+}
+
 q3d_status q3d_check_device_error(q3d_stream_t stream, uint32_t* site_bits) {
   DeviceInfo* dev = nullptr;
   q3d_status st;

@@ -59,6 +59,8 @@ cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t num
                                   cudaStream_t s, int sm_count);
 cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, cudaStream_t s);
 cudaError_t launch_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, cudaStream_t s);
+// *amax = max |x| over n elements of dtype (0 when n == 0); zeroes *amax on s first.
+cudaError_t launch_act_amax(const void* x, int dtype, int64_t n, float* amax, cudaStream_t s, int sm_count);
 
 // Convert w [Cout, K] (dtype) to bf16 [Cout, ld] with zero columns K..ld-1.
 cudaError_t launch_stage_weights(const void* w, int dtype, int32_t Cout, int32_t K, int64_t ld, void* w_bf16,
