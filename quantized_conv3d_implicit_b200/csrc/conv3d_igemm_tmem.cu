@@ -877,13 +877,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar_a_full + 8u * ea);
           // Later blocks of this warp start at slot q0 or above: hand the
           // slots below back (a slot is free once all transform warps have).
+          // With fewer K slices per tile than A stages, sa slices span
+          // several tiles' slots, more than the ring holds, and a warp
+          // hands back slots it never read: there each waits for the
+          // slot's fill first, or the hand-back could land in the previous
+          // use's phase.  Otherwise the stage coupling keeps every warp
+          // within a ring lap.
           const int keep = (s + 2 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
-          for (; released < keep; ++released, hr.next(ring)) mbar_arrive(bar_halo_empty + 8u * hr.e);
+          for (; ok && released < keep; ++released, hr.next(ring)) {
+            if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+            mbar_arrive(bar_halo_empty + 8u * hr.e);
+          }
+        }
+        if (p.ks < p.sa) {  // sa slices can span more slots than the ring: only there can the hand-back fail
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
         }
       }
       if (!ok) break;
-      if (lane == 0)  // a tile with no slice for this group (ks == 1) still hands its slots back
-        for (; released < p.q_slots; ++released, hr.next(ring)) mbar_arrive(bar_halo_empty + 8u * hr.e);
+      // Hand back the tile's remaining slots.  With fewer K slices than A
+      // stages (all of them in a tile with no slice for this group, when
+      // ks == 1) each waits for its fill first: a warp with nothing to
+      // build would otherwise run a ring lap ahead of the others and arrive
+      // in an earlier phase.
+      if (lane == 0)
+        for (; ok && released < p.q_slots; ++released, hr.next(ring)) {
+          if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+          mbar_arrive(bar_halo_empty + 8u * hr.e);
+        }
+      if (p.ks < p.sa) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       gs_base += static_cast<uint32_t>(p.q_slots);
       ga += static_cast<uint32_t>(p.ks);
     }

@@ -53,7 +53,14 @@ struct DeviceInfo {
   bool init = false;
   int major = 0, minor = 0, sm_count = 0;
   unsigned int* err_word = nullptr;
+  // the library's own stream-ordered pool for per-call scratch (staged
+  // weights, partial sums of cut tiles): freed blocks stay cached up to
+  // kPoolKeepBytes across synchronisations, so a call after a synchronise
+  // does not map fresh memory while the GPU waits; the process's default
+  // pool is left as it is
+  cudaMemPool_t pool = nullptr;
 };
+constexpr uint64_t kPoolKeepBytes = uint64_t{1} << 30;
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -79,6 +86,16 @@ q3d_status current_device(DeviceInfo** out) {
       e = cudaGetSymbolAddress(&p, g_device_error_word);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(error word)");
       d.err_word = static_cast<unsigned int*>(p);
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      e = cudaMemPoolCreate(&d.pool, &props);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+      uint64_t keep = kPoolKeepBytes;
+      e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolSetAttribute");
     }
     d.init = true;
   }
@@ -185,6 +202,7 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
   L.x = x->data; L.bias = bias ? bias->data : nullptr; L.y = out->data;
   L.act_amax = quant_act ? act_amax : nullptr;
   L.dtype = x->dtype; L.quant = quant_act ? 1 : 0; L.err = dev->err_word; L.sm_count = dev->sm_count;
+  L.pool = dev->pool;
   return Q3D_OK;
 }
 
@@ -255,8 +273,8 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
     L.w_ld = K;
   } else {
     const int64_t ld = (K + 7) / 8 * 8;
-    e = cudaMallocAsync(&scratch, static_cast<size_t>(Cout * ld * 2), s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(weight staging)");
+    e = cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(Cout * ld * 2), L.pool, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(weight staging)");
     e = q3d::launch_stage_weights(w->data, x->dtype, (int32_t)Cout, (int32_t)K, ld, scratch, s);
     if (e != cudaSuccess) { cudaFreeAsync(scratch, s); return cuda_fail(e, "weight staging launch"); }
     L.w_bf16 = scratch;
@@ -289,6 +307,7 @@ q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_tensor* w
   bool noop = false;
   q3d_status st = prepare_conv(x, w, bias, act_amax, stride, pad_lo, pad_hi, dil, quant_act, out, &g, &L, &noop);
   if (st != Q3D_OK || noop) return st;
+  L.pool = nullptr;  // no device allocation in this entry point: whole tiles only
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (x->dtype == Q3D_BF16 && g.K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {

@@ -46,6 +46,9 @@ struct ConvLaunch {
   int quant;
   unsigned int* err;        // device error word
   int sm_count;
+  // stream-ordered scratch pool of the device (kept cached across
+  // synchronisations), or nullptr where the call must not allocate
+  cudaMemPool_t pool = nullptr;
 };
 
 // Driver entry point for cuTensorMapEncodeTiled (resolved once through the

@@ -159,3 +159,22 @@ def test_small_workload_full_output(cuda_ok):
     y = _run(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act)
     ref = _ref(inp, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act)
     assert_conv_close(to_np_f32(y), ref, wl.name, wl.dtype)
+
+
+@pytest.mark.parametrize("quant", [False, True])
+def test_single_slice_tiles_many_per_cta(cuda_ok, quant):
+    """K = 64 (one K slice per tile, so one transform group has nothing to
+    build) and about seven tiles of four halo slots per CTA against an
+    11-slot ring: the idle group hands its slots back only as they fill, so
+    it cannot lap the ring."""
+    xs, cout, k = (1, 64, 32, 64, 256), 32, (1, 1, 1)
+    plan = api.plan_conv(xs, (cout, 64) + k, 1, 0, 1, torch.bfloat16, kernel="tmem")
+    assert plan["applicable"] and plan["ks"] == 1
+    tiles = xs[0] * xs[2] * plan["n_ohb"] * plan["n_owb"] * plan["n_ntiles"]  # 1x1x1, no padding: OD = D
+    tiles_per_cta = -(-tiles // 148)
+    assert tiles_per_cta * plan["q_slots"] > 2 * plan["ring"]
+    inp = workloads.random_conv_inputs(32, xs, cout, k, dtype=torch.bfloat16, device="cuda")
+    one, zero = (1, 1, 1), (0, 0, 0)
+    y = _run(inp, one, zero, zero, one, quant)
+    ref = _ref(inp, one, zero, zero, one, quant)
+    assert_conv_close(to_np_f32(y), ref, f"single-slice tiles quant={quant}", torch.bfloat16)

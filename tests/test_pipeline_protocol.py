@@ -38,7 +38,9 @@ class Bar:
         return (self.phase & 1) != (phase & 1)
 
 
-def roles(plan, K, taps, ntiles, kernel="fast"):
+def roles(plan, K, taps, ntiles, kernel="fast", units=None):
+    """units (tensor-memory kernel): the CTA's work as (k0, k1) K-slice
+    ranges of successive tiles; default ntiles whole tiles."""
     bars = {}
 
     def bar(name, i, count):
@@ -62,10 +64,16 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
     def slot_hi(s):
         return (min(64 * s + 63, K - 1) // taps) // c_slot
 
+    us = units if units is not None else [(0, ks)] * ntiles
+
+    def unit_slots(k0, k1):   # first halo slot of a unit and its slot count
+        lo = ((64 * k0) // taps) // c_slot
+        return lo, (min(64 * k1, K) - 1) // taps // c_slot - lo + 1
+
     def halo_producer():
         gs = 0
-        for _ in range(ntiles):
-            for _q in range(q_slots):
+        for k0, k1 in us:
+            for _q in range(unit_slots(k0, k1)[1]):
                 e, u = gs % ring, gs // ring
                 if u > 0:
                     yield ("wait", bar("halo_empty", e, halo_empty_count), u - 1)
@@ -74,8 +82,8 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
 
     def weight_producer():
         gb = 0
-        for _ in range(ntiles):
-            for _s in range(ks):
+        for k0, k1 in us:
+            for _s in range(k0, k1):
                 e, u = gb % sb, gb // sb
                 if u > 0:
                     yield ("wait", bar("b_empty", e, 1), u - 1)
@@ -84,9 +92,9 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
 
     def mma():
         ga = gb = gs_base = 0
-        for it in range(ntiles):
+        for it, (k0, k1) in enumerate(us):
             released = 0
-            for s in range(ks):
+            for s in range(k0, k1):
                 ea, eb = ga % sa, gb % sb
                 yield ("wait", bar("a_full", ea, 8 if kernel == "tmem" else wpg), ga // sa)
                 keep = slot_lo(s + 1) if s + 1 < ks else q_slots
@@ -97,9 +105,9 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
                 for i in range(n_mt):
                     for ns in range(n_sub):
                         acc = i * n_sub + ns
-                        if s == 0 and it > 0:
+                        if s == k0 and it > 0:
                             yield ("wait", bar("acc_empty", acc, 4), it - 1)
-                        if s == ks - 1:
+                        if s == k1 - 1:
                             yield ("arrive", bar("acc_full", acc, 1))
                 yield ("arrive", bar("a_empty", ea, 1))
                 yield ("arrive", bar("b_empty", eb, 1))
@@ -108,7 +116,7 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
             gs_base += q_slots
 
     def epilogue():
-        for it in range(ntiles):
+        for it in range(len(us)):
             for i in range(n_mt):
                 for ns in range(n_sub):
                     acc = i * n_sub + ns
@@ -166,10 +174,11 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
         gs_base = ga = 0
         gslice = grp
         hr = 0  # next global slot to hand back
-        for _ in range(ntiles):
-            s = gslice - ga
+        for k0u, k1u in us:
+            q_lo, n_q = unit_slots(k0u, k1u)
+            s = k0u + gslice - ga
             released = 0
-            while s < ks:
+            while s < k1u:
                 ea, ua = gslice % sa, gslice // sa
                 if gslice >= sa:
                     yield ("wait", bar("a_empty", ea, 1), ua - 1)
@@ -185,25 +194,36 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
                     cross1 = not aligned and (taps - phi1) < min(16, nv1) and cs1 + 1 == c_slot
                     q_last = q1 + int(cross1) if nv1 > 0 else q0 + int(cross0)
                     for q in range(q0, q_last + 1):
-                        g = gs_base + q
+                        assert q_lo <= q < q_lo + n_q, "a block reads a slot outside its unit"
+                        g = gs_base + q - q_lo
                         yield ("wait", bar("halo_full", g % ring, 1), g // ring)
                 yield ("arrive", bar("a_full", ea, 8))
-                if s + 2 < ks:
-                    keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot, q_slots)
+                if s + 2 < k1u:
+                    keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot - q_lo, n_q)
                 else:
-                    keep = q_slots
+                    keep = n_q
                 while released < keep:
+                    # with ks < sa, sa slices span several tiles' slots and a
+                    # warp hands back slots it never read: it waits for each
+                    # slot's fill first so it cannot do so a ring lap early
+                    if ks < sa:
+                        yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                     yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                     released += 1
                     hr += 1
                 s += 2
                 gslice += 2
-            while released < q_slots:
+            while released < n_q:
+                # with ks < sa a slot handed back at the end of a tile waits
+                # for its fill first: a warp with no slice in the tile would
+                # otherwise run a ring lap ahead and arrive in an earlier phase
+                if ks < sa:
+                    yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                 yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                 released += 1
                 hr += 1
-            gs_base += q_slots
-            ga += ks
+            gs_base += n_q
+            ga += k1u - k0u
 
     r = {"halo": halo_producer(), "weights": weight_producer(), "mma": mma()}
     for w in range(4):
@@ -213,8 +233,8 @@ def roles(plan, K, taps, ntiles, kernel="fast"):
     return r
 
 
-def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast"):
-    rs = roles(plan, K, taps, ntiles, kernel)
+def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast", units=None):
+    rs = roles(plan, K, taps, ntiles, kernel, units)
     names = list(rs)
     cur = {k: None for k in names}
     done = set()
@@ -378,3 +398,12 @@ def test_tmem_kernel_plans_blocks_within_one_slot_below_16_taps(kshape):
 def test_tmem_kernel_declines_unaligned_rows():
     plan, _, _ = _plan(((1, 8, 4, 16, 12), (8, 8, 3, 3, 3), 1, 1, 1, torch.bfloat16), kernel="tmem")
     assert plan["applicable"] == 0 and plan["TW"] == 0
+
+
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_tmem_kernel_single_slice_tiles_do_not_lap_the_ring(order):
+    """One K slice per tile: the second transform group never builds, yet
+    hands every slot back; seven tiles of four slots on an 11-slot ring."""
+    plan, K, taps = _plan(((1, 64, 32, 64, 256), (32, 64, 1, 1, 1), 1, 0, 1, torch.bfloat16), kernel="tmem")
+    assert plan["ks"] == 1 and 7 * plan["q_slots"] > 2 * plan["ring"]
+    run(plan, K, taps, 7, order=order, seed=5, kernel="tmem")
