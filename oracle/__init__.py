@@ -60,6 +60,8 @@ def _load():
             lib.oracle_fq_block.argtypes = [vp, ctypes.c_int, f32, vp]
             lib.oracle_fp4_fake_quant.restype = ctypes.c_int
             lib.oracle_fp4_fake_quant.argtypes = [vp, i64, f32, vp]
+            lib.oracle_fp4_fake_quant_bs.restype = ctypes.c_int
+            lib.oracle_fp4_fake_quant_bs.argtypes = [vp, i64, f32, ctypes.c_int, vp]
             lib.oracle_act_amax.restype = f32
             lib.oracle_act_amax.argtypes = [vp, i64]
             lib.oracle_round_to_dtype_bits.restype = None
@@ -142,6 +144,19 @@ def fp4_fake_quant(x, amax: float) -> np.ndarray:
     out = np.empty_like(x)
     rc = lib.oracle_fp4_fake_quant(_ptr(x), x.size, float(np.float32(amax)), _ptr(out))
     assert rc == 0
+    return out
+
+
+def fp4_fake_quant_bs(x, amax: float, block_size: int) -> np.ndarray:
+    """Standalone fake-quant with the article's other block sizes (sec. 7.1,
+    7.3: 16, 32, 64, 128 or 256; numel a multiple of it): binary32 outputs
+    before the cast back to x's dtype."""
+    lib = _load()
+    x = _f32(x)
+    out = np.empty_like(x)
+    rc = lib.oracle_fp4_fake_quant_bs(_ptr(x), x.size, float(np.float32(amax)), int(block_size), _ptr(out))
+    if rc != 0:
+        raise ValueError("block_size must be 16, 32, 64, 128 or 256 and divide numel")
     return out
 
 

@@ -149,10 +149,12 @@ uint16_t oracle_f16_bits(float v)
 /* NVFP4 fake-quantisation of one block (sec. 6.2 and 6.3 of the article)    */
 /* ------------------------------------------------------------------------ */
 
-/* Fake-quantise n (1..16) fp32 values as one block; a short block behaves as
- * if zero-filled to 16 (zeros change neither the block maximum nor the other
- * outputs).  act_amax is the tensor-wide absolute maximum.  out[i] receives
- * the dequantised binary32 value. */
+/* Fake-quantise n fp32 values as one block: n = 16 (the fused path), a
+ * short last block of the fused path (as if zero-filled to 16: zeros change
+ * neither the block maximum nor the other outputs), or a block of 32 .. 256
+ * (the standalone call's other block sizes, sec. 7.1 / 7.3).  act_amax is
+ * the tensor-wide absolute maximum.  out[i] receives the dequantised
+ * binary32 value. */
 void oracle_fq_block(const float* v, int n, float act_amax, float* out)
 {
     /* global scale: act_amax / (6 * 448) */
@@ -193,6 +195,18 @@ int oracle_fp4_fake_quant(const float* x, int64_t numel, float amax, float* out)
 {
     if (numel % 16 != 0) return -1;
     for (int64_t b = 0; b < numel; b += 16) oracle_fq_block(x + b, 16, amax, out + b);
+    return 0;
+}
+
+/* Standalone fake-quantisation with the block size the article's call
+ * accepts (sec. 7.1: 16, 32, 64, 128 or 256; sec. 7.3: numel a multiple of
+ * it): consecutive blocks of `block` elements.  Returns 0, or -1 for another
+ * block size or a numel that is not a multiple of it. */
+int oracle_fp4_fake_quant_bs(const float* x, int64_t numel, float amax, int block, float* out)
+{
+    if (block != 16 && block != 32 && block != 64 && block != 128 && block != 256) return -1;
+    if (numel % block != 0) return -1;
+    for (int64_t b = 0; b < numel; b += block) oracle_fq_block(x + b, block, amax, out + b);
     return 0;
 }
 
