@@ -91,11 +91,16 @@ q3d_status current_device(DeviceInfo** out) {
       props.handleTypes = cudaMemHandleTypeNone;
       props.location.type = cudaMemLocationTypeDevice;
       props.location.id = dev;
-      e = cudaMemPoolCreate(&d.pool, &props);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
-      uint64_t keep = kPoolKeepBytes;
-      e = cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolSetAttribute");
+      // without a pool of its own the library uses the default stream-ordered
+      // allocator (correct, only slower after a synchronise)
+      if (cudaMemPoolCreate(&d.pool, &props) == cudaSuccess) {
+        uint64_t keep = kPoolKeepBytes;
+        if (cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess)
+          cudaGetLastError();  // the pool still works, only without the kept blocks
+      } else {
+        d.pool = nullptr;
+        cudaGetLastError();  // not an error of the caller's call
+      }
     }
     d.init = true;
   }
@@ -273,8 +278,9 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
     L.w_ld = K;
   } else {
     const int64_t ld = (K + 7) / 8 * 8;
-    e = cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(Cout * ld * 2), L.pool, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync(weight staging)");
+    e = L.pool ? cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(Cout * ld * 2), L.pool, s)
+               : cudaMallocAsync(&scratch, static_cast<size_t>(Cout * ld * 2), s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream-ordered allocation (weight staging)");
     e = q3d::launch_stage_weights(w->data, x->dtype, (int32_t)Cout, (int32_t)K, ld, scratch, s);
     if (e != cudaSuccess) { cudaFreeAsync(scratch, s); return cuda_fail(e, "weight staging launch"); }
     L.w_bf16 = scratch;
