@@ -8,7 +8,10 @@ synthetic input: the convolution with fused NVFP4 activation fake-quant
 (conv3d_implicit_gemm_pad2, quant_act as the workload says) followed by the
 standalone fake-quantisation of the same activation tensor (fp4_fake_quant).
 The metric is 2*M*Cout*K / step time in TFLOP/s (the convolution's
-operations; the fake-quant adds time, not operations).
+operations; the fake-quant adds time, not operations).  The default workload
+is the largest single-GPU layer (the full-resolution 96-channel edge conv);
+the same JSON line also carries a `layers` object with the convolution alone
+timed on every workload.
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier and a
 device synchronisation on both sides, measured with CUDA events on the
@@ -22,8 +25,12 @@ on its own seeded input (weak scaling, no collective on the data path);
 value = all ranks' operations / max-over-ranks time.
 
 --impl reference times the CPU oracle (the test infrastructure's plain
-reference) on the host cores for the same workload, each step a bounded
-sample of output rows; only rank 0 does work.
+reference) on the host cores for the same workload, each step a bounded,
+uniformly scaled-down sample of the step (a fraction f of the output rows
+and the same fraction of the fake-quant elements); its value is the rate
+measured on that sample, ms_per_step the measured sample time, and the
+full-layer time it implies is reported separately as an estimate.  Only
+rank 0 does work.
 """
 from __future__ import annotations
 
@@ -185,6 +192,92 @@ def pad6(wl):
     return (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
 
 
+def workload_config(wl, world: int = 1) -> dict:
+    """The `config` object of the JSON line (identical in both arms)."""
+    od, oh, ow = wl.out_spatial()
+    esz = {"torch.bfloat16": 2, "torch.float16": 2, "torch.float32": 4}[str(wl.dtype)]
+    x_b = esz
+    for d in wl.x_shape:
+        x_b *= d
+    y_b = esz * wl.x_shape[0] * wl.cout * od * oh * ow
+    w_b = esz * wl.cout * wl.k_gemm
+    set_mib = (x_b + w_b + y_b) / 2**20
+    n_sets = max(2, -(-2 * L2_BYTES // (x_b + w_b + y_b)))
+    return {
+        "workload": wl.name, "x": list(wl.x_shape), "w": [wl.cout, wl.x_shape[1], *wl.kernel],
+        "stride": list(wl.stride), "pad_lo": list(wl.pad_lo), "pad_hi": list(wl.pad_hi), "dil": list(wl.dil),
+        "quant_act": wl.quant_act, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
+        "step": "conv3d_implicit_gemm(quant_act) + fp4_fake_quant(x)",
+        "l2": (f"x+w+y = {set_mib:.0f} MiB per input set; the GPU arm rotates {n_sets} sets "
+               f"({n_sets * set_mib:.0f} MiB > 126 MiB L2)"),
+        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+    }
+
+
+def make_sets(wl, dev, seed, with_fq: bool):
+    """The workload's seeded inputs plus copies, so that the rotated working
+    set exceeds twice the L2."""
+    import torch
+
+    from quantized_conv3d_implicit_b200 import workloads
+    base = workloads.make_inputs(dataclass_replace(wl, seed=seed), device=dev, with_out=True)
+    per_set = sum(t.numel() * t.element_size() for t in (base["x"], base["w"], base["out"]))
+    n_sets = max(2, -(-2 * L2_BYTES // per_set))
+    sets = [base] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in base.items()} for _ in range(n_sets - 1)]
+    if with_fq:
+        for s in sets:
+            s["fq"] = torch.empty_like(s["x"])
+    return sets
+
+
+def conv_call(api, wl, s, stream):
+    api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
+                             wl.quant_act, out=s["out"], stream=stream)
+
+
+def time_conv_only(api, wl, sets, stream, dev, steps, warmup):
+    """Mean and minimum device time (ms) of the convolution alone over
+    `steps` launches rotating over the input sets, CUDA events on the
+    launching stream, after `warmup` launches."""
+    import torch
+    for i in range(warmup):
+        conv_call(api, wl, sets[i % len(sets)], stream)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i, (a, b) in enumerate(ev):
+        a.record(stream)
+        conv_call(api, wl, sets[i % len(sets)], stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if api.check_device_error(stream) != 0:
+        raise RuntimeError(f"device error in {wl.name}")
+    t = [a.elapsed_time(b) for a, b in ev]
+    return statistics.mean(t), min(t)
+
+
+def run_layers(api, args, stream, dev, peak, headline_sets, headline_name, rank):
+    """Every workload's convolution alone: us, TFLOP/s and fraction of the
+    measured BF16 peak, with the clocks seen while they ran."""
+    import torch
+
+    from quantized_conv3d_implicit_b200 import workloads
+    steps = max(5, min(args.steps, 20))
+    out = {}
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    for name, wl in workloads.WORKLOADS.items():
+        sets = headline_sets if name == headline_name else make_sets(wl, dev, wl.seed + 1000 * rank, False)
+        mean_ms, min_ms = time_conv_only(api, wl, sets, stream, dev, steps, max(3, args.warmup))
+        tf = wl.flops / (mean_ms * 1e-3) / 1e12
+        out[name] = {"us": round(mean_ms * 1e3, 2), "us_min": round(min_ms * 1e3, 2), "tflops": round(tf, 2),
+                     "frac": round(tf / peak, 4), "launches": steps}
+        if sets is not headline_sets:
+            del sets
+            torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    return out, clocks
+
+
 def run_ours(args, world, rank, local):
     import torch
 
@@ -193,21 +286,17 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     init_dist(world, "nccl")
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workloads.get(args.workload)
     api.load_library()
     stream = torch.cuda.current_stream(dev)
 
     # independent seeded input per rank; rotate copies so the working set exceeds L2
-    base = workloads.make_inputs(dataclass_replace(wl, seed=wl.seed + 1000 * rank), device=dev, with_out=True)
-    per_set = sum(t.numel() * t.element_size() for t in (base["x"], base["w"], base["out"]))
-    n_sets = max(2, -(-2 * L2_BYTES // per_set))
-    sets = [base] + [{k: (v.clone() if torch.is_tensor(v) else v) for k, v in base.items()} for _ in range(n_sets - 1)]
-    for s in sets:
-        s["fq"] = torch.empty_like(s["x"])
+    sets = make_sets(wl, dev, wl.seed + 1000 * rank, True)
+    n_sets = len(sets)
+    base = sets[0]
 
     def step(s):
-        api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
-                                 wl.quant_act, out=s["out"], stream=stream)
+        conv_call(api, wl, s, stream)
         api.fp4_fake_quant(s["x"], s["act_amax"], out=s["fq"], stream=stream)
 
     for i in range(args.warmup):
@@ -229,8 +318,7 @@ def run_ours(args, world, rank, local):
         s = sets[i % n_sets]
         a, b, c = ev[i]
         a.record(stream)
-        api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
-                                 wl.quant_act, out=s["out"], stream=stream)
+        conv_call(api, wl, s, stream)
         b.record(stream)
         api.fp4_fake_quant(s["x"], s["act_amax"], out=s["fq"], stream=stream)
         c.record(stream)
@@ -247,23 +335,26 @@ def run_ours(args, world, rank, local):
     ms_per_step = total_ms / args.steps
     tflops = world * wl.flops * args.steps / (total_ms * 1e-3) / 1e12
 
+    peaks, peaks_src = load_peaks()
+    peak = peaks["bf16_tflops"]
+    hbm = peaks["hbm_gbs"]
+    x_bytes = base["x"].numel() * base["x"].element_size()
+
     # the global amax that feeds the quantiser (device reduction, outside the
     # step): L2 flushed before every launch, so x streams from HBM
     amax_us = time_act_amax(base["x"], stream, dev, args.steps)
-    big = torch.empty(256 << 20, dtype=torch.bfloat16, device=dev).normal_()  # 512 MiB, > 4x L2
-    amax_big_us = time_act_amax(big, stream, dev, args.steps)
-    big_bytes = big.numel() * big.element_size()
-    del big
+
+    # every workload's convolution alone (outside the step's timed region)
+    layers, layer_clocks = (None, None)
+    if not args.no_layers:
+        layers, layer_clocks = run_layers(api, args, stream, dev, peak, sets, wl.name, rank)
 
     # end-to-end through the public API with pinned host buffers
-    e2e = run_e2e(args, wl, base, stream, dev, world, step_fn=None)
+    e2e = None if args.no_e2e else run_e2e(args, wl, base, stream, dev, world)
 
-    peaks, peaks_src = load_peaks()
-    x_bytes = base["x"].numel() * base["x"].element_size()
     conv_tflops = wl.flops / (conv_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
     launches_per_step = 2 + (0 if (wl.dtype == torch.bfloat16 and wl.k_gemm % 8 == 0) else 1)
-    od, oh, ow = wl.out_spatial()
+    fq_bytes = 2 * x_bytes  # read x, write the fake-quantised copy
     result = {
         "metric": "Conv3D TFLOP/s (2*M*N*K) and % of B200 BF16 dense peak; us/layer",
         "value": round(tflops, 3),
@@ -277,14 +368,7 @@ def run_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[wl.dtype] + "->bf16 mma, f32 acc",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(K)) weights)",
-        "config": {
-            "workload": wl.name, "x": list(wl.x_shape), "w": [wl.cout, wl.x_shape[1], *wl.kernel],
-            "stride": list(wl.stride), "pad_lo": list(wl.pad_lo), "pad_hi": list(wl.pad_hi), "dil": list(wl.dil),
-            "quant_act": wl.quant_act, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
-            "step": "conv3d_implicit_gemm(quant_act) + fp4_fake_quant(x)",
-            "l2": f"inputs rotate over {n_sets} copies ({n_sets * per_set / 2**20:.0f} MiB > 126 MiB L2)",
-            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-        },
+        "config": workload_config(wl, world),
         "layer_us": round(conv_ms * 1e3, 2),
         "fake_quant_us": round(fq_ms * 1e3, 2),
         "layer_frac_of_peak": round(conv_tflops / peak, 4),
@@ -293,20 +377,26 @@ def run_ours(args, world, rank, local):
             "frac": round(conv_tflops / peak, 4), "traffic": profiled_traffic(wl.name),
             "kernel": "conv3d_igemm_tmem (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
         },
+        "fake_quant": {
+            "us": round(fq_ms * 1e3, 2), "bytes": fq_bytes, "bound": "hbm",
+            "achieved": round(fq_bytes / (fq_ms * 1e-3) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(fq_bytes / (fq_ms * 1e-3) / 1e9 / hbm, 4), "kernel": "fp4_fake_quant_kernel",
+            "l2": "timed inside the step (inputs rotate past L2)", "peak_source": f"{peaks_src} hbm_gbs",
+        },
         "act_amax": {
             "us": round(amax_us, 2), "bytes": x_bytes, "bound": "hbm",
-            "achieved": round(x_bytes / (amax_us * 1e-6) / 1e9, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(x_bytes / (amax_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+            "achieved": round(x_bytes / (amax_us * 1e-6) / 1e9, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(x_bytes / (amax_us * 1e-6) / 1e9 / hbm, 4),
             "kernel": "act_amax_kernel", "l2": "flushed (256 MiB write) before each launch",
             "peak_source": f"{peaks_src} hbm_gbs",
-            "large_input": {"bytes": big_bytes, "us": round(amax_big_us, 2),
-                            "achieved": round(big_bytes / (amax_big_us * 1e-6) / 1e9, 1),
-                            "frac": round(big_bytes / (amax_big_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)},
         },
         "clocks": clocks,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
     }
+    if layers is not None:
+        result["layers"] = layers
+        result["layers_clocks"] = layer_clocks
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, base, budget_s=args.cpu_budget)
     if rank == 0:
@@ -321,7 +411,7 @@ def dataclass_replace(wl, **kw):
     return dataclasses.replace(wl, **kw)
 
 
-def run_e2e(args, wl, base, stream, dev, world, step_fn=None):
+def run_e2e(args, wl, base, stream, dev, world):
     """Same metric through the public calls with pinned host inputs: every step
     copies x, w, bias and act_amax host->device, runs the hot path and copies
     the convolution output and the fake-quantised tensor back."""
@@ -329,7 +419,8 @@ def run_e2e(args, wl, base, stream, dev, world, step_fn=None):
 
     from quantized_conv3d_implicit_b200 import api
 
-    host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in base.items()}
+    host = {k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in base.items()
+            if k in ("x", "w", "bias", "act_amax")}
     dx = torch.empty_like(base["x"])
     dw = torch.empty_like(base["w"])
     db = None if base["bias"] is None else torch.empty_like(base["bias"])
@@ -373,40 +464,44 @@ def run_e2e(args, wl, base, stream, dev, world, step_fn=None):
 # CPU oracle timing (test infrastructure: the only place bench.py runs it)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng):
-    import numpy as np
-
+def oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng):
+    """One scaled-down step on the host cores: `rows` random output rows (all
+    Cout) of the convolution and the same fraction rows / M of the
+    fake-quant elements (whole blocks).  Returns (conv s, fake-quant s,
+    fraction of the step done)."""
     import oracle
     ms = rng.integers(0, wl.m_gemm, rows)
     t = time.perf_counter()
     oracle.conv3d(x_np, w_np, b_np, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act, amax, m_list=ms)
     t_conv = time.perf_counter() - t
-    start = int(rng.integers(0, max(1, x_np.size // 16 - fq_elems // 16))) * 16
+    frac = rows / wl.m_gemm
+    fq_elems = max(16, int(round(x_np.size * frac / 16)) * 16)
+    start = int(rng.integers(0, max(1, (x_np.size - fq_elems) // 16 + 1))) * 16
     t = time.perf_counter()
     oracle.fp4_fake_quant(x_np.reshape(-1)[start:start + fq_elems], amax)
     t_fq = time.perf_counter() - t
-    return t_conv, t_fq, ms.size
+    return t_conv, t_fq, frac
+
+
+def _rows_for(wl, x_np, w_np, b_np, amax, rng, seconds):
+    t_conv, _, _ = oracle_sample_step(wl, x_np, w_np, b_np, amax, 16, rng)
+    return int(max(32, min(wl.m_gemm, seconds / max(t_conv / 16, 1e-6))))
 
 
 def cpu_baseline(wl, base, budget_s: float = 15.0):
-    import numpy as np
     x_np = base["x"].float().cpu().numpy()
     w_np = base["w"].float().cpu().numpy()
     b_np = None if base["bias"] is None else base["bias"].float().cpu().numpy()
     amax = float(base["act_amax"].item())
+    import numpy as np
     rng = np.random.default_rng(1234)
-    # calibrate on a few rows, then size the sample to the time budget
-    t_conv, _, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, 16, 16 * 1024, rng)
-    per_row = max(t_conv / n, 1e-6)
-    rows = int(max(32, min(wl.m_gemm, budget_s * 0.8 / per_row)))
-    fq_elems = 1 << 20
-    t_conv, t_fq, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng)
-    # extrapolate one full step (all M rows + the whole fake-quant tensor)
-    step_s = t_conv * wl.m_gemm / n + t_fq * (x_np.size / fq_elems)
-    return {"value": wl.flops / step_s / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{n} random output rows x all {wl.cout} channels ({t_conv:.1f} s) + fake-quant of "
-                      f"{fq_elems} elements ({t_fq:.2f} s), extrapolated to the full layer "
-                      f"({step_s:.0f} s per step)"}
+    rows = _rows_for(wl, x_np, w_np, b_np, amax, rng, budget_s * 0.8)
+    t_conv, t_fq, frac = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng)
+    sample_s = t_conv + t_fq
+    return {"value": frac * wl.flops / sample_s / 1e12, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{rows} random output rows x all {wl.cout} channels ({t_conv:.1f} s) + the same fraction "
+                      f"({frac:.2e}) of the fake-quant elements ({t_fq:.2f} s); full layer would take "
+                      f"about {sample_s / frac:.0f} s at this rate"}
 
 
 def run_reference(args, world, rank, local):
@@ -416,36 +511,34 @@ def run_reference(args, world, rank, local):
     import numpy as np
 
     from quantized_conv3d_implicit_b200 import workloads
-    wl = workloads.WORKLOADS[args.workload]
+    wl = workloads.get(args.workload)
     base = workloads.make_inputs(wl, device="cpu")
     x_np = base["x"].float().numpy()
     w_np = base["w"].float().numpy()
     b_np = None if base["bias"] is None else base["bias"].float().numpy()
     amax = float(base["act_amax"].item())
     rng = np.random.default_rng(99)
-    t_conv, _, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, 16, 16 * 1024, rng)
-    rows = int(max(32, min(wl.m_gemm, 1.0 / max(t_conv / n, 1e-6))))   # about 1 s of work per step
-    fq_elems = 1 << 18
+    rows = _rows_for(wl, x_np, w_np, b_np, amax, rng, 1.0)   # about 1 s of work per step
     for _ in range(args.warmup):
-        oracle_sample_step(wl, x_np, w_np, b_np, amax, max(8, rows // 8), fq_elems, rng)
-    tot_conv = tot_fq = 0.0
+        oracle_sample_step(wl, x_np, w_np, b_np, amax, max(8, rows // 8), rng)
+    tot = 0.0
+    frac = rows / wl.m_gemm
     for _ in range(args.steps):
-        tc, tf, n = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, fq_elems, rng)
-        tot_conv += tc
-        tot_fq += tf
-    step_s = (tot_conv / args.steps) * wl.m_gemm / rows + (tot_fq / args.steps) * (x_np.size / fq_elems)
-    value = wl.flops / step_s / 1e12
-    od, oh, ow = wl.out_spatial()
-    sample = (f"each step: {rows} random output rows x all {wl.cout} channels + fake-quant of {fq_elems} "
-              f"elements, extrapolated to the full layer")
+        tc, tf, frac = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng)
+        tot += tc + tf
+    step_s = tot / args.steps
+    value = frac * wl.flops / step_s / 1e12
+    sample = (f"each step: {rows} random output rows x all {wl.cout} channels + the same fraction ({frac:.2e}) "
+              f"of the fake-quant elements")
     print(json.dumps({
         "impl": "reference",
         "metric": "Conv3D TFLOP/s (2*M*N*K) and % of B200 BF16 dense peak; us/layer",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 accumulate over bf16/fp4 operands (CPU oracle)", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
-                   "quant_act": wl.quant_act},
+        "config": workload_config(wl, world),
+        "sample_fraction": frac,
+        "full_layer_ms_estimate": step_s / frac * 1e3,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -480,12 +573,14 @@ def main(argv=None):
     from quantized_conv3d_implicit_b200 import workloads
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS) + sorted(workloads.CROPS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-layers", action="store_true", help="skip the per-workload convolution timings")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end timing with host copies")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -31,6 +31,13 @@
  *     for the last non-OK status on the calling host thread.
  *   - Requires a compute-capability 10.x device (B200); otherwise
  *     Q3D_ERR_ARCH.
+ *   - Per-device state (the device error word's address, the staging area
+ *     of conv3d_implicit_gemm_noalloc, a memory pool) is looked up on the
+ *     first call on each device and kept for the life of the process.  Do
+ *     not keep using the library on a device after cudaDeviceReset() on it:
+ *     the addresses it cached belong to the destroyed context.
+ *   - Host-side test hooks (not part of the convolution path) are declared
+ *     separately in q3d_testing.h.
  */
 #ifndef Q3D_H_
 #define Q3D_H_
@@ -195,52 +202,19 @@ Q3D_API q3d_status q3d_check_device_error(q3d_stream_t stream, uint32_t* site_bi
 Q3D_API int32_t q3d_version(void);
 
 /*
- * q3d_selftest_formats -- TEST HOOK, not part of the convolution path.
- * Applies the device format conversions of the quantiser to n binary32
- * inputs: e2m1[i] = E2M1 RNE-saturating value of in[i] (sign kept),
- * e4m3[i] = E4M3 RNE-saturating value of |in[i]|.  All pointers are device
- * pointers; enqueued on `stream`.
+ * q3d_conv_out_shape -- out_shape = [N, Cout, OD, OH, OW] of a convolution
+ * of x [N, Cin, D, H, W] with w [Cout, Cin, kD, kH, kW] (host only, no CUDA
+ * call, no device needed): the output extents of
+ * torch.nn.functional.conv3d, which the article's call promises (sec. 7.1),
+ * with separate leading and trailing padding:
+ *   OD = floor((D + pad_lo_d + pad_hi_d - dil_d*(kD-1) - 1) / stride_d) + 1,
+ * likewise OH, OW.  All arrays are host arrays.  Q3D_ERR_NULLPTR,
+ * Q3D_ERR_INVALID_ARG (Cin mismatch, N or Cout < 0, stride or dilation < 1,
+ * pad < 0, kernel extent < 1, or an empty output extent).
  */
-Q3D_API q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream);
-
-/*
- * q3d_selftest_ratio -- TEST HOOK, not part of the convolution path.
- * Applies the device step that feeds the E4M3 block-scale rounding
- * (Model-Optimizer "Conv3D Implicit GEMM CUDA kernel", sec. 6.2: the block
- * maximum over 6 g, clamped to 448) to n pairs: out[i] = min(RN(bmax[i] /
- * t[i]), 448), a NaN quotient giving 448.  The device computes it as every
- * quantiser in this library does.  All pointers are device pointers of n
- * binary32 values; enqueued on `stream`.  Q3D_ERR_NULLPTR / _INVALID_ARG
- * (n < 0) before anything is enqueued.
- */
-Q3D_API q3d_status q3d_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, q3d_stream_t stream);
-
-/*
- * q3d_plan_conv -- TEST HOOK (host only, no CUDA call): the tiling and
- * pipeline plan the specialised sm_100a kernel would use for a convolution of
- * this geometry and dtype.  plan[0..plan_len) receives, in order: applicable
- * (0/1), TH, TW, n_mt, groups, n_tile, n_ntiles, n_sub, sub_n, K slices per
- * tile, channels per halo slot, halo slots per tile, halo ring entries,
- * A stages, B stages, TMEM columns, shared-memory bytes, tiles along OH,
- * tiles along OW, vectorised halo reads (0/1), halo box W, H and D extents;
- * further entries are 0.
- */
-Q3D_API q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
-                                 const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
-                                 int32_t dtype, int32_t* plan, int32_t plan_len);
-
-/*
- * q3d_plan_conv_tmem -- TEST HOOK (host only, no CUDA call): as
- * q3d_plan_conv, for the kernel that builds the A operand in tensor memory.
- * Same field order; groups (transform warp groups, each taking the K
- * slices of one parity) is always 2, TMEM columns 512, vectorised reads 0,
- * and one more entry follows the halo box extents: the first TMEM column of
- * the A stages.  applicable = 0 where that kernel does not apply (x rows
- * not a multiple of 16 bytes, more than 343 taps, or no plan that fits).
- */
-Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+Q3D_API q3d_status q3d_conv_out_shape(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
                                       const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
-                                      int32_t dtype, int32_t* plan, int32_t plan_len);
+                                      int64_t out_shape[5]);
 
 #ifdef __cplusplus
 }  /* extern "C" */

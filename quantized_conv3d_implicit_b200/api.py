@@ -25,8 +25,8 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "q3d_act_amax", "q3d_last_error",
-           "q3d_check_device_error", "q3d_version", "q3d_selftest_formats", "q3d_selftest_ratio",
-           "q3d_plan_conv", "q3d_plan_conv_tmem")
+           "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
+           "q3d_selftest_ratio", "q3d_plan_conv", "q3d_plan_conv_tmem")
 
 
 class Q3DTensor(ctypes.Structure):
@@ -78,6 +78,8 @@ def load_library(path: Optional[str] = None):
         lib.q3d_selftest_ratio.restype = ctypes.c_int
         lib.q3d_selftest_ratio.argtypes = [vp, vp, ctypes.c_int64, vp, vp]
         i64x5 = ctypes.POINTER(ctypes.c_int64)
+        lib.q3d_conv_out_shape.restype = ctypes.c_int
+        lib.q3d_conv_out_shape.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, i64x5]
         for name in ("q3d_plan_conv", "q3d_plan_conv_tmem"):
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
@@ -142,13 +144,24 @@ def _check(lib, status: int):
 
 
 def out_shape(x_shape, w_shape, stride=1, padding=0, dilation=1):
-    s, d = _triple(stride), _triple(dilation)
+    """[N, Cout, OD, OH, OW] of the convolution, as the library computes it
+    (q3d_conv_out_shape); raises Q3DError for an invalid geometry."""
+    lib = load_library()
     lo, hi = _pads(padding)
-    dims = []
-    for i in range(3):
-        span = x_shape[2 + i] + lo[i] + hi[i] - d[i] * (w_shape[2 + i] - 1) - 1
-        dims.append(span // s[i] + 1 if span >= 0 else 0)
-    return (x_shape[0], w_shape[0], *dims)
+    a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    a5 = lambda t: (ctypes.c_int64 * 5)(*[int(v) for v in t])  # noqa: E731
+    o = (ctypes.c_int64 * 5)()
+    _check(lib, lib.q3d_conv_out_shape(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi),
+                                       a3(_triple(dilation)), o))
+    return tuple(int(v) for v in o)
+
+
+def _check_amax(act_amax, x, quant_act):
+    if quant_act:
+        if act_amax is None:
+            raise ValueError("quant_act requires act_amax")
+        if act_amax.dtype != torch.float32 or act_amax.numel() != 1 or act_amax.device != x.device:
+            raise ValueError("act_amax must be a one-element float32 tensor on x's device")
 
 
 def conv3d_implicit_gemm(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
@@ -158,22 +171,25 @@ def conv3d_implicit_gemm(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.
     accumulation, result in x.dtype), optionally fake-quantising the
     activation operand to NVFP4 (act_amax: float32 device tensor with one
     element).  padding may be an int, a 3-tuple or a 6-tuple
-    (d_lo, d_hi, h_lo, h_hi, w_lo, w_hi)."""
+    (d_lo, d_hi, h_lo, h_hi, w_lo, w_hi); symmetric padding goes through the
+    C entry point conv3d_implicit_gemm, asymmetric padding through
+    conv3d_implicit_gemm_pad2."""
     lib = load_library()
     lo, hi = _pads(padding)
     if out is None:
         out = torch.empty(out_shape(x.shape, w.shape, stride, padding, dilation), dtype=x.dtype, device=x.device)
-    if quant_act:
-        if act_amax is None:
-            raise ValueError("quant_act requires act_amax")
-        if act_amax.dtype != torch.float32 or act_amax.numel() != 1 or act_amax.device != x.device:
-            raise ValueError("act_amax must be a one-element float32 tensor on x's device")
+    _check_amax(act_amax, x, quant_act)
     arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
     xs, ws, os_, bs = _tensor(x), _tensor(w), _tensor(out), _tensor(bias)
     amax_ptr = act_amax.data_ptr() if (quant_act and act_amax is not None) else None
-    st = lib.conv3d_implicit_gemm_pad2(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
-                                       arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
-                                       _stream_handle(stream))
+    if lo == hi:   # symmetric padding: the article's signature (sec. 7.1)
+        st = lib.conv3d_implicit_gemm(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
+                                      arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
+                                      _stream_handle(stream))
+    else:
+        st = lib.conv3d_implicit_gemm_pad2(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
+                                           arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
+                                           _stream_handle(stream))
     _check(lib, st)
     return out
 
@@ -187,8 +203,7 @@ def conv3d_implicit_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, out: torch.Te
     fixed 16 MiB area per device).  `out` must be preallocated."""
     lib = load_library()
     lo, hi = _pads(padding)
-    if quant_act and (act_amax is None or act_amax.dtype != torch.float32 or act_amax.numel() != 1):
-        raise ValueError("quant_act requires a one-element float32 act_amax tensor")
+    _check_amax(act_amax, x, quant_act)
     arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
     xs, ws, os_, bs = _tensor(x), _tensor(w), _tensor(out), _tensor(bias)
     amax_ptr = act_amax.data_ptr() if quant_act else None

@@ -527,8 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpB) {
     // ------------------------------------------------------------ weight producer
     if (lane == 0) {
-      uint32_t gb = 0;
-      int64_t last = -1;
+      uint32_t gb = 0;  // weight stages issued
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
@@ -542,18 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < p.n_sub; ++i)
             tma_load_2d(base + p.off_b + e * p.b_stage_bytes + static_cast<uint32_t>(i * p.sub_n) * 128u, &tmap_w,
                         bar_b_full + 8u * e, kBlockK * s, tc.nt * p.n_tile + i * p.sub_n);
-          last = gb;
         }
       }
-      if (!ok && last >= 0)
-        mbar_wait(bar_b_full + 8u * static_cast<uint32_t>(last % p.sb), static_cast<uint32_t>(last / p.sb) & 1u, p.err,
-                  kSiteDrain);
+      if (!ok) drain_ring(bar_b_full, static_cast<uint32_t>(p.sb), gb, p.err, kSiteDrain);
     }
   } else if (warp == kWarpHalo) {
     // ------------------------------------------------------------ halo producer
     if (lane == 0) {
-      uint32_t gs = 0;
-      int64_t last = -1;
+      uint32_t gs = 0;  // halo slots issued
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x) {
         const TileCoord tc = decode_tile(p, t);
@@ -569,12 +564,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(bar_halo_full + 8u * e, p.slot_tx);
           tma_load_5d(base + p.off_halo + e * p.slot_bytes, &tmap_x, bar_halo_full + 8u * e, w0, h0, d0,
                       q * p.c_slot, tc.n);
-          last = gs;
         }
       }
-      if (!ok && last >= 0)
-        mbar_wait(bar_halo_full + 8u * static_cast<uint32_t>(last % p.ring),
-                  static_cast<uint32_t>(last / p.ring) & 1u, p.err, kSiteDrain);
+      if (!ok) drain_ring(bar_halo_full, static_cast<uint32_t>(p.ring), gs, p.err, kSiteDrain);
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer

@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include "q3d.h"
+#include "q3d_testing.h"
 #include "q3d_internal.h"
 
 namespace q3d {
@@ -53,8 +54,8 @@ struct DeviceInfo {
   bool init = false;
   int major = 0, minor = 0, sm_count = 0;
   unsigned int* err_word = nullptr;
-  // the library's own stream-ordered pool for per-call scratch (staged
-  // weights, partial sums of cut tiles): freed blocks stay cached up to
+  // the library's own stream-ordered pool for per-call scratch (the BF16
+  // copy of weights that cannot be read in place): freed blocks stay cached up to
   // kPoolKeepBytes across synchronisations, so a call after a synchronise
   // does not map fresh memory while the GPU waits; the process's default
   // pool is left as it is
@@ -112,6 +113,24 @@ q3d_status current_device(DeviceInfo** out) {
 }
 
 bool dtype_ok(int32_t dt) { return dt == Q3D_F32 || dt == Q3D_F16 || dt == Q3D_BF16; }
+
+// Output extents of a convolution (torch.nn.functional.conv3d's formula with
+// separate leading and trailing padding); Q3D_OK or an argument error.
+q3d_status conv_out_dims(const int64_t in_dims[3], const int64_t k_dims[3], const int32_t stride[3],
+                         const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int64_t o_dims[3]) {
+  for (int i = 0; i < 3; ++i) {
+    if (stride[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "stride[%d] = %d must be >= 1", i, stride[i]);
+    if (dil[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "dilation[%d] = %d must be >= 1", i, dil[i]);
+    if (pad_lo[i] < 0 || pad_hi[i] < 0) return fail(Q3D_ERR_INVALID_ARG, "padding[%d] must be >= 0", i);
+    if (k_dims[i] < 1 || in_dims[i] < 0) return fail(Q3D_ERR_INVALID_ARG, "extents along dim %d must be >= 0", i);
+    const int64_t span = in_dims[i] + pad_lo[i] + pad_hi[i] - static_cast<int64_t>(dil[i]) * (k_dims[i] - 1) - 1;
+    if (span < 0)
+      return fail(Q3D_ERR_INVALID_ARG, "kernel extent exceeds the padded input along dim %d (empty output)", i);
+    o_dims[i] = span / stride[i] + 1;
+  }
+  return Q3D_OK;
+}
+
 int64_t dtype_size(int32_t dt) { return dt == Q3D_F32 ? 4 : 2; }
 
 int64_t numel(const q3d_tensor* t) {
@@ -154,11 +173,6 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
   if (quant_act && !act_amax) return fail(Q3D_ERR_NULLPTR, "quant_act requires act_amax");
   if (w->dtype != x->dtype || out->dtype != x->dtype || (bias && bias->dtype != x->dtype))
     return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "w, bias and out must have the dtype of x");
-  for (int i = 0; i < 3; ++i) {
-    if (stride[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "stride[%d] = %d must be >= 1", i, stride[i]);
-    if (dil[i] < 1) return fail(Q3D_ERR_INVALID_ARG, "dilation[%d] = %d must be >= 1", i, dil[i]);
-    if (pad_lo[i] < 0 || pad_hi[i] < 0) return fail(Q3D_ERR_INVALID_ARG, "padding[%d] must be >= 0", i);
-  }
   const int64_t N = x->shape[0], C = x->shape[1], D = x->shape[2], H = x->shape[3], W = x->shape[4];
   const int64_t Cout = w->shape[0], KD = w->shape[2], KH = w->shape[3], KW = w->shape[4];
   if (w->shape[1] != C)
@@ -169,12 +183,7 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
   if (bias && bias->shape[0] != Cout) return fail(Q3D_ERR_INVALID_ARG, "bias must have shape [Cout]");
   const int64_t in_dims[3] = {D, H, W}, k_dims[3] = {KD, KH, KW};
   int64_t o_dims[3];
-  for (int i = 0; i < 3; ++i) {
-    const int64_t span = in_dims[i] + pad_lo[i] + pad_hi[i] - static_cast<int64_t>(dil[i]) * (k_dims[i] - 1) - 1;
-    if (span < 0)
-      return fail(Q3D_ERR_INVALID_ARG, "kernel extent exceeds the padded input along dim %d (empty output)", i);
-    o_dims[i] = span / stride[i] + 1;
-  }
+  if ((st = conv_out_dims(in_dims, k_dims, stride, pad_lo, pad_hi, dil, o_dims)) != Q3D_OK) return st;
   if (out->shape[0] != N || out->shape[1] != Cout || out->shape[2] != o_dims[0] || out->shape[3] != o_dims[1] ||
       out->shape[4] != o_dims[2])
     return fail(Q3D_ERR_INVALID_ARG, "out must have shape [%lld, %lld, %lld, %lld, %lld]", (long long)N,
@@ -313,7 +322,6 @@ q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_tensor* w
   bool noop = false;
   q3d_status st = prepare_conv(x, w, bias, act_amax, stride, pad_lo, pad_hi, dil, quant_act, out, &g, &L, &noop);
   if (st != Q3D_OK || noop) return st;
-  L.pool = nullptr;  // no device allocation in this entry point: whole tiles only
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (x->dtype == Q3D_BF16 && g.K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {
@@ -406,6 +414,25 @@ q3d_status q3d_check_device_error(q3d_stream_t stream, uint32_t* site_bits) {
   return Q3D_OK;
 }
 
+q3d_status q3d_conv_out_shape(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                              const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                              int64_t out_shape[5]) {
+  if (!x_shape || !w_shape || !stride || !pad_lo || !pad_hi || !dil || !out_shape)
+    return fail(Q3D_ERR_NULLPTR, "NULL pointer");
+  if (w_shape[1] != x_shape[1])
+    return fail(Q3D_ERR_INVALID_ARG, "w has %lld input channels but x has %lld (groups != 1 is not supported)",
+                (long long)w_shape[1], (long long)x_shape[1]);
+  if (x_shape[0] < 0 || w_shape[0] < 0) return fail(Q3D_ERR_INVALID_ARG, "N and Cout must be >= 0");
+  const int64_t in_dims[3] = {x_shape[2], x_shape[3], x_shape[4]}, k_dims[3] = {w_shape[2], w_shape[3], w_shape[4]};
+  int64_t o_dims[3];
+  const q3d_status st = conv_out_dims(in_dims, k_dims, stride, pad_lo, pad_hi, dil, o_dims);
+  if (st != Q3D_OK) return st;
+  out_shape[0] = x_shape[0];
+  out_shape[1] = w_shape[0];
+  for (int i = 0; i < 3; ++i) out_shape[2 + i] = o_dims[i];
+  return Q3D_OK;
+}
+
 q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream) {
   if (!in || !e2m1 || !e4m3) return fail(Q3D_ERR_NULLPTR, "NULL pointer");
   if (n < 0) return fail(Q3D_ERR_INVALID_ARG, "n < 0");
@@ -437,14 +464,10 @@ static q3d_status plan_geom(const int64_t x_shape[5], const int64_t w_shape[5], 
   if (!dtype_ok(dtype)) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "dtype");
   q3d::ConvGeom& g = *gp;
   const int64_t k_dims[3] = {w_shape[2], w_shape[3], w_shape[4]};
+  const int64_t in_dims[3] = {x_shape[2], x_shape[3], x_shape[4]};
   int64_t o_dims[3];
-  for (int i = 0; i < 3; ++i) {
-    if (stride[i] < 1 || dil[i] < 1 || pad_lo[i] < 0 || pad_hi[i] < 0 || k_dims[i] < 1)
-      return fail(Q3D_ERR_INVALID_ARG, "bad stride/pad/dilation/kernel");
-    const int64_t span = x_shape[2 + i] + pad_lo[i] + pad_hi[i] - static_cast<int64_t>(dil[i]) * (k_dims[i] - 1) - 1;
-    if (span < 0) return fail(Q3D_ERR_INVALID_ARG, "empty output");
-    o_dims[i] = span / stride[i] + 1;
-  }
+  const q3d_status st = conv_out_dims(in_dims, k_dims, stride, pad_lo, pad_hi, dil, o_dims);
+  if (st != Q3D_OK) return st;
   if (w_shape[1] != x_shape[1]) return fail(Q3D_ERR_INVALID_ARG, "groups != 1");
   g.N = (int32_t)x_shape[0]; g.C = (int32_t)x_shape[1]; g.D = (int32_t)x_shape[2]; g.H = (int32_t)x_shape[3];
   g.W = (int32_t)x_shape[4];

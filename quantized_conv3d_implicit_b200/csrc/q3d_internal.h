@@ -46,8 +46,9 @@ struct ConvLaunch {
   int quant;
   unsigned int* err;        // device error word
   int sm_count;
-  // stream-ordered scratch pool of the device (kept cached across
-  // synchronisations), or nullptr where the call must not allocate
+  // stream-ordered pool of the device for the staged BF16 weights (kept
+  // cached across synchronisations), or nullptr (then the default
+  // stream-ordered allocator); the kernels never read it
   cudaMemPool_t pool = nullptr;
 };
 

@@ -91,6 +91,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
   }
 }
 
+// After an abort, wait (bounded) for every copy a producer may still have in
+// flight in a ring of n entries whose full barriers count its issues: issue i
+// went to entry i % n and completes that entry's phase of parity (i / n) & 1.
+// Only the last min(issued, n) issues can be outstanding (each earlier entry
+// was handed back empty, hence landed, before its reuse); waiting on an
+// already completed phase returns at once.  A CTA must not exit while a bulk
+// copy into its shared memory is still running.
+__device__ __forceinline__ void drain_ring(uint32_t full_bar0, uint32_t n, uint32_t issued, unsigned int* err,
+                                           unsigned int site) {
+  const uint32_t first = issued > n ? issued - n : 0u;
+  for (uint32_t i = first; i < issued; ++i) mbar_wait(full_bar0 + 8u * (i % n), (i / n) & 1u, err, site);
+}
+
 // ---------------------------------------------------------------------------
 // proxy fences
 // ---------------------------------------------------------------------------

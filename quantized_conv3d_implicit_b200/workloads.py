@@ -98,7 +98,23 @@ WORKLOADS = {
 
 # the five configurations in order (the third and fourth have two entries)
 SMALL = "tiny_16x16_fp32"
-HEADLINE = "wan_mid_384_bf16"
+# the largest single-GPU layer: the benchmark's default workload
+HEADLINE = "edge_full_96_bf16"
+
+# Fewer-frame copies of the full-resolution layers: the same spatial extent,
+# hence the same tiling plan and per-tile work, with a smaller input, for
+# profiler captures that must hold only a few GB on the device.
+CROPS = {
+    "edge_full_96_bf16_d5": dataclasses.replace(WORKLOADS["edge_full_96_bf16"], name="edge_full_96_bf16_d5",
+                                                x_shape=(1, 96, 5, 480, 832)),
+}
+
+
+def get(name: str) -> Workload:
+    """A workload or crop by name."""
+    if name in WORKLOADS:
+        return WORKLOADS[name]
+    return CROPS[name]
 
 
 def make_inputs(wl: Workload | str, device="cpu", with_out: bool = False):

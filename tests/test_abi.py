@@ -12,7 +12,7 @@ import torch
 from quantized_conv3d_implicit_b200 import api, build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "q3d.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("q3d.h", "q3d_testing.h")]
 
 
 @pytest.fixture(scope="module")
@@ -22,7 +22,7 @@ def lib():
 
 
 def _declared():
-    src = open(HEADER).read()
+    src = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"Q3D_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
 
 
@@ -114,6 +114,58 @@ def test_fake_quant_validation(lib):
     assert lib.fp4_fake_quant(r(T((2, 16))), FAKE * 4096, r(T((2, 16), 1, FAKE * 256)), None) == 3
     assert lib.fp4_fake_quant(r(T((2, 16))), FAKE * 4096, r(T((16, 2), 2, FAKE * 256)), None) == 2
     assert lib.fp4_fake_quant(r(T((0, 16))), FAKE * 4096, r(T((0, 16), 2, FAKE * 256)), None) == 0
+
+
+def conv_sym(lib, x, w, out, pad=(1, 1, 1), amax=None, quant=0):
+    arr = lambda v: (ctypes.c_int32 * 3)(*v) if v is not None else None  # noqa: E731
+    r = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731
+    return lib.conv3d_implicit_gemm(r(x), r(w), None, amax, arr((1, 1, 1)), arr(pad), arr((1, 1, 1)), quant, r(out),
+                                    None)
+
+
+def test_symmetric_entry_point_validation(lib):
+    x, w, out = good()
+    assert conv_sym(lib, x, w, out, pad=None) == 1
+    assert b"pad" in lib.q3d_last_error()
+    assert conv_sym(lib, x, w, out, pad=(-1, 1, 1)) == 2
+    assert conv_sym(lib, x, w, T((1, 5, 3, 8, 9), 2, FAKE * 256)) == 2     # out shape for pad 1
+    assert conv_sym(lib, x, w, out, quant=1) == 1                           # quant without act_amax
+    assert conv_sym(lib, T((0, 4, 3, 8, 8)), w, T((0, 5, 3, 8, 8), 2, FAKE * 256)) == 0
+
+
+def test_conv_out_shape(lib):
+    a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    a5 = lambda t: (ctypes.c_int64 * 5)(*t)  # noqa: E731
+    o = (ctypes.c_int64 * 5)()
+    # causal temporal padding, stride (1, 2, 2), dilation (1, 2, 2)
+    st = lib.q3d_conv_out_shape(a5((2, 8, 17, 64, 63)), a5((24, 8, 3, 3, 3)), a3((1, 2, 2)), a3((2, 1, 1)),
+                                a3((0, 1, 1)), a3((1, 2, 2)), o)
+    assert st == 0
+    # floor((I + lo + hi - dil*(k-1) - 1) / s) + 1 along each dim
+    assert tuple(o) == (2, 24, 17, 31, 31)
+    assert api.out_shape((2, 8, 17, 64, 63), (24, 8, 3, 3, 3), (1, 2, 2), (2, 0, 1, 1, 1, 1), (1, 2, 2)) == \
+        (2, 24, 17, 31, 31)
+    assert lib.q3d_conv_out_shape(a5((1, 8, 2, 2, 2)), a5((4, 8, 5, 1, 1)), a3((1, 1, 1)), a3((0, 0, 0)),
+                                  a3((0, 0, 0)), a3((1, 1, 1)), o) == 2        # empty output
+    assert lib.q3d_conv_out_shape(a5((1, 8, 4, 4, 4)), a5((4, 7, 1, 1, 1)), a3((1, 1, 1)), a3((0, 0, 0)),
+                                  a3((0, 0, 0)), a3((1, 1, 1)), o) == 2        # groups != 1
+    assert lib.q3d_conv_out_shape(None, a5((4, 8, 1, 1, 1)), a3((1, 1, 1)), a3((0, 0, 0)), a3((0, 0, 0)),
+                                  a3((1, 1, 1)), o) == 1
+    with pytest.raises(api.Q3DError):
+        api.out_shape((1, 8, 4, 4, 4), (4, 8, 3, 3, 3), 0, 0, 1)
+
+
+def test_noalloc_binding_rejects_host_act_amax(lib):
+    x = torch.zeros((1, 4, 3, 8, 8), dtype=torch.bfloat16)
+    w = torch.zeros((5, 4, 3, 3, 3), dtype=torch.bfloat16)
+    y = torch.zeros((1, 5, 3, 8, 8), dtype=torch.bfloat16)
+    bad = torch.zeros(1, dtype=torch.float32, device="meta")   # not on x's device
+    with pytest.raises(ValueError):
+        api.conv3d_implicit_gemm_noalloc(x, w, y, None, 1, 1, 1, act_amax=bad, quant_act=True)
+    with pytest.raises(ValueError):
+        api.conv3d_implicit_gemm_noalloc(x, w, y, None, 1, 1, 1, act_amax=None, quant_act=True)
+    with pytest.raises(ValueError):
+        api.conv3d_implicit_gemm(x, w, None, 1, 1, 1, act_amax=torch.zeros(2), quant_act=True, out=y)
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")

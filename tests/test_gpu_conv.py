@@ -80,19 +80,34 @@ def test_conv_small_shapes(cuda_ok, kernel, case, quant, dtype):
     assert_conv_close(to_np_f32(y), ref, f"case {case} quant={quant} {dtype}", dtype)
 
 
+# act_amax settings that reach every branch of the fused quantiser's scale
+# step (article sec. 6.2): the tensor's own max|x| (the normal case); 0 (g = 0,
+# so the ratio is 0/0 or inf, clamped to 448, and the scale 0 falls back to
+# 1.0); a fiftieth of max|x| (blocks whose maximum exceeds act_amax: the ratio
+# is clamped to 448 and the E2M1 codes saturate at 6); 2688 = 6 * 448 (g = 1);
+# and 1e-6 (every block scale is below 1e-5 and falls back to 1.0).
+AMAX_MODES = ("max", "zero", "max/50", "2688", "1e-6")
+
+
+def _amax_value(mode, x):
+    m = float(x.float().abs().max())
+    return {"max": m, "zero": 0.0, "max/50": m / 50.0, "2688": 2688.0, "1e-6": 1e-6}[mode]
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("quant", [False, True])
+@pytest.mark.parametrize("mode", ("noquant",) + AMAX_MODES)
 @pytest.mark.parametrize("width", [11, 16])
-def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, quant, dtype, width):
+def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, mode, dtype, width):
     # one-hot weights: y[:, co] = A[:, k(co)], a single nonzero product per
     # output, so the FP32 accumulator holds the BF16 operand exactly and the
     # whole im2col row (quantised or not) is reproduced bit for bit; W = 16
     # reaches the TMA-fed kernels, W = 11 the general one
+    quant = mode != "noquant"
     xs, k = (1, 5, 4, 9, width), (3, 3, 3)
     K = 5 * 27
     g = torch.Generator().manual_seed(3)
     x = (torch.randn(xs, generator=g) * 3).to(dtype)
-    amax = x.float().abs().max().reshape(1)
+    amax = torch.tensor([_amax_value(mode if quant else "max", x)], dtype=torch.float32)
     for start in range(0, K, 128):
         cols = list(range(start, min(K, start + 128)))
         w = torch.zeros((len(cols), K), dtype=torch.float32)
@@ -106,6 +121,23 @@ def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, quant, dtype, wid
                                                                         torch.float16: "float16",
                                                                         torch.bfloat16: "bfloat16"}[dtype])
         assert np.array_equal(bits(y), ref_bits), start
+
+
+# shapes of SHAPES that reach the TMA-fed kernels' distinct plans: a partial
+# last block, dilation, stride 2, 5x5x5, two N tiles, two subtiles
+EDGE_SHAPES = (10, 11, 12, 13, 14, 16)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("mode", ("zero", "max/50", "2688", "1e-6"))
+@pytest.mark.parametrize("case", EDGE_SHAPES)
+def test_conv_small_shapes_amax_edge_cases(cuda_ok, kernel, case, mode, dtype):
+    xs, cout, k, s, plo, phi, d = SHAPES[case]
+    inp = workloads.random_conv_inputs(400 + case, xs, cout, k, dtype=dtype, bias=True, device="cuda", scale=2.0)
+    inp["act_amax"] = torch.tensor([_amax_value(mode, inp["x"])], dtype=torch.float32, device="cuda")
+    y = _run(inp, s, plo, phi, d, True)
+    ref = _ref(inp, s, plo, phi, d, True)
+    assert_conv_close(to_np_f32(y), ref, f"case {case} act_amax {mode} {dtype}", dtype)
 
 
 def test_determinism(cuda_ok, kernel):
@@ -122,6 +154,29 @@ def test_symmetric_entry_point_and_noop(cuda_ok):
     assert_conv_close(to_np_f32(y), ref, "symmetric", torch.bfloat16)
     e = api.conv3d_implicit_gemm(inp["x"][:0], inp["w"], padding=1)
     assert e.shape[0] == 0
+
+
+@pytest.mark.parametrize("quant", [False, True])
+def test_symmetric_c_entry_point_through_ctypes(cuda_ok, quant):
+    """conv3d_implicit_gemm with its symmetric pad[3], called straight
+    through the C ABI (no binding logic in between), against the oracle."""
+    import ctypes
+    lib = api.load_library()
+    xs, cout, k = (1, 12, 5, 11, 24), 40, (3, 3, 3)
+    inp = workloads.random_conv_inputs(77, xs, cout, k, dtype=torch.bfloat16, device="cuda")
+    stride, pad, dil = (1, 2, 1), (1, 2, 1), (1, 1, 2)
+    oshape = api.out_shape(xs, (cout, xs[1]) + k, stride, pad, dil)
+    y = torch.full(oshape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    a3 = lambda v: (ctypes.c_int32 * 3)(*v)  # noqa: E731
+    tx, tw, tb, ty = api._tensor(inp["x"]), api._tensor(inp["w"]), api._tensor(inp["bias"]), api._tensor(y)
+    st = lib.conv3d_implicit_gemm(ctypes.byref(tx), ctypes.byref(tw), ctypes.byref(tb),
+                                  inp["act_amax"].data_ptr() if quant else None, a3(stride), a3(pad), a3(dil),
+                                  int(quant), ctypes.byref(ty), None)
+    assert st == 0, lib.q3d_last_error()
+    torch.cuda.synchronize()
+    assert api.check_device_error() == 0
+    ref = _ref(inp, stride, pad, pad, dil, quant)
+    assert_conv_close(to_np_f32(y), ref, f"symmetric C entry quant={quant}", torch.bfloat16)
 
 
 def _sample_rows(wl, rng, n_random):
