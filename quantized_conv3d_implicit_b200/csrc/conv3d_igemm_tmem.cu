@@ -39,6 +39,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "nvfp4.cuh"
 #include "q3d_internal.h"
@@ -86,7 +87,7 @@ struct TmemParams {
   int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
-  uint32_t off_b, off_halo, off_tab, off_phase, off_bar;
+  uint32_t off_dq, off_b, off_halo, off_code, off_phase, off_bar;
 };
 
 struct TileCoord {
@@ -157,9 +158,6 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, int& a, int& b, int& c, int& d) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr));
 }
-__device__ __forceinline__ void ld_shared_v2f(uint32_t addr, float& a, float& b) {
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(a), "=f"(b) : "r"(addr));
-}
 
 // E2M1 codes (round to nearest even, saturating) of four non-negative
 // values, one per nibble of the low 16 bits (a0 lowest).
@@ -191,32 +189,6 @@ __device__ __forceinline__ uint32_t maxabs_f16x2(uint32_t a, uint32_t b) {
   asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
-
-// Per-element views of a packed pair of 16-bit inputs.
-template <typename T>
-struct Half2;
-template <>
-struct Half2<__nv_bfloat16> {
-  // |x| as an operand modifier of the consuming multiply or max
-  static __device__ __forceinline__ float abs_lo(uint32_t w) { return fabsf(__uint_as_float(w << 16)); }
-  static __device__ __forceinline__ float abs_hi(uint32_t w) { return fabsf(__uint_as_float(w & 0xFFFF0000u)); }
-  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_bf16x2(a, b); }
-  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
-};
-template <>
-struct Half2<__half> {
-  static __device__ __forceinline__ float abs_lo(uint32_t w) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0x7FFFu)));
-  }
-  static __device__ __forceinline__ float abs_hi(uint32_t w) {
-    return __half2float(__ushort_as_half(static_cast<unsigned short>((w >> 16) & 0x7FFFu)));
-  }
-  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_f16x2(a, b); }
-  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) {
-    return cvt_bf16x2(__half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))),
-                      __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu))));
-  }
-};
 
 // Dequantisation table of one row's block: the BF16 bit patterns of q*scale
 // for the eight E2M1 magnitudes q in code order {0, .5, 1, 1.5, 2, 3, 4, 6},
@@ -252,57 +224,238 @@ __device__ __forceinline__ void dq4(const DqTable& t, float a0, float a1, float 
   o23 = __byte_perm(lo, hi, 0x7362) | (sgn23 & 0x80008000u);
 }
 
-// (scale, 1/scale) of a row's block from its |v| maximum: the correctly
-// rounded bmax / (6 g) clamped to 448, E4M3 code, then the per-CTA table
-// indexed by the code.
-__device__ __forceinline__ void block_scale(float bmax, const Nvfp4Global& G, uint32_t tab, float& s, float& inv) {
-  const float r = nvfp4_ratio(bmax, G.t, G.rt);
+// Per-CTA quantiser tables in shared memory.
+//  - Entry table: for every E4M3 code of a block scale (0..127), 32 bytes:
+//    the block's DqTable (16 B) and 1/scale (binary32), where scale =
+//    E4M3(code) * g, or 1.0 when that is below 1e-5.
+//  - BF16 inputs only, code table: a block maximum of a BF16 input is itself
+//    a BF16 value, and the scale step (ratio to 6 g, clamp to 448, E4M3
+//    rounding) is a monotone function of it; the table maps each BF16 bit
+//    pattern b in [lo, hi] to the byte offset of its code's entry.  The
+//    window spans the 22 binades from 2^-11 t (every smaller maximum gives
+//    code 0) up past 2^9 t (every larger one clamps to 448), so patterns
+//    outside it take the entry of the nearer end.  The entries are computed
+//    with the same device arithmetic as the direct path, so both give the
+//    same code for every maximum.
+constexpr int kDqEntryBytes = 32;
+constexpr int kDqTableBytes = 128 * kDqEntryBytes;
+constexpr int kCodeBinades = 22;
+constexpr int kCodeEntries = kCodeBinades * 128;  // BF16 has 128 patterns per binade
+constexpr int kCodeTableBytes = kCodeEntries * 2;
+
+struct QCtx {
+  Nvfp4Global G;
+  uint32_t dq;      // shared address of the entry table
+  uint32_t cb;      // shared address of the code table minus 2 * lo
+  uint32_t lo, hi;  // BF16 bit patterns covered by the code table
+};
+
+__device__ __forceinline__ uint32_t e4m3_code(float r) {
   uint16_t code;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(code) : "f"(0.0f), "f"(r));
-  ld_shared_v2f(tab + (code & 0x7Fu) * 8u, s, inv);
+  return code & 0x7Fu;
 }
 
-// One row x one 16-column block: the 16 BF16 values of A as 8 packed words.
-// addr0: shared address of the row's element for the block's first column
-// in channel c0; off[j]: byte offset of column j from addr0 (tap offset,
-// plus the distance to channel c0 + 1 for the columns past the channel end).
-// nvalid < 16 only in a partial last block (columns >= K read as zero).
+// Shared address of the entry for a block maximum given as a binary32 value.
+__device__ __forceinline__ uint32_t entry_of_max(float bmax, const QCtx& q) {
+  return q.dq + e4m3_code(nvfp4_ratio(bmax, q.G.t, q.G.rt)) * kDqEntryBytes;
+}
+
+__device__ __forceinline__ void load_entry(uint32_t e, DqTable& t, float& inv) {
+  int a, b, c, d;
+  ld_shared_v4(e, a, b, c, d);
+  t.lo_a = static_cast<uint32_t>(a);
+  t.lo_b = static_cast<uint32_t>(b);
+  t.hi_a = static_cast<uint32_t>(c);
+  t.hi_b = static_cast<uint32_t>(d);
+  inv = __uint_as_float(ld_shared_u32(e + 16u));
+}
+
+// Per-element views of a packed pair of 16-bit inputs.
 template <typename T>
-__device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], int nvalid, bool quant, const Nvfp4Global& G,
-                                          uint32_t tab, uint32_t (&out)[8]) {
-  if constexpr (sizeof(T) == 2) {
-    uint32_t r[16];
-    if (nvalid >= 16) {
+struct Half2;
+template <>
+struct Half2<__nv_bfloat16> {
+  // |x| as an operand modifier of the consuming multiply or max
+  static __device__ __forceinline__ float abs_lo(uint32_t w) { return fabsf(__uint_as_float(w << 16)); }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) { return fabsf(__uint_as_float(w & 0xFFFF0000u)); }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_bf16x2(a, b); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
+  // entry of a block from the packed |v| maximum of its eight words: the
+  // larger half's BF16 pattern indexes the code table (clamped to its window)
+  static __device__ __forceinline__ uint32_t entry(uint32_t m, const QCtx& q) {
+    const uint32_t m2 = maxabs_bf16x2(m, __byte_perm(m, 0u, 0x1032));
+    const uint32_t b = min(max(m2 & 0x7FFFu, q.lo), q.hi);
+    return q.dq + ld_shared_u16(q.cb + 2u * b);
+  }
+};
+template <>
+struct Half2<__half> {
+  static __device__ __forceinline__ float abs_lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0x7FFFu)));
+  }
+  static __device__ __forceinline__ float abs_hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>((w >> 16) & 0x7FFFu)));
+  }
+  static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_f16x2(a, b); }
+  static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) {
+    return cvt_bf16x2(__half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16))),
+                      __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu))));
+  }
+  static __device__ __forceinline__ uint32_t entry(uint32_t m, const QCtx& q) {
+    return entry_of_max(fmaxf(abs_lo(m), abs_hi(m)), q);
+  }
+};
+
+// |v| maximum of a block held as eight packed words.
+template <typename T>
+__device__ __forceinline__ uint32_t maxabs8(const uint32_t (&p)[8]) {
+  using H = Half2<T>;
+  return H::maxabs(H::maxabs(H::maxabs(p[0], p[1]), H::maxabs(p[2], p[3])),
+                   H::maxabs(H::maxabs(p[4], p[5]), H::maxabs(p[6], p[7])));
+}
+
+// Quantise one block of a 16-bit input (eight packed words) with its entry.
+template <typename T>
+__device__ __forceinline__ void quant8(const uint32_t (&pk)[8], const DqTable& dt, float inv, uint32_t (&out)[8]) {
+  using H = Half2<T>;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) r[j] = ld_shared_u16(addr0 + static_cast<uint32_t>(off[j]));
-    } else {
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w0 = pk[2 * i], w1 = pk[2 * i + 1];
+    dq4(dt, __fmul_rn(H::abs_lo(w0), inv), __fmul_rn(H::abs_hi(w0), inv), __fmul_rn(H::abs_lo(w1), inv),
+        __fmul_rn(H::abs_hi(w1), inv), w0, w1, out[2 * i], out[2 * i + 1]);
+  }
+}
+
+// Two blocks of a 16-bit input (two rows, or two blocks of one row), each
+// quantised with its own scale; the two chains are interleaved so each hides
+// the other's latency.  Without quantisation the values are only converted.
+template <typename T>
+__device__ __forceinline__ void quant8_x2(const uint32_t (&pa)[8], const uint32_t (&pb)[8], bool quant, const QCtx& q,
+                                          uint32_t (&out_a)[8], uint32_t (&out_b)[8]) {
+  if (!quant) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) r[j] = j < nvalid ? ld_shared_u16(addr0 + static_cast<uint32_t>(off[j])) : 0u;
+    for (int i = 0; i < 8; ++i) {
+      out_a[i] = Half2<T>::to_bf16x2(pa[i]);
+      out_b[i] = Half2<T>::to_bf16x2(pb[i]);
     }
-    uint32_t pk[8];
+    return;
+  }
+  const uint32_t ma = maxabs8<T>(pa), mb = maxabs8<T>(pb);
+  const uint32_t ea = Half2<T>::entry(ma, q), eb = Half2<T>::entry(mb, q);
+  DqTable da, db;
+  float ia, ib;
+  load_entry(ea, da, ia);
+  load_entry(eb, db, ib);
+  quant8<T>(pa, da, ia, out_a);
+  quant8<T>(pb, db, ib, out_b);
+}
+
+template <int OFF>
+__device__ __forceinline__ uint32_t ld_shared_u16_at(uint32_t addr) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1+%2];" : "=h"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
+// Gathers of one row's 16 values of a block into eight packed words.
+//  - By tap offsets: addr0 + off[j] for column j (columns past K read zero
+//    when nvalid < 16).
+//  - By rows (kernels three taps wide): the block's taps lie on six rows of
+//    three columns DWB bytes apart; rb[r] is the address of row r's first
+//    column and the block starts at column P3 of row 0, so every column step
+//    is an immediate of the load.
+template <typename T>
+__device__ __forceinline__ void gather_taps(uint32_t addr0, const int (&off)[16], int nvalid, uint32_t (&pk)[8]) {
+  static_assert(sizeof(T) == 2, "16-bit inputs only");
+  uint32_t r[16];
+  if (nvalid >= 16) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) pk[i] = __byte_perm(r[2 * i], r[2 * i + 1], 0x5410);
+    for (int j = 0; j < 16; ++j) r[j] = ld_shared_u16(addr0 + static_cast<uint32_t>(off[j]));
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) r[j] = j < nvalid ? ld_shared_u16(addr0 + static_cast<uint32_t>(off[j])) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = __byte_perm(r[2 * i], r[2 * i + 1], 0x5410);
+}
+
+template <int P3, int DWB, int... J>
+__device__ __forceinline__ void gather_rows_seq(const uint32_t (&rb)[6], uint32_t (&r)[16],
+                                                std::integer_sequence<int, J...>) {
+  ((r[J] = ld_shared_u16_at<((P3 + J) % 3) * DWB>(rb[(P3 + J) / 3])), ...);
+}
+template <int P3, int DWB>
+__device__ __forceinline__ void gather_rows(const uint32_t (&rb)[6], uint32_t (&pk)[8]) {
+  uint32_t r[16];
+  gather_rows_seq<P3, DWB>(rb, r, std::make_integer_sequence<int, 16>{});
+#pragma unroll
+  for (int i = 0; i < 8; ++i) pk[i] = __byte_perm(r[2 * i], r[2 * i + 1], 0x5410);
+}
+
+// Row bases of a block from its phase-table row (six row offsets), with the
+// rows from `split` on moved by `adj` (their channel opens the next slot).
+__device__ __forceinline__ void row_bases(uint32_t org, uint32_t prow, int split, int adj, uint32_t (&rb)[6]) {
+  int o[8];
+  ld_shared_v4(prow, o[0], o[1], o[2], o[3]);
+  ld_shared_v4(prow + 16u, o[4], o[5], o[6], o[7]);
+#pragma unroll
+  for (int r = 0; r < 6; ++r) rb[r] = org + static_cast<uint32_t>(o[r] + (r >= split ? adj : 0));
+}
+
+// The 16 tap offsets of a phase-table row.
+__device__ __forceinline__ void load_taps(uint32_t prow, int (&off)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 4) ld_shared_v4(prow + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
+}
+
+// The 16 tap offsets of a block from a row-gather phase-table row: tap j is
+// column (p3 + j) % 3 of row (p3 + j) / 3, p3 = phi % 3.
+template <int DWB>
+__device__ __forceinline__ void taps_from_rows(uint32_t prow, int p3, int (&off)[16]) {
+  int o[8];
+  ld_shared_v4(prow, o[0], o[1], o[2], o[3]);
+  ld_shared_v4(prow + 16u, o[4], o[5], o[6], o[7]);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int a = j / 3, b = j % 3;  // p3 + j = 3a + b + p3
+    const bool wrap = b + p3 >= 3;
+    off[j] = (wrap ? o[a + 1 < 8 ? a + 1 : 7] : o[a]) + (b + p3 - (wrap ? 3 : 0)) * DWB;
+  }
+}
+
+// Quantise (or only convert) one block of a 16-bit input.
+template <typename T>
+__device__ __forceinline__ void quant8_1(const uint32_t (&pk)[8], bool quant, const QCtx& q, uint32_t (&out)[8]) {
+  if (!quant) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = Half2<T>::to_bf16x2(pk[i]);
+    return;
+  }
+  DqTable dt;
+  float inv;
+  load_entry(Half2<T>::entry(maxabs8<T>(pk), q), dt, inv);
+  quant8<T>(pk, dt, inv, out);
+}
+
+// One row x one 16-column block of any input type: the 16 BF16 values of A as
+// 8 packed words, gathered by tap offsets (nvalid < 16 only in a partial
+// last block).
+template <typename T>
+__device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], int nvalid, bool quant, const QCtx& q,
+                                          uint32_t (&out)[8]) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t pk[8];
+    gather_taps<T>(addr0, off, nvalid, pk);
     if (!quant) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) out[i] = Half2<T>::to_bf16x2(pk[i]);
       return;
     }
-    uint32_t m01 = Half2<T>::maxabs(pk[0], pk[1]), m23 = Half2<T>::maxabs(pk[2], pk[3]);
-    uint32_t m45 = Half2<T>::maxabs(pk[4], pk[5]), m67 = Half2<T>::maxabs(pk[6], pk[7]);
-    m01 = Half2<T>::maxabs(m01, m23);
-    m45 = Half2<T>::maxabs(m45, m67);
-    m01 = Half2<T>::maxabs(m01, m45);
-    const float bmax = fmaxf(Half2<T>::abs_lo(m01), Half2<T>::abs_hi(m01));
-    float s, inv;
-    block_scale(bmax, G, tab, s, inv);
-    const DqTable dt = dq_table(s);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t w0 = pk[2 * i], w1 = pk[2 * i + 1];
-      dq4(dt, __fmul_rn(Half2<T>::abs_lo(w0), inv), __fmul_rn(Half2<T>::abs_hi(w0), inv),
-          __fmul_rn(Half2<T>::abs_lo(w1), inv), __fmul_rn(Half2<T>::abs_hi(w1), inv), w0, w1, out[2 * i],
-          out[2 * i + 1]);
-    }
+    DqTable dt;
+    float inv;
+    load_entry(Half2<T>::entry(maxabs8<T>(pk), q), dt, inv);
+    quant8<T>(pk, dt, inv, out);
   } else {
     float v[16];
     if (nvalid >= 16) {
@@ -321,9 +474,9 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
     float bmax = fabsf(v[0]);
 #pragma unroll
     for (int j = 1; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
-    float s, inv;
-    block_scale(bmax, G, tab, s, inv);
-    const DqTable dt = dq_table(s);
+    DqTable dt;
+    float inv;
+    load_entry(entry_of_max(bmax, q), dt, inv);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int j = 4 * i;
@@ -336,107 +489,10 @@ __device__ __forceinline__ void row_block(uint32_t addr0, const int (&off)[16], 
   }
 }
 
-// Two rows (the same output position in two subtiles) of one full 16-column
-// block of a 16-bit input, sharing the tap offsets: the two load, maximum,
-// scale and dequantisation chains are interleaved so each hides the other's
-// latency.  Same results as two row_block calls.
-template <typename T>
-__device__ __forceinline__ void row_block_x2(uint32_t addr_a, uint32_t addr_b, const int (&off)[16], bool quant,
-                                             const Nvfp4Global& G, uint32_t tab, uint32_t (&out_a)[8], uint32_t (&out_b)[8]) {
-  static_assert(sizeof(T) == 2, "16-bit inputs only");
-  uint32_t pa[8], pb[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t a0 = ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i]));
-    const uint32_t b0 = ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i]));
-    const uint32_t a1 = ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i + 1]));
-    const uint32_t b1 = ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i + 1]));
-    pa[i] = __byte_perm(a0, a1, 0x5410);
-    pb[i] = __byte_perm(b0, b1, 0x5410);
-  }
-  if (!quant) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      out_a[i] = Half2<T>::to_bf16x2(pa[i]);
-      out_b[i] = Half2<T>::to_bf16x2(pb[i]);
-    }
-    return;
-  }
-  uint32_t ma = Half2<T>::maxabs(Half2<T>::maxabs(pa[0], pa[1]), Half2<T>::maxabs(pa[2], pa[3]));
-  uint32_t mb = Half2<T>::maxabs(Half2<T>::maxabs(pb[0], pb[1]), Half2<T>::maxabs(pb[2], pb[3]));
-  ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
-  mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
-  float sa, ia, sb, ib;
-  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), G, tab, sa, ia);
-  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), G, tab, sb, ib);
-  const DqTable da = dq_table(sa), db = dq_table(sb);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t a0 = pa[2 * i], a1 = pa[2 * i + 1], b0 = pb[2 * i], b1 = pb[2 * i + 1];
-    dq4(da, __fmul_rn(Half2<T>::abs_lo(a0), ia), __fmul_rn(Half2<T>::abs_hi(a0), ia),
-        __fmul_rn(Half2<T>::abs_lo(a1), ia), __fmul_rn(Half2<T>::abs_hi(a1), ia), a0, a1, out_a[2 * i],
-        out_a[2 * i + 1]);
-    dq4(db, __fmul_rn(Half2<T>::abs_lo(b0), ib), __fmul_rn(Half2<T>::abs_hi(b0), ib),
-        __fmul_rn(Half2<T>::abs_lo(b1), ib), __fmul_rn(Half2<T>::abs_hi(b1), ib), b0, b1, out_b[2 * i],
-        out_b[2 * i + 1]);
-  }
-}
-
-// Two full 16-column blocks of one row (a transform warp's pair b0, b0 + 1
-// in a single-subtile tile) of a 16-bit input, each with its own channel
-// origin and phase-table row; the two chains are interleaved.  Each block's
-// tap offsets are read just before its gathers to keep register use low.
-// Same results as two row_block calls.
-template <typename T>
-__device__ __forceinline__ void row_block_2b(uint32_t addr_a, uint32_t prow_a, uint32_t addr_b, uint32_t prow_b,
-                                             bool quant, const Nvfp4Global& G, uint32_t tab, uint32_t (&out_a)[8],
-                                             uint32_t (&out_b)[8]) {
-  static_assert(sizeof(T) == 2, "16-bit inputs only");
-  uint32_t pa[8], pb[8];
-  {
-    int off[16];
-#pragma unroll
-    for (int j = 0; j < 16; j += 4) ld_shared_v4(prow_a + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      pa[i] = __byte_perm(ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i])),
-                          ld_shared_u16(addr_a + static_cast<uint32_t>(off[2 * i + 1])), 0x5410);
-  }
-  {
-    int off[16];
-#pragma unroll
-    for (int j = 0; j < 16; j += 4) ld_shared_v4(prow_b + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      pb[i] = __byte_perm(ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i])),
-                          ld_shared_u16(addr_b + static_cast<uint32_t>(off[2 * i + 1])), 0x5410);
-  }
-  if (!quant) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      out_a[i] = Half2<T>::to_bf16x2(pa[i]);
-      out_b[i] = Half2<T>::to_bf16x2(pb[i]);
-    }
-    return;
-  }
-  uint32_t ma = Half2<T>::maxabs(Half2<T>::maxabs(pa[0], pa[1]), Half2<T>::maxabs(pa[2], pa[3]));
-  uint32_t mb = Half2<T>::maxabs(Half2<T>::maxabs(pb[0], pb[1]), Half2<T>::maxabs(pb[2], pb[3]));
-  ma = Half2<T>::maxabs(ma, Half2<T>::maxabs(Half2<T>::maxabs(pa[4], pa[5]), Half2<T>::maxabs(pa[6], pa[7])));
-  mb = Half2<T>::maxabs(mb, Half2<T>::maxabs(Half2<T>::maxabs(pb[4], pb[5]), Half2<T>::maxabs(pb[6], pb[7])));
-  float sa, ia, sb, ib;
-  block_scale(fmaxf(Half2<T>::abs_lo(ma), Half2<T>::abs_hi(ma)), G, tab, sa, ia);
-  block_scale(fmaxf(Half2<T>::abs_lo(mb), Half2<T>::abs_hi(mb)), G, tab, sb, ib);
-  const DqTable da = dq_table(sa), db = dq_table(sb);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t a0 = pa[2 * i], a1 = pa[2 * i + 1], b0 = pb[2 * i], b1 = pb[2 * i + 1];
-    dq4(da, __fmul_rn(Half2<T>::abs_lo(a0), ia), __fmul_rn(Half2<T>::abs_hi(a0), ia),
-        __fmul_rn(Half2<T>::abs_lo(a1), ia), __fmul_rn(Half2<T>::abs_hi(a1), ia), a0, a1, out_a[2 * i],
-        out_a[2 * i + 1]);
-    dq4(db, __fmul_rn(Half2<T>::abs_lo(b0), ib), __fmul_rn(Half2<T>::abs_hi(b0), ib),
-        __fmul_rn(Half2<T>::abs_lo(b1), ib), __fmul_rn(Half2<T>::abs_hi(b1), ib), b0, b1, out_b[2 * i],
-        out_b[2 * i + 1]);
-  }
+// Column step in bytes of the row gather (kernels three taps wide, 16-bit
+// input, W dilation 1 or 2), or 0 where the tap-offset gather applies.
+__host__ __device__ inline int row_gather_step(const ConvGeom& g, int esz) {
+  return (esz == 2 && g.KW == 3 && (g.dw == 1 || g.dw == 2)) ? g.dw * esz : 0;
 }
 
 struct MmaBars {
@@ -513,8 +569,10 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
 
 // kPairs: the tile has at least two M-subtiles, built in interleaved pairs
 // (a separate instantiation, so single-subtile tiles keep their register
-// allocation).
-template <typename T, bool kPairs>
+// allocation).  kDWB > 0: 16-bit input and a kernel three taps wide whose
+// taps along W are kDWB bytes apart (dilation * element size), gathered by
+// rows with immediate column offsets; 0: gathered by tap offsets.
+template <typename T, bool kPairs, int kDWB>
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
                              const __grid_constant__ CUtensorMap tmap_w) {
@@ -698,30 +756,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;          // output position within a subtile
     const int th = row / p.TW, tw = row % p.TW;
     const uint32_t halo_base = base + p.off_halo;
-    const uint32_t tab = base + p.off_tab;
     const uint32_t phase_tab = base + p.off_phase;
     const int xf_tid = threadIdx.x - kWarpXf0 * 32;
 
-    // Per-CTA tables: (scale, 1/scale) for every non-negative E4M3 code, and
-    // for every block phase phi (column of the block's first element within
-    // its channel) the byte offsets of the block's 16 taps from that
-    // channel's origin, the columns past the channel end taken in the next
-    // channel as if it followed contiguously (chan_bytes further on).
-    const Nvfp4Global G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
+    // Per-CTA tables (quantiser tables as described at QCtx).  The phase
+    // table holds, for every block phase phi (column of the block's first
+    // element within its channel), 16 ints: with the row gather (kDWB > 0)
+    // the byte offsets of the six tap rows the block touches (column 0 of
+    // each), otherwise the byte offsets of the block's 16 taps, both from the
+    // origin of the block's first channel, the columns past the channel end
+    // taken in the next channel as if it followed contiguously (chan_bytes
+    // further on).
+    QCtx q{};
+    q.G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
+    q.dq = base + p.off_dq;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      // the window starts 11 binades below t's binade (pattern 0 if t is
+      // that small)
+      const int e_t = static_cast<int>((__float_as_uint(q.G.t) >> 23) & 0xFFu);
+      q.lo = static_cast<uint32_t>(max(e_t - 11, 0)) << 7;
+      q.hi = q.lo + static_cast<uint32_t>(kCodeEntries - 1);
+      q.cb = base + p.off_code - 2u * q.lo;
+    }
     {
-      if (p.quant && xf_tid < 128) {
-        uint32_t h2;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
-        const float s8 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-        float s = __fmul_rn(s8, G.g);
-        if (s < 1e-5f) s = 1.0f;
-        float* e = reinterpret_cast<float*>(smem + p.off_tab + xf_tid * 8);
-        e[0] = s;
-        e[1] = __frcp_rn(s);
+      if (p.quant) {
+        if (xf_tid < 128) {
+          uint32_t h2;
+          asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
+          const float s8 = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+          float s = __fmul_rn(s8, q.G.g);
+          if (s < 1e-5f) s = 1.0f;
+          const DqTable dt = dq_table(s);
+          uint32_t* e = reinterpret_cast<uint32_t*>(smem + p.off_dq + xf_tid * kDqEntryBytes);
+          e[0] = dt.lo_a;
+          e[1] = dt.lo_b;
+          e[2] = dt.hi_a;
+          e[3] = dt.hi_b;
+          e[4] = __float_as_uint(__frcp_rn(s));
+        }
+        if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+          uint16_t* ct = reinterpret_cast<uint16_t*>(smem + p.off_code);
+          for (int i = xf_tid; i < kCodeEntries; i += kNumXfWarps * 32)
+            ct[i] = static_cast<uint16_t>(entry_of_max(__uint_as_float((q.lo + static_cast<uint32_t>(i)) << 16), q) - q.dq);
+        }
       }
       int* ph = reinterpret_cast<int*>(smem + p.off_phase);
       for (int i = xf_tid; i < g.taps * 16; i += kNumXfWarps * 32) {
-        const int tt = (i >> 4) + (i & 15);
+        const int phi = i >> 4, j = i & 15;
+        if (kDWB > 0 && j >= 6) {
+          ph[i] = 0;
+          continue;
+        }
+        // tap tt from the block's first channel's origin: the block's tap j,
+        // or (row gather) column 0 of its row j
+        const int tt = kDWB > 0 ? (phi / 3 + j) * 3 : phi + j;
         const int nch = tt / g.taps;  // channels past the block's first one
         const int t = tt - nch * g.taps;
         const int chan = nch * static_cast<int>(p.chan_bytes);
@@ -795,15 +883,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
                                ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
+        const bool quant = p.quant != 0;
         bool pair_done = false;
         if constexpr (!kPairs && sizeof(T) == 2) {
           // single subtile, both blocks full and within their slots: one interleaved pass
           if (nv0 >= 32 && !cross0 && !cross1) {
+            const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0;
+            const uint32_t org1 = halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb) + thr0;
+            uint32_t pa[8], pb[8];
+            if constexpr (kDWB > 0) {
+              uint32_t ra[6], rb[6];
+              row_bases(org0, phase_tab + static_cast<uint32_t>(phi * 64), 6, 0, ra);
+              row_bases(org1, phase_tab + static_cast<uint32_t>(phi1 * 64), 6, 0, rb);
+              // the second block starts 16 columns on, one column further in the row pattern
+              switch (phi % 3) {
+                case 0: gather_rows<0, kDWB>(ra, pa); gather_rows<1, kDWB>(rb, pb); break;
+                case 1: gather_rows<1, kDWB>(ra, pa); gather_rows<2, kDWB>(rb, pb); break;
+                default: gather_rows<2, kDWB>(ra, pa); gather_rows<0, kDWB>(rb, pb); break;
+              }
+            } else {
+              int off[16];
+              load_taps(phase_tab + static_cast<uint32_t>(phi * 64), off);
+              gather_taps<T>(org0, off, 16, pa);
+              load_taps(phase_tab + static_cast<uint32_t>(phi1 * 64), off);
+              gather_taps<T>(org1, off, 16, pb);
+            }
             uint32_t wa[8], wb[8];
-            row_block_2b<T>(halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0,
-                            phase_tab + static_cast<uint32_t>(phi * 64),
-                            halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb) + thr0,
-                            phase_tab + static_cast<uint32_t>(phi1 * 64), p.quant != 0, G, tab, wa, wb);
+            quant8_x2<T>(pa, pb, quant, q, wa, wb);
             tmem_st8(a_col, wa);
             tmem_st8(a_col + 8u, wb);
             pair_done = true;
@@ -822,33 +928,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int phb = bb ? phi1 : phi, csb = bb ? cs1 : cs0, splitb = bb ? split1 : split0;
           const RingPos hb = bb ? h1 : h0;
           const uint32_t org = halo_base + hb.e * p.slot_bytes + static_cast<uint32_t>(csb * cb);
-          int off[16];
           const uint32_t prow = phase_tab + static_cast<uint32_t>(phb * 64);
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) ld_shared_v4(prow + 4u * j, off[j], off[j + 1], off[j + 2], off[j + 3]);
-          if (bb ? cross1 : cross0) {
-            // the next channel opens the next ring slot: move its columns there
+          // the block's second channel opens the next ring slot: its columns move by adj
+          int adj = 0;
+          const bool crossb = bb ? cross1 : cross0;
+          if (crossb) {
             RingPos hn = hb;
             hn.next(ring);
-            const int adj = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org) - cb;
+            adj = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org) - cb;
+          }
+          int i = 0;
+          if constexpr (kDWB > 0) {
+            if (nv >= 16) {
+              // rows of three taps: the rows of the next channel start at
+              // row (taps - phi + phi % 3) / 3 of the block
+              const int p3 = phb % 3;
+              uint32_t rb0[6];
+              row_bases(org + thr0, prow, crossb ? (g.taps - phb + p3) / 3 : 6, adj, rb0);
+              if constexpr (kPairs) {
+                for (; i + 1 < p.n_mt; i += 2) {
+                  uint32_t ra[6], rb[6], pa[8], pb[8], wa[8], wb[8];
+#pragma unroll
+                  for (int r = 0; r < 6; ++r) {
+                    ra[r] = rb0[r] + static_cast<uint32_t>(i) * thr_step;
+                    rb[r] = ra[r] + thr_step;
+                  }
+                  switch (p3) {
+                    case 0: gather_rows<0, kDWB>(ra, pa); gather_rows<0, kDWB>(rb, pb); break;
+                    case 1: gather_rows<1, kDWB>(ra, pa); gather_rows<1, kDWB>(rb, pb); break;
+                    default: gather_rows<2, kDWB>(ra, pa); gather_rows<2, kDWB>(rb, pb); break;
+                  }
+                  quant8_x2<T>(pa, pb, quant, q, wa, wb);
+                  tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
+                  tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
+                }
+              }
+              for (; i < p.n_mt; ++i) {
+                uint32_t ra[6], pa[8], wa[8];
+#pragma unroll
+                for (int r = 0; r < 6; ++r) ra[r] = rb0[r] + static_cast<uint32_t>(i) * thr_step;
+                switch (p3) {
+                  case 0: gather_rows<0, kDWB>(ra, pa); break;
+                  case 1: gather_rows<1, kDWB>(ra, pa); break;
+                  default: gather_rows<2, kDWB>(ra, pa); break;
+                }
+                quant8_1<T>(pa, quant, q, wa);
+                tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
+              }
+              continue;
+            }
+          }
+          // by tap offsets (the row-gather table is expanded to taps first)
+          int off[16];
+          if constexpr (kDWB > 0)
+            taps_from_rows<kDWB>(prow, phb % 3, off);
+          else
+            load_taps(prow, off);
+          if (crossb) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) off[j] += (j >= splitb) ? adj : 0;
           }
-          int i = 0;
           if constexpr (kPairs && sizeof(T) == 2) {
             // full blocks, subtiles in pairs: interleaved chains
             if (nv >= 16)
               for (; i + 1 < p.n_mt; i += 2) {
-                uint32_t wa[8], wb[8];
+                uint32_t pa[8], pb[8], wa[8], wb[8];
                 const uint32_t ra = org + thr0 + static_cast<uint32_t>(i) * thr_step;
-                row_block_x2<T>(ra, ra + thr_step, off, p.quant != 0, G, tab, wa, wb);
+                gather_taps<T>(ra, off, 16, pa);
+                gather_taps<T>(ra + thr_step, off, 16, pb);
+                quant8_x2<T>(pa, pb, quant, q, wa, wb);
                 tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
                 tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
               }
           }
           for (; i < p.n_mt; ++i) {
             uint32_t w[8];
-            row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, p.quant != 0, G, tab, w);
+            row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, quant, q, w);
             tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
           }
         }
@@ -914,14 +1069,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T>
-cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
-                              size_t smem, cudaStream_t s) {
-  auto kern = p.n_mt >= 2 ? conv3d_igemm_tmem_kernel<T, true> : conv3d_igemm_tmem_kernel<T, false>;
+template <typename T, bool kPairs, int kDWB>
+cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid, size_t smem,
+                             cudaStream_t s) {
+  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
   return cudaGetLastError();
+}
+
+// Row gather for 16-bit inputs and kernels three taps wide with W dilation 1
+// or 2; tap-offset gather otherwise.
+template <typename T>
+cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
+                              size_t smem, cudaStream_t s) {
+  const int dwb = row_gather_step(p.g, sizeof(T));
+  const bool pairs = p.n_mt >= 2;
+  if constexpr (sizeof(T) == 2) {
+    if (dwb == 2)
+      return pairs ? launch_tmem_inst<T, true, 2>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 2>(p, tx, tw, grid, smem, s);
+    if (dwb == 4)
+      return pairs ? launch_tmem_inst<T, true, 4>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 4>(p, tx, tw, grid, smem, s);
+  }
+  return pairs ? launch_tmem_inst<T, true, 0>(p, tx, tw, grid, smem, s)
+               : launch_tmem_inst<T, false, 0>(p, tx, tw, grid, smem, s);
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -1009,6 +1183,9 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
 
   const int chan_bytes = static_cast<int>(p.chan_bytes);
   const int phase_bytes = g.taps * 64;
+  // quantiser tables: the per-code entries, and for BF16 inputs the code
+  // table of the block maxima
+  const int code_bytes = dtype == 2 ? kCodeTableBytes : 0;
   // Halo ring: the transform warps hand a slot back as soon as they are past
   // it, so the ring only has to hold one slice's slots for progress; it is
   // sized for sa slices plus two, and any shared memory left after the
@@ -1032,8 +1209,8 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
       for (int b = 8; b >= 2; --b) {
         int r = span + 2;
         const int nbar = 2 * r + 2 * b + 2 * a + 2 * kMaxAcc + 1;
-        int total = 1024 + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
-                    64 /* pad after the halo ring */ + 1024 /* scale table */ + phase_bytes + nbar * 8 + 16;
+        int total = 1024 + kDqTableBytes + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
+                    64 /* pad after the halo ring */ + code_bytes + phase_bytes + nbar * 8 + 16;
         if (total <= kMaxSmem) {
           const int extra = std::min(32 - r, (kMaxSmem - total) / (static_cast<int>(p.slot_bytes) + 16));
           if (extra > 0) {
@@ -1041,10 +1218,11 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
             total += extra * (static_cast<int>(p.slot_bytes) + 16);
           }
           p.sa = a; p.sb = b; p.ring = r;
-          p.off_b = 0;
+          p.off_dq = 0;
+          p.off_b = kDqTableBytes;  // a multiple of 1024, as the swizzled weight stages need
           p.off_halo = p.off_b + b * p.b_stage_bytes;
-          p.off_tab = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
-          p.off_phase = p.off_tab + 1024u;
+          p.off_code = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
+          p.off_phase = p.off_code + static_cast<uint32_t>(code_bytes);
           p.off_bar = p.off_phase + static_cast<uint32_t>(phase_bytes);
           smem = static_cast<size_t>(total);
           return true;
