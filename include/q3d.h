@@ -172,6 +172,20 @@ Q3D_API q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_t
 Q3D_API q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream);
 
 /*
+ * fp4_fake_quant_bs -- fp4_fake_quant with the other block sizes the
+ * article's call accepts (sec. 7.1: fp4_block_size 16, 32, 64, 128 or 256;
+ * sec. 7.3: the flat tensor viewed as [numel / block_size, block_size]).
+ *   block_size  16, 32, 64, 128 or 256; numel % block_size == 0.
+ *   x, amax, out  as for fp4_fake_quant (block_size 16 is that call).
+ * Each block of block_size consecutive elements takes one E4M3 scale from
+ * its own |v| maximum; the quantiser is otherwise the same.  Bit-exact with
+ * the CPU oracle.  Q3D_ERR_INVALID_ARG for another block size or a numel
+ * that is not a multiple of it, before anything is enqueued.
+ */
+Q3D_API q3d_status fp4_fake_quant_bs(const q3d_tensor* x, const float* amax, int32_t block_size, q3d_tensor* out,
+                                     q3d_stream_t stream);
+
+/*
  * q3d_act_amax -- *amax = max |x| over every element of x, the global amax
  * that conv3d_implicit_gemm(quant_act) and fp4_fake_quant take.  The article
  * feeds its quantiser this scalar: its usage example (sec. 7.2) passes

@@ -24,7 +24,7 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
-           "fp4_fake_quant", "q3d_act_amax", "q3d_last_error",
+           "fp4_fake_quant", "fp4_fake_quant_bs", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
            "q3d_selftest_ratio", "q3d_plan_conv", "q3d_plan_conv_tmem")
 
@@ -66,6 +66,8 @@ def load_library(path: Optional[str] = None):
         lib.conv3d_implicit_gemm_noalloc.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.fp4_fake_quant.restype = ctypes.c_int
         lib.fp4_fake_quant.argtypes = [T, vp, T, vp]
+        lib.fp4_fake_quant_bs.restype = ctypes.c_int
+        lib.fp4_fake_quant_bs.argtypes = [T, vp, ctypes.c_int32, T, vp]
         lib.q3d_act_amax.restype = ctypes.c_int
         lib.q3d_act_amax.argtypes = [T, vp, vp]
         lib.q3d_last_error.restype = ctypes.c_char_p
@@ -215,15 +217,20 @@ def conv3d_implicit_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, out: torch.Te
 
 
 def fp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: Optional[torch.Tensor] = None,
-                   stream=None) -> torch.Tensor:
-    """NVFP4 fake-quantisation (blocks of 16 consecutive elements) through libq3d."""
+                   stream=None, block_size: int = 16) -> torch.Tensor:
+    """NVFP4 fake-quantisation through libq3d: consecutive blocks of
+    block_size (16, 32, 64, 128 or 256) elements, each with its own E4M3
+    scale.  block_size 16 calls fp4_fake_quant, the others fp4_fake_quant_bs."""
     lib = load_library()
     if out is None:
         out = torch.empty_like(x)
-    if amax.dtype != torch.float32 or amax.numel() != 1:
-        raise ValueError("amax must be a one-element float32 tensor")
+    if amax.dtype != torch.float32 or amax.numel() != 1 or amax.device != x.device:
+        raise ValueError("amax must be a one-element float32 tensor on x's device")
     xs, os_ = _tensor(x), _tensor(out)
-    st = lib.fp4_fake_quant(_ref(xs), amax.data_ptr(), _ref(os_), _stream_handle(stream))
+    if block_size == 16:
+        st = lib.fp4_fake_quant(_ref(xs), amax.data_ptr(), _ref(os_), _stream_handle(stream))
+    else:
+        st = lib.fp4_fake_quant_bs(_ref(xs), amax.data_ptr(), int(block_size), _ref(os_), _stream_handle(stream))
     _check(lib, st)
     return out
 

@@ -1,5 +1,6 @@
 // fp4_fake_quant.cu -- standalone NVFP4 fake-quantisation (Model-Optimizer
-// "Conv3D Implicit GEMM CUDA kernel" article, sec. 6.4 and 7.3).
+// "Conv3D Implicit GEMM CUDA kernel" article, sec. 6.4 and 7.3), with the
+// block sizes its call accepts (16, 32, 64, 128, 256; sec. 7.1).
 //
 // B200 design: the op is a pure stream over HBM (read 16 elements, write 16
 // elements, ~40 ALU ops per element-block).  One thread owns one block of 16
@@ -87,23 +88,40 @@ struct BlockIO<T, false> {
   }
 };
 
-template <typename T, bool kVec>
+// One thread per 16 consecutive elements; a quantisation block of 16 * G
+// elements is held by G consecutive lanes (G = 1, 2, 4, 8, 16; the article's
+// block sizes 16 .. 256, sec. 7.1), whose |v| maxima meet in xor shuffles
+// within the lane group.  The loop is uniform per warp (a warp covers 512
+// consecutive elements, a whole number of blocks), so every lane of a group
+// reaches the shuffles; lanes past the end take zeros and store nothing.
+template <typename T, bool kVec, int G>
 __global__ void __launch_bounds__(256) fp4_fake_quant_kernel(const T* x, T* y,
-                                                             const float* __restrict__ amax, int64_t nblocks) {
-  const Nvfp4Global G = nvfp4_global(__ldg(amax));
+                                                             const float* __restrict__ amax, int64_t nunits) {
+  const Nvfp4Global gs = nvfp4_global(__ldg(amax));
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b - lane < nunits; b += stride) {
+    const bool live = b < nunits;
     float v[16];
-    BlockIO<T, kVec>::load(x + b * 16, v);
+    if (live) {
+      BlockIO<T, kVec>::load(x + b * 16, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+    }
     float bmax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 16; ++i) bmax = fmaxf(bmax, fabsf(v[i]));
+    if constexpr (G > 1) {
+#pragma unroll
+      for (int o = 1; o < G; o <<= 1) bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, o));
+    }
     float scale, inv;
-    nvfp4_block_scale(bmax, G, scale, inv);
+    nvfp4_block_scale(bmax, gs, scale, inv);
     float o[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) nvfp4_pair(v[2 * i], v[2 * i + 1], inv, scale, o[2 * i], o[2 * i + 1]);
-    BlockIO<T, kVec>::store(y + b * 16, o);
+    if (live) BlockIO<T, kVec>::store(y + b * 16, o);
   }
 }
 
@@ -127,30 +145,43 @@ __global__ void selftest_ratio_kernel(const float* __restrict__ bmax, const floa
   out[i] = nvfp4_ratio(bmax[i], ti, __frcp_rn(ti));
 }
 
+template <typename T, bool kVec>
+cudaError_t launch_fq_groups(const void* x, void* y, int64_t nunits, const float* amax, int group, int grid,
+                             cudaStream_t s) {
+  const T* xi = static_cast<const T*>(x);
+  T* yo = static_cast<T*>(y);
+  switch (group) {
+    case 1: fp4_fake_quant_kernel<T, kVec, 1><<<grid, 256, 0, s>>>(xi, yo, amax, nunits); break;
+    case 2: fp4_fake_quant_kernel<T, kVec, 2><<<grid, 256, 0, s>>>(xi, yo, amax, nunits); break;
+    case 4: fp4_fake_quant_kernel<T, kVec, 4><<<grid, 256, 0, s>>>(xi, yo, amax, nunits); break;
+    case 8: fp4_fake_quant_kernel<T, kVec, 8><<<grid, 256, 0, s>>>(xi, yo, amax, nunits); break;
+    default: fp4_fake_quant_kernel<T, kVec, 16><<<grid, 256, 0, s>>>(xi, yo, amax, nunits); break;
+  }
+  return cudaGetLastError();
+}
+
 template <typename T>
-cudaError_t launch_fq_typed(const void* x, void* y, int64_t numel, const float* amax, cudaStream_t s, int sm_count) {
-  const int64_t nblocks = numel / 16;
+cudaError_t launch_fq_typed(const void* x, void* y, int64_t numel, int block, const float* amax, cudaStream_t s,
+                            int sm_count) {
+  const int64_t nunits = numel / 16;
   const int threads = 256;
-  int64_t want = (nblocks + threads - 1) / threads;
+  int64_t want = (nunits + threads - 1) / threads;
   const int64_t cap = static_cast<int64_t>(sm_count) * 8;
   const int grid = static_cast<int>(want < cap ? (want < 1 ? 1 : want) : cap);
   const bool vec = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (reinterpret_cast<uintptr_t>(y) % 16 == 0);
-  if (vec)
-    fp4_fake_quant_kernel<T, true><<<grid, threads, 0, s>>>(static_cast<const T*>(x), static_cast<T*>(y), amax, nblocks);
-  else
-    fp4_fake_quant_kernel<T, false><<<grid, threads, 0, s>>>(static_cast<const T*>(x), static_cast<T*>(y), amax, nblocks);
-  return cudaGetLastError();
+  return vec ? launch_fq_groups<T, true>(x, y, nunits, amax, block / 16, grid, s)
+             : launch_fq_groups<T, false>(x, y, nunits, amax, block / 16, grid, s);
 }
 
 }  // namespace
 
-cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, const float* amax,
+cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, int block, const float* amax,
                                   cudaStream_t s, int sm_count) {
   if (numel == 0) return cudaSuccess;
   switch (dtype) {
-    case 0: return launch_fq_typed<float>(x, y, numel, amax, s, sm_count);
-    case 1: return launch_fq_typed<__half>(x, y, numel, amax, s, sm_count);
-    default: return launch_fq_typed<__nv_bfloat16>(x, y, numel, amax, s, sm_count);
+    case 0: return launch_fq_typed<float>(x, y, numel, block, amax, s, sm_count);
+    case 1: return launch_fq_typed<__half>(x, y, numel, block, amax, s, sm_count);
+    default: return launch_fq_typed<__nv_bfloat16>(x, y, numel, block, amax, s, sm_count);
   }
 }
 

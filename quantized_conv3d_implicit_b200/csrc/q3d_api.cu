@@ -352,9 +352,16 @@ q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_tensor* w
   return Q3D_OK;
 }
 
-q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+q3d_status fake_quant_blocks(const q3d_tensor* x, const float* amax, int32_t block, q3d_tensor* out,
+                             q3d_stream_t stream) {
   if (!x || !out) return fail(Q3D_ERR_NULLPTR, "x or out is NULL");
   if (!amax) return fail(Q3D_ERR_NULLPTR, "amax is NULL");
+  if (block != 16 && block != 32 && block != 64 && block != 128 && block != 256)
+    return fail(Q3D_ERR_INVALID_ARG, "block_size %d is not 16, 32, 64, 128 or 256", block);
   if (x->ndim < 1 || x->ndim > 5) return fail(Q3D_ERR_INVALID_ARG, "x must have rank 1..5");
   q3d_status st;
   if ((st = check_tensor(x, "x", x->ndim)) != Q3D_OK) return st;
@@ -363,16 +370,30 @@ q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* ou
   for (int i = 0; i < x->ndim; ++i)
     if (out->shape[i] != x->shape[i]) return fail(Q3D_ERR_INVALID_ARG, "out must have the shape of x");
   const int64_t n = numel(x);
-  if (n % 16 != 0) return fail(Q3D_ERR_INVALID_ARG, "numel (%lld) must be a multiple of 16", (long long)n);
+  if (n % block != 0)
+    return fail(Q3D_ERR_INVALID_ARG, "numel (%lld) must be a multiple of the block size %d", (long long)n, block);
   if (n == 0) return Q3D_OK;
   if (out->data != x->data && overlaps(out, x))
     return fail(Q3D_ERR_INVALID_ARG, "out partially overlaps x");
   DeviceInfo* dev = nullptr;
   if ((st = current_device(&dev)) != Q3D_OK) return st;
-  cudaError_t e = q3d::launch_fp4_fake_quant(x->data, out->data, x->dtype, n, amax,
+  cudaError_t e = q3d::launch_fp4_fake_quant(x->data, out->data, x->dtype, n, block, amax,
                                              reinterpret_cast<cudaStream_t>(stream), dev->sm_count);
   if (e != cudaSuccess) return cuda_fail(e, "fp4_fake_quant launch");
   return Q3D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_tensor* out, q3d_stream_t stream) {
+  return fake_quant_blocks(x, amax, 16, out, stream);
+}
+
+q3d_status fp4_fake_quant_bs(const q3d_tensor* x, const float* amax, int32_t block_size, q3d_tensor* out,
+                             q3d_stream_t stream) {
+  return fake_quant_blocks(x, amax, block_size, out, stream);
 }
 
 q3d_status q3d_act_amax(const q3d_tensor* x, float* amax, q3d_stream_t stream) {

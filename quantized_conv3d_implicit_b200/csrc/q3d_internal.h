@@ -59,7 +59,8 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_tiled();
 
-cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, const float* amax,
+// block: elements per quantisation block (16, 32, 64, 128 or 256; numel a multiple of it)
+cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, int block, const float* amax,
                                   cudaStream_t s, int sm_count);
 cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, cudaStream_t s);
 cudaError_t launch_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, cudaStream_t s);

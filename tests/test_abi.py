@@ -116,6 +116,18 @@ def test_fake_quant_validation(lib):
     assert lib.fp4_fake_quant(r(T((0, 16))), FAKE * 4096, r(T((0, 16), 2, FAKE * 256)), None) == 0
 
 
+def test_fake_quant_block_size_validation(lib):
+    r = ctypes.byref
+    x, out = T((4, 64), 2, FAKE), T((4, 64), 2, FAKE * 256)
+    for bs in (0, 8, 48, 512, -16):
+        assert lib.fp4_fake_quant_bs(r(x), FAKE * 4096, bs, r(out), None) == 2, bs
+        assert b"block_size" in lib.q3d_last_error()
+    # numel 256: a multiple of 16..256; numel 96 is not a multiple of 64
+    assert lib.fp4_fake_quant_bs(r(T((6, 16))), FAKE * 4096, 64, r(T((6, 16), 2, FAKE * 256)), None) == 2
+    assert lib.fp4_fake_quant_bs(r(T((0, 64))), FAKE * 4096, 256, r(T((0, 64), 2, FAKE * 256)), None) == 0
+    assert lib.fp4_fake_quant_bs(r(x), None, 32, r(out), None) == 1
+
+
 def conv_sym(lib, x, w, out, pad=(1, 1, 1), amax=None, quant=0):
     arr = lambda v: (ctypes.c_int32 * 3)(*v) if v is not None else None  # noqa: E731
     r = lambda t: ctypes.byref(t) if t is not None else None  # noqa: E731

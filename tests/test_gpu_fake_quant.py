@@ -158,3 +158,65 @@ def test_fake_quant_full_size_workload_inputs(cuda_ok, name):
         ref = oracle.fp4_fake_quant_bits(xf[lo:hi].float().cpu().numpy(), np.float32(amax.item()), dt)
         assert np.array_equal(bits(yf[lo:hi]), ref), (name, s)
     assert api.check_device_error() == 0
+
+
+# --- the article's other block sizes (sec. 7.1: fp4_block_size 16..256) ---
+
+BLOCK_SIZES = (16, 32, 64, 128, 256)
+
+
+def _ref_bs(x, amax, bs, dt):
+    return oracle.round_to_dtype_bits(oracle.fp4_fake_quant_bs(x, np.float32(amax), bs), dt)
+
+
+@pytest.mark.parametrize("dtype", list(DTYPES))
+@pytest.mark.parametrize("bs", BLOCK_SIZES)
+@pytest.mark.parametrize("amax_mode", ["max", "zero", "small"])
+def test_fake_quant_block_sizes_bit_exact(cuda_ok, dtype, bs, amax_mode):
+    # 1007 blocks: a numel that is a multiple of bs but not of 512 elements
+    # (the span of one warp), so the last warp holds a partial span
+    x = _blocks(11, 1007 * bs // 16, dtype).reshape(-1)
+    xm = float(x.float().abs().max())
+    amax = {"max": xm, "zero": 0.0, "small": xm / 50}[amax_mode]
+    y = api.fp4_fake_quant(x.cuda(), torch.tensor([amax], dtype=torch.float32).cuda(), block_size=bs)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(y), _ref_bs(x.float().numpy(), amax, bs, DTYPES[dtype]))
+
+
+@pytest.mark.parametrize("dtype", list(DTYPES))
+@pytest.mark.parametrize("bs", (32, 256))
+def test_fake_quant_block_sizes_unaligned_and_inplace(cuda_ok, dtype, bs):
+    x = _blocks(12, 300 * bs // 16 + 1, dtype).reshape(-1).cuda()
+    amax = x.float().abs().max().reshape(1)
+    n = 299 * bs
+    for off in (16, 1):
+        xs = x[off: off + n]
+        y = api.fp4_fake_quant(xs, amax, block_size=bs)
+        assert np.array_equal(bits(y), _ref_bs(xs.float().cpu().numpy(), amax.item(), bs, DTYPES[dtype])), off
+    z = x[:n].clone()
+    api.fp4_fake_quant(z, amax, out=z, block_size=bs)
+    assert np.array_equal(bits(z), _ref_bs(x[:n].float().cpu().numpy(), amax.item(), bs, DTYPES[dtype]))
+
+
+def test_fake_quant_block_size_errors_and_empty(cuda_ok):
+    amax = torch.ones(1, device="cuda")
+    with pytest.raises(api.Q3DError):
+        api.fp4_fake_quant(torch.zeros(96, device="cuda"), amax, block_size=64)
+    with pytest.raises(api.Q3DError):
+        api.fp4_fake_quant(torch.zeros(96, device="cuda"), amax, block_size=48)
+    assert api.fp4_fake_quant(torch.empty(0, device="cuda"), amax, block_size=256).numel() == 0
+
+
+def test_fake_quant_block_128_on_a_full_layer_input(cuda_ok):
+    # the article's default block size on a whole activation tensor, sampled
+    inp = workloads.make_inputs("wan_mid_384_bf16", device="cuda")
+    x, amax = inp["x"].reshape(-1), inp["act_amax"]
+    y = api.fp4_fake_quant(x, amax, block_size=128)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(8)
+    nb = x.numel() // 128
+    for s in np.unique(np.concatenate([[0, nb - 512], rng.integers(0, nb - 512, 32)])):
+        lo, hi = int(s) * 128, (int(s) + 512) * 128
+        assert np.array_equal(bits(y[lo:hi]), _ref_bs(x[lo:hi].float().cpu().numpy(), amax.item(), 128,
+                                                       "bfloat16")), s
+    assert api.check_device_error() == 0
