@@ -10,8 +10,12 @@ The arithmetic lives in ``q3d_oracle.c`` (plain C, compiled with gcc,
 Every function states the passage of the Model-Optimizer "Conv3D Implicit
 GEMM CUDA kernel" article it follows (sections 5.1, 6.1-6.4, 7.1).
 
+The MXFP4 functions follow the CANN aclnnFlatQuantV2 page instead (its
+per-group route with E2M1 output, steps 3 and 4).
+
 Parity pins: tests/test_oracle_formats.py, tests/test_oracle_fake_quant.py,
-tests/test_oracle_conv.py.  No function here is "parity unpinned".
+tests/test_oracle_conv.py, tests/test_oracle_mxfp4.py.  No function here is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -62,6 +66,12 @@ def _load():
             lib.oracle_fp4_fake_quant.argtypes = [vp, i64, f32, vp]
             lib.oracle_fp4_fake_quant_bs.restype = ctypes.c_int
             lib.oracle_fp4_fake_quant_bs.argtypes = [vp, i64, f32, ctypes.c_int, vp]
+            lib.oracle_mx_scale_exp.restype = ctypes.c_int
+            lib.oracle_mx_scale_exp.argtypes = [f32, f32]
+            lib.oracle_mxfp4_block.restype = ctypes.c_int
+            lib.oracle_mxfp4_block.argtypes = [vp, ctypes.c_int, f32, vp, vp]
+            lib.oracle_mxfp4_fake_quant.restype = ctypes.c_int
+            lib.oracle_mxfp4_fake_quant.argtypes = [vp, i64, f32, vp, vp, vp]
             lib.oracle_act_amax.restype = f32
             lib.oracle_act_amax.argtypes = [vp, i64]
             lib.oracle_round_to_dtype_bits.restype = None
@@ -158,6 +168,45 @@ def fp4_fake_quant_bs(x, amax: float, block_size: int) -> np.ndarray:
     if rc != 0:
         raise ValueError("block_size must be 16, 32, 64, 128 or 256 and divide numel")
     return out
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 (the CANN aclnnFlatQuantV2 page: per-group route, steps 3 and 4)
+# ---------------------------------------------------------------------------
+
+def mx_scale_exp(amax: float, dst_max: float = 0.0) -> int:
+    """Shared exponent E of an MXFP4 group (scale 2^E) from its |v| maximum:
+    floor(log2 amax) - 2 when dst_max is 0, else the exponent of
+    amax / dst_max rounded up when that quotient is not a power of two."""
+    return int(_load().oracle_mx_scale_exp(float(np.float32(amax)), float(np.float32(dst_max))))
+
+
+def mxfp4_block(v, dst_max: float = 0.0):
+    """One group (1..32 values): (dequantised binary32 values, signed 4-bit
+    codes, E)."""
+    lib = _load()
+    v = _f32(v)
+    out = np.empty_like(v)
+    codes = np.empty(v.shape, np.uint8)
+    e = lib.oracle_mxfp4_block(_ptr(v), int(v.size), float(np.float32(dst_max)), _ptr(out),
+                               codes.ctypes.data_as(ctypes.c_void_p))
+    return out, codes, int(e)
+
+
+def mxfp4_fake_quant(x, dst_max: float = 0.0):
+    """MXFP4 over the fp32 values of x (numel % 32 == 0, groups of 32
+    consecutive elements): (dequantised binary32 values in x's shape, E8M0
+    scale bytes [numel / 32], signed 4-bit codes [numel])."""
+    lib = _load()
+    x = _f32(x)
+    out = np.empty_like(x)
+    scales = np.empty(x.size // 32, np.uint8)
+    codes = np.empty(x.size, np.uint8)
+    rc = lib.oracle_mxfp4_fake_quant(_ptr(x), x.size, float(np.float32(dst_max)), _ptr(out),
+                                     scales.ctypes.data_as(ctypes.c_void_p), codes.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError("numel must be a multiple of 32 and dst_max 0 or in [6, 12]")
+    return out, scales, codes
 
 
 def act_amax(x) -> np.float32:

@@ -26,6 +26,11 @@
  * Where the article stops (rounding of E2M1 ties and of the E4M3 scale) the
  * specification of this library fixes round-to-nearest-even for both.
  *
+ * The MXFP4 functions follow a second page, the CANN aclnnFlatQuantV2
+ * article (its per-group route with E2M1 output: groups of 32, a
+ * power-of-two E8M0 scale, the dstTypeMax rule); see the comment above
+ * oracle_mx_scale_exp.
+ *
  * Every floating-point step of the fake-quantiser is one IEEE-754 binary32
  * operation with round-to-nearest-even, written in the order the article
  * gives it.  Build with -ffp-contract=off and without -ffast-math so the C
@@ -207,6 +212,93 @@ int oracle_fp4_fake_quant_bs(const float* x, int64_t numel, float amax, int bloc
     if (block != 16 && block != 32 && block != 64 && block != 128 && block != 256) return -1;
     if (numel % block != 0) return -1;
     for (int64_t b = 0; b < numel; b += block) oracle_fq_block(x + b, block, amax, out + b);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 (E2M1 values, power-of-two E8M0 scale, groups of 32)                */
+/* ------------------------------------------------------------------------ */
+
+/* Source: the CANN aclnnFlatQuantV2 page (its step 3, the per-group route
+ * with FLOAT4_E2M1 output, and step 4, the dstTypeMax rule).  A group of 32
+ * consecutive elements shares one scale 2^E stored as E8M0 (exponent only,
+ * E in [-127, 127], biased code E + 127):
+ *   dst_max == 0  (step 3): E = floor(log2(max|v|)) - emax, emax = 2, the
+ *                 exponent of E2M1's largest magnitude 6 = 1.5 * 2^2;
+ *   dst_max != 0  (step 4): S = max|v| / dst_max in binary32; E is the
+ *                 unbiased exponent of S, raised by one when S is a normal
+ *                 number with a biased exponent below 254 and a nonzero
+ *                 mantissa (the scale rounds up, so no element exceeds
+ *                 dst_max before the E2M1 rounding).
+ * Each element becomes E2M1_RNE_SAT(v * 2^-E) (the product is exact) and
+ * dequantises to that code times 2^E.  Readings where the page is silent:
+ * floor(log2) of a zero or subnormal maximum, and the exponent of a
+ * subnormal S, clamp to -127 (the E8M0 minimum); E is clamped to <= 127. */
+static int mx_floor_log2(float a)
+{
+    /* exponent of a binary32 value; zero and subnormals give -127 */
+    uint32_t u;
+    memcpy(&u, &a, 4);
+    int be = (int)((u >> 23) & 0xffu);
+    if (be == 0) return -127;
+    return be - 127;
+}
+
+int oracle_mx_scale_exp(float amax, float dst_max)
+{
+    int e;
+    if (dst_max == 0.0f) {
+        e = mx_floor_log2(amax) - 2;
+    } else {
+        float s = amax / dst_max;
+        uint32_t u;
+        memcpy(&u, &s, 4);
+        int be = (int)((u >> 23) & 0xffu);
+        e = mx_floor_log2(s);
+        if (be != 0 && be < 254 && (u & 0x007fffffu) != 0) e += 1;
+    }
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* One group of n values (n = 32 in the call below): codes[i] receives the
+ * signed 4-bit E2M1 code (sign bit 3, magnitude code 0..7), out[i] the
+ * dequantised binary32 value; returns E. */
+int oracle_mxfp4_block(const float* v, int n, float dst_max, float* out, uint8_t* codes)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > amax) amax = a;
+    }
+    int e = oracle_mx_scale_exp(amax, dst_max);
+    double down = ldexp(1.0, -e), up = ldexp(1.0, e);
+    for (int i = 0; i < n; ++i) {
+        float x = (float)((double)v[i] * down);      /* exact: a power of two */
+        float q = oracle_e2m1_rne_sat(x);
+        int mag = 0;
+        while (mag < 7 && kE2M1Mag[mag] != fabs((double)q)) ++mag;
+        if (codes) codes[i] = (uint8_t)(mag | (signbit(q) ? 8 : 0));
+        out[i] = (float)((double)q * up);
+    }
+    return e;
+}
+
+/* MXFP4 over a flat tensor (numel % 32 == 0): out receives the dequantised
+ * values, scales (if not NULL) the E8M0 byte E + 127 of each group, codes (if
+ * not NULL) the signed 4-bit code of each element.  Returns 0, or -1 for a
+ * numel that is not a multiple of 32 or a dst_max that is neither 0 nor in
+ * [6, 12]. */
+int oracle_mxfp4_fake_quant(const float* x, int64_t numel, float dst_max, float* out, uint8_t* scales,
+                            uint8_t* codes)
+{
+    if (numel % 32 != 0) return -1;
+    if (!(dst_max == 0.0f || (dst_max >= 6.0f && dst_max <= 12.0f))) return -1;
+    for (int64_t b = 0; b < numel; b += 32) {
+        int e = oracle_mxfp4_block(x + b, 32, dst_max, out + b, codes ? codes + b : NULL);
+        if (scales) scales[b / 32] = (uint8_t)(e + 127);
+    }
     return 0;
 }
 
