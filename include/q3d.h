@@ -14,7 +14,10 @@
  *     scales, blocks of 16 consecutive K elements of one A row, global scale
  *     act_amax / (6*448), tiny-scale fallback 1.0), rounding to nearest even;
  *   - fp4_fake_quant: sec. 6.4 and 7.3 (the same quantiser on a flat tensor
- *     viewed as [numel/16, 16]).
+ *     viewed as [numel/16, 16]), fp4_fake_quant_bs the block sizes 32..256
+ *     of sec. 7.1.
+ * mxfp4_quantize follows a second page, the CANN aclnnFlatQuantV2 article
+ * (MXFP4: E2M1 with a power-of-two scale per 32 elements).
  *
  * Conventions for every call:
  *   - All tensor data pointers are DEVICE pointers to contiguous row-major
@@ -184,6 +187,33 @@ Q3D_API q3d_status fp4_fake_quant(const q3d_tensor* x, const float* amax, q3d_te
  */
 Q3D_API q3d_status fp4_fake_quant_bs(const q3d_tensor* x, const float* amax, int32_t block_size, q3d_tensor* out,
                                      q3d_stream_t stream);
+
+/*
+ * mxfp4_quantize -- MXFP4 quantisation of x: groups of 32 consecutive
+ * elements (memory order) share one power-of-two scale 2^E, stored as an
+ * E8M0 byte E + 127, and every element becomes an E2M1 value (round to
+ * nearest, ties to even, saturating at 6).  Follows the CANN
+ * aclnnFlatQuantV2 page, its per-group route with FLOAT4_E2M1 output
+ * (step 3) and the dstTypeMax rule (step 4):
+ *   dst_type_max == 0:  E = floor(log2(group max |x|)) - 2;
+ *   dst_type_max in [6, 12]:  E = exponent of S = group max / dst_type_max
+ *       (binary32 division), plus one when S is normal, below the top binade
+ *       and not a power of two (the scale rounds up);
+ *   E is clamped to [-127, 127] (a zero or subnormal maximum or S gives -127).
+ * Arguments (device pointers, caller-owned):
+ *   x       rank 1..5, F32/F16/BF16, numel % 32 == 0.
+ *   out     NULL, or the dequantised tensor E2M1 * 2^E in x's shape and
+ *           dtype (may be x itself, not a partial overlap).
+ *   scales  NULL, or numel / 32 bytes: the E8M0 byte of each group in order.
+ *   codes   NULL, or numel / 2 bytes of packed E2M1 codes (sign in bit 3 of
+ *           each nibble; element 2i in the low nibble of byte i).
+ * At least one of out, scales, codes; none may overlap x or each other.
+ * Bit-exact with the CPU oracle.  Q3D_ERR_NULLPTR / _INVALID_ARG (numel,
+ * dst_type_max, shape, overlap) / _UNSUPPORTED_DTYPE before anything is
+ * enqueued.
+ */
+Q3D_API q3d_status mxfp4_quantize(const q3d_tensor* x, float dst_type_max, q3d_tensor* out, uint8_t* scales,
+                                  uint8_t* codes, q3d_stream_t stream);
 
 /*
  * q3d_act_amax -- *amax = max |x| over every element of x, the global amax

@@ -24,7 +24,7 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
 EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
-           "fp4_fake_quant", "fp4_fake_quant_bs", "q3d_act_amax", "q3d_last_error",
+           "fp4_fake_quant", "fp4_fake_quant_bs", "mxfp4_quantize", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
            "q3d_selftest_ratio", "q3d_plan_conv", "q3d_plan_conv_tmem")
 
@@ -68,6 +68,8 @@ def load_library(path: Optional[str] = None):
         lib.fp4_fake_quant.argtypes = [T, vp, T, vp]
         lib.fp4_fake_quant_bs.restype = ctypes.c_int
         lib.fp4_fake_quant_bs.argtypes = [T, vp, ctypes.c_int32, T, vp]
+        lib.mxfp4_quantize.restype = ctypes.c_int
+        lib.mxfp4_quantize.argtypes = [T, ctypes.c_float, T, vp, vp, vp]
         lib.q3d_act_amax.restype = ctypes.c_int
         lib.q3d_act_amax.argtypes = [T, vp, vp]
         lib.q3d_last_error.restype = ctypes.c_char_p
@@ -233,6 +235,25 @@ def fp4_fake_quant(x: torch.Tensor, amax: torch.Tensor, out: Optional[torch.Tens
         st = lib.fp4_fake_quant_bs(_ref(xs), amax.data_ptr(), int(block_size), _ref(os_), _stream_handle(stream))
     _check(lib, st)
     return out
+
+
+def mxfp4_quantize(x: torch.Tensor, dst_type_max: float = 0.0, out: Optional[torch.Tensor] = None,
+                   want_out: bool = True, want_codes: bool = True, stream=None):
+    """MXFP4 through libq3d: groups of 32 elements with a power-of-two E8M0
+    scale.  Returns (dequantised tensor or None, E8M0 scale bytes [numel/32],
+    packed E2M1 codes [numel/2] or None)."""
+    lib = load_library()
+    if want_out and out is None:
+        out = torch.empty_like(x)
+    n = x.numel()
+    scales = torch.empty(n // 32, dtype=torch.uint8, device=x.device)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=x.device) if want_codes else None
+    xs = _tensor(x)
+    os_ = _tensor(out) if want_out else None
+    st = lib.mxfp4_quantize(_ref(xs), float(dst_type_max), _ref(os_), scales.data_ptr() if n else None,
+                            codes.data_ptr() if (codes is not None and n) else None, _stream_handle(stream))
+    _check(lib, st)
+    return (out if want_out else None), scales, codes
 
 
 def act_amax(x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

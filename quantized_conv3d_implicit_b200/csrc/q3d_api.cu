@@ -396,6 +396,50 @@ q3d_status fp4_fake_quant_bs(const q3d_tensor* x, const float* amax, int32_t blo
   return fake_quant_blocks(x, amax, block_size, out, stream);
 }
 
+q3d_status mxfp4_quantize(const q3d_tensor* x, float dst_type_max, q3d_tensor* out, uint8_t* scales, uint8_t* codes,
+                          q3d_stream_t stream) {
+  if (!x) return fail(Q3D_ERR_NULLPTR, "x is NULL");
+  if (!out && !scales && !codes) return fail(Q3D_ERR_NULLPTR, "out, scales and codes are all NULL");
+  if (!(dst_type_max == 0.0f || (dst_type_max >= 6.0f && dst_type_max <= 12.0f)))
+    return fail(Q3D_ERR_INVALID_ARG, "dst_type_max must be 0 or in [6, 12]");
+  if (x->ndim < 1 || x->ndim > 5) return fail(Q3D_ERR_INVALID_ARG, "x must have rank 1..5");
+  q3d_status st;
+  if ((st = check_tensor(x, "x", x->ndim)) != Q3D_OK) return st;
+  if (out) {
+    if ((st = check_tensor(out, "out", x->ndim)) != Q3D_OK) return st;
+    if (out->dtype != x->dtype) return fail(Q3D_ERR_UNSUPPORTED_DTYPE, "out must have the dtype of x");
+    for (int i = 0; i < x->ndim; ++i)
+      if (out->shape[i] != x->shape[i]) return fail(Q3D_ERR_INVALID_ARG, "out must have the shape of x");
+  }
+  const int64_t n = numel(x);
+  if (n % 32 != 0) return fail(Q3D_ERR_INVALID_ARG, "numel (%lld) must be a multiple of 32", (long long)n);
+  if (n == 0) return Q3D_OK;
+  const uintptr_t x0 = reinterpret_cast<uintptr_t>(x->data), x1 = x0 + static_cast<uintptr_t>(n * dtype_size(x->dtype));
+  if (out && out->data != x->data && overlaps(out, x)) return fail(Q3D_ERR_INVALID_ARG, "out partially overlaps x");
+  const struct { const uint8_t* p; int64_t bytes; const char* name; } side[2] = {{scales, n / 32, "scales"},
+                                                                                 {codes, n / 2, "codes"}};
+  for (const auto& b : side) {
+    if (!b.p) continue;
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(b.p), b1 = b0 + static_cast<uintptr_t>(b.bytes);
+    if (b0 < x1 && x0 < b1) return fail(Q3D_ERR_INVALID_ARG, "%s overlaps x", b.name);
+    if (out) {
+      const uintptr_t o0 = reinterpret_cast<uintptr_t>(out->data), o1 = o0 + (x1 - x0);
+      if (b0 < o1 && o0 < b1) return fail(Q3D_ERR_INVALID_ARG, "%s overlaps out", b.name);
+    }
+  }
+  if (scales && codes) {
+    const uintptr_t s0 = reinterpret_cast<uintptr_t>(scales), c0 = reinterpret_cast<uintptr_t>(codes);
+    if (s0 < c0 + static_cast<uintptr_t>(n / 2) && c0 < s0 + static_cast<uintptr_t>(n / 32))
+      return fail(Q3D_ERR_INVALID_ARG, "scales overlaps codes");
+  }
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  cudaError_t e = q3d::launch_mxfp4(x->data, out ? out->data : nullptr, scales, codes, x->dtype, n, dst_type_max,
+                                    reinterpret_cast<cudaStream_t>(stream), dev->sm_count);
+  if (e != cudaSuccess) return cuda_fail(e, "mxfp4 launch");
+  return Q3D_OK;
+}
+
 q3d_status q3d_act_amax(const q3d_tensor* x, float* amax, q3d_stream_t stream) {
   if (!x) return fail(Q3D_ERR_NULLPTR, "x is NULL");
   if (!amax) return fail(Q3D_ERR_NULLPTR, "amax is NULL");

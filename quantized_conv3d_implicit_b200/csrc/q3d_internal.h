@@ -62,6 +62,10 @@ EncodeTiledFn get_encode_tiled();
 // block: elements per quantisation block (16, 32, 64, 128 or 256; numel a multiple of it)
 cudaError_t launch_fp4_fake_quant(const void* x, void* y, int dtype, int64_t numel, int block, const float* amax,
                                   cudaStream_t s, int sm_count);
+// MXFP4 over numel elements (numel % 32 == 0): any of y (dequantised, dtype),
+// scales (E8M0 byte per group of 32) and codes (packed E2M1, 2 per byte) may be null.
+cudaError_t launch_mxfp4(const void* x, void* y, uint8_t* scales, uint8_t* codes, int dtype, int64_t numel,
+                         float dst_max, cudaStream_t s, int sm_count);
 cudaError_t launch_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, cudaStream_t s);
 cudaError_t launch_selftest_ratio(const float* bmax, const float* t, int64_t n, float* out, cudaStream_t s);
 // *amax = max |x| over n elements of dtype (0 when n == 0); zeroes *amax on s first.

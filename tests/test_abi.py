@@ -190,3 +190,17 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
 def test_python_binding_errors_without_library(tmp_path):
     with pytest.raises(RuntimeError):
         api.load_library(str(tmp_path / "missing.so"))
+
+
+def test_mxfp4_validation(lib):
+    r = ctypes.byref
+    x, out = T((4, 64), 2, FAKE), T((4, 64), 2, FAKE * 256)
+    assert lib.mxfp4_quantize(None, 0.0, r(out), None, None, None) == 1
+    assert lib.mxfp4_quantize(r(x), 0.0, None, None, None, None) == 1          # nothing to write
+    for bad in (1.0, 5.5, 12.5, -6.0):
+        assert lib.mxfp4_quantize(r(x), bad, r(out), None, None, None) == 2
+    assert lib.mxfp4_quantize(r(T((3, 16))), 0.0, r(T((3, 16), 2, FAKE * 256)), None, None, None) == 2   # 48 % 32
+    assert lib.mxfp4_quantize(r(x), 0.0, r(T((4, 64), 1, FAKE * 256)), None, None, None) == 3
+    assert lib.mxfp4_quantize(r(x), 0.0, None, FAKE + 8, None, None) == 2        # scales inside x
+    assert lib.mxfp4_quantize(r(x), 0.0, None, FAKE * 4096, FAKE * 4096 + 4, None) == 2   # scales overlap codes
+    assert lib.mxfp4_quantize(r(T((0, 64))), 0.0, None, FAKE * 4096, None, None) == 0
