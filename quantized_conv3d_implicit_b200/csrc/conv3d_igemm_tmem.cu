@@ -87,7 +87,8 @@ struct TmemParams {
   int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
-  uint32_t off_dq, off_b, off_halo, off_code, off_phase, off_bar;
+  uint32_t off_dq, off_b, off_halo, off_code, off_epi, off_phase, off_bar;
+  int y_vec;  // y is 16-byte aligned and OW a multiple of 16 / sizeof(T): vector stores
 };
 
 struct TileCoord {
@@ -693,22 +694,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpEpi0 && warp < kWarpEpi0 + 4) {
     // ------------------------------------------------------------ epilogue
+    // Warp qw drains TMEM lanes 32*qw.. (subtile rows = output positions), 16
+    // channels per step: tcgen05.ld gives each lane its position's 16 FP32
+    // accumulators, the bias is added in FP32 and the result rounded to the
+    // output dtype, and the 32 positions x 16 channels pass through the
+    // warp's shared staging rows (one row of 32 positions per channel), so
+    // that each lane then writes kPer consecutive ow of one channel as one
+    // 16-byte store.  A lane's store unit covers positions kPer*gq..+kPer-1 of
+    // the warp (one row segment, since kPer divides TW), the same for every
+    // step; units at the ragged edge of OW fall back to element stores.  When
+    // OW is not a multiple of kPer (or y is not 16-byte aligned) no row start
+    // is aligned, and each lane instead writes its own position for the 16
+    // channels (consecutive lanes hold consecutive ow).  The accumulator is
+    // handed back to the MMA as soon as its last step is in registers.
+    constexpr int kEsz = static_cast<int>(sizeof(T));
+    constexpr int kPer = 16 / kEsz;          // positions per 16-byte store
+    constexpr int kGroups = 32 / kPer;       // store units per channel row
+    constexpr int kUnits = kGroups / 2;      // store units per lane per step (16 channels x kGroups / 32)
+    constexpr uint32_t kPitch = 32 * kEsz + 16;
     const int qw = warp - kWarpEpi0;  // == warp % 4: TMEM lanes 32*qw..
-    const int lr = qw * 32 + lane;    // row within a subtile
-    const int th_l = lr / p.TW, tw_l = lr % p.TW;
+    const uint32_t stage = base + p.off_epi + static_cast<uint32_t>(qw) * 16u * kPitch;
+    const int gq = lane % kGroups;           // this lane's position group
+    const int r0 = qw * 32 + gq * kPer;      // its first row within a subtile
+    const int th_u = r0 / p.TW, tw_u = r0 % p.TW;
     const int S_hw = g.OH * g.OW;
     const int64_t S = static_cast<int64_t>(g.OD) * S_hw;
+    const bool vec_ok = p.y_vec != 0;
     T* y = static_cast<T*>(p.y);
     const T* bias = static_cast<const T*>(p.bias);
     uint32_t it = 0;
     bool ok = true;
     for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
       const TileCoord tc = decode_tile(p, t);
-      const int ow = tc.ow0 + tw_l;
+      const int ow = tc.ow0 + tw_u;
       for (int i = 0; ok && i < p.n_mt; ++i) {
-        const int oh = tc.oh0 + i * p.TH + th_l;
-        const bool valid = oh < g.OH && ow < g.OW;
-        const int64_t ybase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
+        const int oh = tc.oh0 + i * p.TH + th_u;
+        const bool row_ok = oh < g.OH && ow < g.OW;
+        const bool full = row_ok && ow + kPer <= g.OW;
+        const int64_t ubase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
                               static_cast<int64_t>(oh) * g.OW + ow;
         for (int ns = 0; ns < p.n_sub; ++ns) {
           const int acc = i * p.n_sub + ns;
@@ -724,21 +747,78 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t v[16];
             tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
             tmem_wait_ld();
-            if (valid) {
+            if (c0 + 16 >= p.sub_n) {  // the accumulator is in registers: hand it back
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar_acc_empty + 8u * acc);
+            }
+            if (!vec_ok) {
+              // rows whose length breaks 16-byte alignment: each lane writes its
+              // own position for the 16 channels (consecutive lanes, consecutive ow)
+              const int r = qw * 32 + lane;
+              const int ohp = tc.oh0 + i * p.TH + r / p.TW, owp = tc.ow0 + r % p.TW;
+              if (ohp < g.OH && owp < g.OW) {
+                T* dst = y + (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
+                         static_cast<int64_t>(ohp) * g.OW + owp;
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int co = co0 + c0 + j;
-                if (co < g.Cout) {
-                  float f = __uint_as_float(v[j]);
-                  if (bias) f = __fadd_rn(f, DTypeOps<T>::to_f32(bias[co]));
-                  y[ybase + static_cast<int64_t>(co) * S] = DTypeOps<T>::from_f32(f);
+                for (int j = 0; j < 16; ++j) {
+                  const int co = co0 + c0 + j;
+                  if (co < g.Cout) {
+                    float f = __uint_as_float(v[j]);
+                    if (bias) f = __fadd_rn(f, DTypeOps<T>::to_f32(__ldg(bias + co)));
+                    dst[static_cast<int64_t>(co) * S] = DTypeOps<T>::from_f32(f);
+                  }
+                }
+              }
+              continue;
+            }
+            // bias, rounding, and the staging rows (row j = channel co0 + c0 + j)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int co = co0 + c0 + j;
+              float f = __uint_as_float(v[j]);
+              if (bias && co < g.Cout) f = __fadd_rn(f, DTypeOps<T>::to_f32(__ldg(bias + co)));
+              const T o = DTypeOps<T>::from_f32(f);
+              const uint32_t a = stage + static_cast<uint32_t>(j) * kPitch + static_cast<uint32_t>(lane * kEsz);
+              if constexpr (kEsz == 2) {
+                unsigned short b;
+                memcpy(&b, &o, 2);
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(a), "h"(b) : "memory");
+              } else {
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(__float_as_uint(f)) : "memory");
+              }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < kUnits; ++k) {
+              const int j = lane / kGroups + k * (32 / kGroups);
+              const int co = co0 + c0 + j;
+              if (co < g.Cout && row_ok) {
+                const uint32_t a = stage + static_cast<uint32_t>(j) * kPitch + static_cast<uint32_t>(gq * 16);
+                int w0, w1, w2, w3;
+                ld_shared_v4(a, w0, w1, w2, w3);
+                T* dst = y + ubase + static_cast<int64_t>(co) * S;
+                if (full) {
+                  __stcs(reinterpret_cast<int4*>(dst), make_int4(w0, w1, w2, w3));
+                } else {
+                  const uint32_t ws[4] = {static_cast<uint32_t>(w0), static_cast<uint32_t>(w1),
+                                          static_cast<uint32_t>(w2), static_cast<uint32_t>(w3)};
+#pragma unroll
+                  for (int e = 0; e < kPer; ++e) {
+                    if (ow + e < g.OW) {
+                      if constexpr (kEsz == 2) {
+                        const unsigned short b = static_cast<unsigned short>(ws[e >> 1] >> (16 * (e & 1)));
+                        memcpy(dst + e, &b, 2);
+                      } else {
+                        dst[e] = __uint_as_float(ws[e]);
+                      }
+                    }
+                  }
                 }
               }
             }
+            __syncwarp();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar_acc_empty + 8u * acc);
         }
       }
     }
@@ -1186,6 +1266,8 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   // quantiser tables: the per-code entries, and for BF16 inputs the code
   // table of the block maxima
   const int code_bytes = dtype == 2 ? kCodeTableBytes : 0;
+  // epilogue staging: 4 warps x 16 channel rows x (32 positions + 16 bytes)
+  const int epi_bytes = 4 * 16 * (32 * esz + 16);
   // Halo ring: the transform warps hand a slot back as soon as they are past
   // it, so the ring only has to hold one slice's slots for progress; it is
   // sized for sa slices plus two, and any shared memory left after the
@@ -1210,7 +1292,7 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
         int r = span + 2;
         const int nbar = 2 * r + 2 * b + 2 * a + 2 * kMaxAcc + 1;
         int total = 1024 + kDqTableBytes + b * static_cast<int>(p.b_stage_bytes) + r * static_cast<int>(p.slot_bytes) +
-                    64 /* pad after the halo ring */ + code_bytes + phase_bytes + nbar * 8 + 16;
+                    64 /* pad after the halo ring */ + code_bytes + epi_bytes + phase_bytes + nbar * 8 + 16;
         if (total <= kMaxSmem) {
           const int extra = std::min(32 - r, (kMaxSmem - total) / (static_cast<int>(p.slot_bytes) + 16));
           if (extra > 0) {
@@ -1222,7 +1304,8 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
           p.off_b = kDqTableBytes;  // a multiple of 1024, as the swizzled weight stages need
           p.off_halo = p.off_b + b * p.b_stage_bytes;
           p.off_code = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
-          p.off_phase = p.off_code + static_cast<uint32_t>(code_bytes);
+          p.off_epi = p.off_code + static_cast<uint32_t>(code_bytes);
+          p.off_phase = p.off_epi + static_cast<uint32_t>(epi_bytes);
           p.off_bar = p.off_phase + static_cast<uint32_t>(phase_bytes);
           smem = static_cast<size_t>(total);
           return true;
@@ -1255,6 +1338,7 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   size_t smem = 0;
   if (!plan_tmem(g, L.dtype, p, smem)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
+  p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;
 
   EncodeTiledFn encode = get_encode_tiled();
   if (!encode) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }
