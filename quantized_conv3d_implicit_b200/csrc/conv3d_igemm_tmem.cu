@@ -60,7 +60,6 @@ constexpr int kBlockK = 64;
 constexpr int kMaxSmem = 232448;  // 227 KB dynamic shared memory per CTA
 constexpr int kMaxAcc = 8;
 constexpr int kMaxTaps = 343;     // 7x7x7
-constexpr int kMaxStages = 8;     // A stages in tensor memory
 constexpr uint32_t kTmemCols = 512;
 
 struct TmemParams {
@@ -85,8 +84,7 @@ struct TmemParams {
   int sa, sb;
   uint32_t b_stage_bytes;
   int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
-  int groups;             // transform groups (2 or 4): a warp's step is groups K slices
-  int dks_c, dks_phi;     // groups * 64 = dks_c * taps + dks_phi (a transform warp's step)
+  int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
   uint32_t off_dq, off_b, off_halo, off_code, off_epi, off_phase, off_bar;
@@ -574,10 +572,8 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
 // (a separate instantiation, so single-subtile tiles keep their register
 // allocation).  kDWB > 0: 16-bit input and a kernel three taps wide whose
 // taps along W are kDWB bytes apart (dilation * element size), gathered by
-// rows with immediate column offsets; 0: gathered by tap offsets.  kG:
-// transform groups (2 or 4); group g builds the K slices of index g mod kG,
-// each warp kG adjacent 16-column blocks of them.
-template <typename T, bool kPairs, int kDWB, int kG>
+// rows with immediate column offsets; 0: gathered by tap offsets.
+template <typename T, bool kPairs, int kDWB>
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
                              const __grid_constant__ CUtensorMap tmap_w) {
@@ -613,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_b_empty + 8u * i, 1);
     }
     for (int i = 0; i < p.sa; ++i) {
-      mbar_init(bar_a_full + 8u * i, kNumXfWarps / kG);  // the warps of the slice's group
+      mbar_init(bar_a_full + 8u * i, kNumXfWarps / 2);  // the 8 warps of the slice's group
       mbar_init(bar_a_empty + 8u * i, 1);
     }
     for (int i = 0; i < kMaxAcc; ++i) {
@@ -828,17 +824,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kWarpXf0) {
     // ------------------------------------------------------------ transform
-    // kG groups of 16 / kG warps take the K slices whose global index is
-    // their group index mod kG; within a group, warp w owns TMEM lane
-    // quadrant w % 4 (the lanes its tcgen05.st may reach) and kG adjacent
-    // 16-column blocks b0 .. b0 + kG - 1 of each of its slices, for every
-    // subtile (two groups: blocks 0-1 or 2-3; four groups: all four).
+    // Two groups of 8 warps take the K slices of alternate global index;
+    // within a group, warp w owns TMEM lane quadrant w % 4 (the lanes its
+    // tcgen05.st may reach) and two adjacent 16-column blocks b0, b0 + 1 of
+    // each of its slices, for every subtile.
     constexpr uint32_t esz = sizeof(T);
-    constexpr int kLanesB = 4 / kG;            // warps per quadrant within a group
     const int xw = warp - kWarpXf0;
     const int quad = warp & 3;                 // TMEM lanes 32*quad..+31
-    const int grp = xw / (4 * kLanesB);        // global slices of this residue mod kG
-    const int b0 = ((xw >> 2) % kLanesB) * kG; // first of the warp's kG blocks
+    const int grp = xw >> 3;                   // global slices of this parity
+    const int b0 = ((xw >> 2) & 1) * 2;        // first of the warp's two blocks
     const int row = quad * 32 + lane;          // output position within a subtile
     const int th = row / p.TW, tw = row % p.TW;
     const uint32_t halo_base = base + p.off_halo;
@@ -934,23 +928,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       int cs0 = c0 - q0 * p.c_slot;
       RingPos h0 = ring_pos(gs_base + static_cast<uint32_t>(q0), ring);
       int released = 0;  // halo slots of this tile this warp has handed back
-      for (; s < p.ks; s += kG, gslice += kG) {
+      for (; s < p.ks; s += 2, gslice += 2, as.next(static_cast<uint32_t>(p.sa)), as.next(static_cast<uint32_t>(p.sa))) {
         const uint32_t ea = as.e;
         if (gslice >= static_cast<uint32_t>(p.sa) &&
             !wait_or_abort(bar_a_empty + 8u * ea, as.ph ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t a_slice = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
-                                 ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
-        // the warp's blocks in pairs jb, jb + 1: (kA, phiA, csA, qA, hA) is block jb
-        int kA = k0, phiA = phi, csA = cs0, qA = q0;
-        RingPos hA = h0;
-#pragma unroll 1
-        for (int jb = 0; jb < kG; jb += 2) {
-        // block jb + 1 starts 16 columns on
-        int phi1 = phiA + p.dk16_phi, cs1 = csA + p.dk16_c, q1 = qA;
-        RingPos h1 = hA;
+        // block b0 + 1 starts 16 columns on
+        int phi1 = phi + p.dk16_phi, cs1 = cs0 + p.dk16_c, q1 = q0;
+        RingPos h1 = h0;
         if (phi1 >= g.taps) {
           phi1 -= g.taps;
           ++cs1;
@@ -960,42 +947,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++q1;
           h1.next(ring);
         }
-        const int nv0 = g.K - kA, nv1 = nv0 - 16;
-        const int split0 = g.taps - phiA, split1 = g.taps - phi1;  // columns j >= split are in the next channel
+        const int nv0 = g.K - k0, nv1 = nv0 - 16;
+        const int split0 = g.taps - phi, split1 = g.taps - phi1;  // columns j >= split are in the next channel
         // the block's second channel opens the next slot (never with slot-aligned blocks)
-        const bool cross0 = !p.slot_aligned && split0 < min(16, nv0) && csA + 1 == p.c_slot;
+        const bool cross0 = !p.slot_aligned && split0 < min(16, nv0) && cs0 + 1 == p.c_slot;
         const bool cross1 = !p.slot_aligned && split1 < min(16, nv1) && cs1 + 1 == p.c_slot;
-        // halo slots the two blocks read: qA .. q_last
+        // halo slots the two blocks read: q0 .. q_last
         if (nv0 > 0) {
-          const int q_last = nv1 > 0 ? q1 + (cross1 ? 1 : 0) : qA + (cross0 ? 1 : 0);
-          RingPos hw = hA;
-          for (int q = qA; ok && q <= q_last; ++q, hw.next(ring))
+          const int q_last = nv1 > 0 ? q1 + (cross1 ? 1 : 0) : q0 + (cross0 ? 1 : 0);
+          RingPos hw = h0;
+          for (int q = q0; ok && q <= q_last; ++q, hw.next(ring))
             ok = wait_or_abort(bar_halo_full + 8u * hw.e, hw.ph, p.err, kSiteHaloFull, abort_flag);
         }
         if (!ok) break;
         tc_fence_after();
-        const uint32_t a_col = a_slice + 8u * static_cast<uint32_t>(jb);
+        const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
+                               ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
         const bool quant = p.quant != 0;
         bool pair_done = false;
         if constexpr (!kPairs && sizeof(T) == 2) {
           // single subtile, both blocks full and within their slots: one interleaved pass
           if (nv0 >= 32 && !cross0 && !cross1) {
-            const uint32_t org0 = halo_base + hA.e * p.slot_bytes + static_cast<uint32_t>(csA * cb) + thr0;
+            const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0;
             const uint32_t org1 = halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb) + thr0;
             uint32_t pa[8], pb[8];
             if constexpr (kDWB > 0) {
               uint32_t ra[6], rb[6];
-              row_bases(org0, phase_tab + static_cast<uint32_t>(phiA * 64), 6, 0, ra);
+              row_bases(org0, phase_tab + static_cast<uint32_t>(phi * 64), 6, 0, ra);
               row_bases(org1, phase_tab + static_cast<uint32_t>(phi1 * 64), 6, 0, rb);
               // the second block starts 16 columns on, one column further in the row pattern
-              switch (phiA % 3) {
+              switch (phi % 3) {
                 case 0: gather_rows<0, kDWB>(ra, pa); gather_rows<1, kDWB>(rb, pb); break;
                 case 1: gather_rows<1, kDWB>(ra, pa); gather_rows<2, kDWB>(rb, pb); break;
                 default: gather_rows<2, kDWB>(ra, pa); gather_rows<0, kDWB>(rb, pb); break;
               }
             } else {
               int off[16];
-              load_taps(phase_tab + static_cast<uint32_t>(phiA * 64), off);
+              load_taps(phase_tab + static_cast<uint32_t>(phi * 64), off);
               gather_taps<T>(org0, off, 16, pa);
               load_taps(phase_tab + static_cast<uint32_t>(phi1 * 64), off);
               gather_taps<T>(org1, off, 16, pb);
@@ -1017,8 +1005,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < p.n_mt; ++i) tmem_st8(colb + static_cast<uint32_t>(i * 32), z);
             continue;
           }
-          const int phb = bb ? phi1 : phiA, csb = bb ? cs1 : csA, splitb = bb ? split1 : split0;
-          const RingPos hb = bb ? h1 : hA;
+          const int phb = bb ? phi1 : phi, csb = bb ? cs1 : cs0, splitb = bb ? split1 : split0;
+          const RingPos hb = bb ? h1 : h0;
           const uint32_t org = halo_base + hb.e * p.slot_bytes + static_cast<uint32_t>(csb * cb);
           const uint32_t prow = phase_tab + static_cast<uint32_t>(phb * 64);
           // the block's second channel opens the next ring slot: its columns move by adj
@@ -1033,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kDWB > 0) {
             if (nv >= 16) {
               // rows of three taps: the rows of the next channel start at
-              // row (taps - phb + phb % 3) / 3 of the block
+              // row (taps - phi + phi % 3) / 3 of the block
               const int p3 = phb % 3;
               uint32_t rb0[6];
               row_bases(org + thr0, prow, crossb ? (g.taps - phb + p3) / 3 : 6, adj, rb0);
@@ -1099,32 +1087,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
           }
         }
-        // the next pair starts 16 columns after block jb + 1
-        if (jb + 2 < kG) {
-          kA += 32;
-          phiA = phi1 + p.dk16_phi;
-          csA = cs1 + p.dk16_c;
-          qA = q1;
-          hA = h1;
-          if (phiA >= g.taps) {
-            phiA -= g.taps;
-            ++csA;
-          }
-          while (csA >= p.c_slot) {
-            csA -= p.c_slot;
-            ++qA;
-            hA.next(ring);
-          }
-        }
-        }  // pairs of blocks
-        if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        // this warp's next slice is kG on: its blocks move kG * 64 columns
-        k0 += kG * kBlockK;
-        phi += p.dks_phi;
-        int dc = p.dks_c;
+        // this warp's next slice is two on: its blocks move 128 columns
+        k0 += 2 * kBlockK;
+        phi += p.dk2_phi;
+        int dc = p.dk2_c;
         if (phi >= g.taps) {
           phi -= g.taps;
           ++dc;
@@ -1145,7 +1114,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // slot's fill first, or the hand-back could land in the previous
           // use's phase.  Otherwise the stage coupling keeps every warp
           // within a ring lap.
-          const int keep = (s + kG < p.ks) ? min(q0, p.q_slots) : p.q_slots;
+          const int keep = (s + 2 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
           for (; ok && released < keep; ++released, hr.next(ring)) {
             if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
             mbar_arrive(bar_halo_empty + 8u * hr.e);
@@ -1155,7 +1124,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
         }
-        for (int j = 0; j < kG; ++j) as.next(static_cast<uint32_t>(p.sa));
       }
       if (!ok) break;
       // Hand back the tile's remaining slots.  With fewer K slices than A
@@ -1181,28 +1149,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, bool kPairs, int kDWB, int kG>
+template <typename T, bool kPairs, int kDWB>
 cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid, size_t smem,
                              cudaStream_t s) {
-  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB, kG>;
+  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
   return cudaGetLastError();
-}
-
-template <typename T, int kDWB, int kG>
-cudaError_t launch_tmem_pairs(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
-                              size_t smem, cudaStream_t s) {
-  return p.n_mt >= 2 ? launch_tmem_inst<T, true, kDWB, kG>(p, tx, tw, grid, smem, s)
-                     : launch_tmem_inst<T, false, kDWB, kG>(p, tx, tw, grid, smem, s);
-}
-
-template <typename T, int kDWB>
-cudaError_t launch_tmem_groups(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
-                               size_t smem, cudaStream_t s) {
-  return p.groups == 4 ? launch_tmem_pairs<T, kDWB, 4>(p, tx, tw, grid, smem, s)
-                       : launch_tmem_pairs<T, kDWB, 2>(p, tx, tw, grid, smem, s);
 }
 
 // Row gather for 16-bit inputs and kernels three taps wide with W dilation 1
@@ -1211,11 +1165,17 @@ template <typename T>
 cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                               size_t smem, cudaStream_t s) {
   const int dwb = row_gather_step(p.g, sizeof(T));
+  const bool pairs = p.n_mt >= 2;
   if constexpr (sizeof(T) == 2) {
-    if (dwb == 2) return launch_tmem_groups<T, 2>(p, tx, tw, grid, smem, s);
-    if (dwb == 4) return launch_tmem_groups<T, 4>(p, tx, tw, grid, smem, s);
+    if (dwb == 2)
+      return pairs ? launch_tmem_inst<T, true, 2>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 2>(p, tx, tw, grid, smem, s);
+    if (dwb == 4)
+      return pairs ? launch_tmem_inst<T, true, 4>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 4>(p, tx, tw, grid, smem, s);
   }
-  return launch_tmem_groups<T, 0>(p, tx, tw, grid, smem, s);
+  return pairs ? launch_tmem_inst<T, true, 0>(p, tx, tw, grid, smem, s)
+               : launch_tmem_inst<T, false, 0>(p, tx, tw, grid, smem, s);
 }
 
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -1273,7 +1233,7 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   if (bTW == 0) return false;
   p.TW = bTW; p.TH = 128 / bTW; p.n_mt = bMT;
   p.a_col0 = a_col0_of(bMT);
-  p.sa = std::min(kMaxStages, stages_of(bMT));
+  p.sa = std::min(4, stages_of(bMT));
   p.n_owb = ceil_div(g.OW, p.TW);
   p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
   p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;
@@ -1285,6 +1245,8 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
   p.ks = ceil_div(g.K, kBlockK);
   p.num_tiles = static_cast<int64_t>(g.N) * g.OD * p.n_ohb * p.n_owb * n_ntiles;
   p.b_stage_bytes = static_cast<uint32_t>(n_tile) * 128u;
+  p.dk2_c = 2 * kBlockK / g.taps;
+  p.dk2_phi = 2 * kBlockK - p.dk2_c * g.taps;
   p.dk16_c = 16 / g.taps;
   p.dk16_phi = 16 - p.dk16_c * g.taps;
   // Fewer than 16 taps: a block spans several channels, so slots hold a
@@ -1318,7 +1280,7 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
     p.slot_tx = static_cast<uint32_t>(p.c_slot) * p.chan_bytes;
     p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
     // fewer A stages shrink the halo window the ring must cover
-    const int sa_max = std::min(kMaxStages, stages_of(bMT));
+    const int sa_max = std::min(4, stages_of(bMT));
     for (int a = sa_max; a >= 2; --a) {
       int span = 1;
       for (int s0 = 0; s0 < p.ks; ++s0) {
@@ -1338,11 +1300,6 @@ static bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem)
             total += extra * (static_cast<int>(p.slot_bytes) + 16);
           }
           p.sa = a; p.sb = b; p.ring = r;
-          // four transform groups need a fifth A stage, so that a group's
-          // next slice never waits for the MMA to consume its previous one
-          p.groups = a >= 5 ? 4 : 2;
-          p.dks_c = p.groups * kBlockK / g.taps;
-          p.dks_phi = p.groups * kBlockK - p.dks_c * g.taps;
           p.off_dq = 0;
           p.off_b = kDqTableBytes;  // a multiple of 1024, as the swizzled weight stages need
           p.off_halo = p.off_b + b * p.b_stage_bytes;
@@ -1364,7 +1321,7 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   TmemParams p{};
   size_t smem = 0;
   const bool ok = plan_tmem(g, dtype, p, smem);
-  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, p.groups, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
+  const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));

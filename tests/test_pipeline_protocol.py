@@ -96,7 +96,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
             released = 0
             for s in range(k0, k1):
                 ea, eb = ga % sa, gb % sb
-                yield ("wait", bar("a_full", ea, 16 // G if kernel == "tmem" else wpg), ga // sa)
+                yield ("wait", bar("a_full", ea, 8 if kernel == "tmem" else wpg), ga // sa)
                 keep = slot_lo(s + 1) if s + 1 < ks else q_slots
                 while not xf_release and released < keep:
                     yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
@@ -167,12 +167,10 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
             gs_base += q_slots
 
     def transform_tmem(w):
-        # tensor-memory kernel: G groups of 16 / G warps; group grp takes the
-        # global slices whose index is grp mod G, warp w blocks b0 .. b0 + G - 1
-        # of each; it waits for the halo slots those read and hands back the
-        # slots below its next slice's first block
-        lanes_b = 4 // G
-        grp, b0 = w // (4 * lanes_b), ((w >> 2) % lanes_b) * G
+        # tensor-memory kernel: group w >> 3 takes the global slices of its
+        # parity; warp w handles blocks b0, b0 + 1 of each, waits for the halo
+        # slots those read and hands back the slots below its next pair
+        grp, b0 = w >> 3, ((w >> 2) & 1) * 2
         gs_base = ga = 0
         gslice = grp
         hr = 0  # next global slot to hand back
@@ -184,16 +182,14 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                 ea, ua = gslice % sa, gslice // sa
                 if gslice >= sa:
                     yield ("wait", bar("a_empty", ea, 1), ua - 1)
-                aligned = (c_slot * taps) % 16 == 0   # no block straddles two slots
-                for jb in range(0, G, 2):             # the warp's blocks in pairs
-                    k0 = 64 * s + 16 * (b0 + jb)
-                    if k0 >= K:
-                        continue
+                k0 = 64 * s + 16 * b0
+                if k0 < K:
                     c0, phi = divmod(k0, taps)
                     q0, cs0 = divmod(c0, c_slot)
                     c1, phi1 = divmod(k0 + 16, taps)
                     q1, cs1 = divmod(c1, c_slot)
                     nv0, nv1 = K - k0, K - k0 - 16
+                    aligned = (c_slot * taps) % 16 == 0   # no block straddles two slots
                     cross0 = not aligned and (taps - phi) < min(16, nv0) and cs0 + 1 == c_slot
                     cross1 = not aligned and (taps - phi1) < min(16, nv1) and cs1 + 1 == c_slot
                     q_last = q1 + int(cross1) if nv1 > 0 else q0 + int(cross0)
@@ -201,9 +197,9 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                         assert q_lo <= q < q_lo + n_q, "a block reads a slot outside its unit"
                         g = gs_base + q - q_lo
                         yield ("wait", bar("halo_full", g % ring, 1), g // ring)
-                yield ("arrive", bar("a_full", ea, 16 // G))
-                if s + G < k1u:
-                    keep = min(((64 * (s + G) + 16 * b0) // taps) // c_slot - q_lo, n_q)
+                yield ("arrive", bar("a_full", ea, 8))
+                if s + 2 < k1u:
+                    keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot - q_lo, n_q)
                 else:
                     keep = n_q
                 while released < keep:
@@ -215,8 +211,8 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                     yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                     released += 1
                     hr += 1
-                s += G
-                gslice += G
+                s += 2
+                gslice += 2
             while released < n_q:
                 # with ks < sa a slot handed back at the end of a tile waits
                 # for its fill first: a warp with no slice in the tile would
@@ -342,10 +338,7 @@ def test_sim_detects_aliasing_when_stages_fewer_than_groups():
 
 
 def _check_tmem_invariants(p, taps):
-    assert p["tmem_cols"] == 512
-    # four groups only with a fifth A stage (a group's next slice never waits
-    # for the MMA to consume its previous one)
-    assert p["groups"] == (4 if p["sa"] >= 5 else 2)
+    assert p["groups"] == 2 and p["tmem_cols"] == 512
     if taps < 16:
         # a block spans several channels: slots must hold whole blocks
         assert (p["c_slot"] * taps) % 16 == 0
