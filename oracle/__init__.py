@@ -78,6 +78,10 @@ def _load():
             lib.oracle_round_to_dtype_bits.argtypes = [vp, i64, ctypes.c_int, vp]
             lib.oracle_out_dim.restype = i64
             lib.oracle_out_dim.argtypes = [i64] * 6
+            lib.oracle_conv3d_ex.restype = ctypes.c_int
+            lib.oracle_conv3d_ex.argtypes = [vp, i64, i64, i64, i64, i64, vp, i64, i64, i64, i64, vp,
+                                             i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int, f32, f32,
+                                             vp, i64, ctypes.c_int, vp]
             lib.oracle_conv3d.restype = ctypes.c_int
             lib.oracle_conv3d.argtypes = ([vp, i64, i64, i64, i64, i64, vp, i64, i64, i64, i64, vp,
                                            i32p, i32p, i32p, i32p, ctypes.c_int, f32, vp, i64,
@@ -232,10 +236,18 @@ def out_dims(in_dhw, k_dhw, stride, pad_lo, pad_hi, dil):
                                         int(pad_hi[i]), int(dil[i]))) for i in range(3))
 
 
+QUANT_FORMATS = {"nvfp4": 1, "mxfp4": 2}
+
+
 def conv3d(x, w, bias=None, stride=(1, 1, 1), pad_lo=(0, 0, 0), pad_hi=None, dil=(1, 1, 1),
-           quant_act: bool = False, act_amax: float = 0.0, m_list=None, nthreads: int = 0) -> np.ndarray:
+           quant_act: bool = False, act_amax: float = 0.0, m_list=None, nthreads: int = 0,
+           quant_format: str = "nvfp4", block_size: int = 16, dst_max: float = 0.0) -> np.ndarray:
     """Reference convolution in binary64 over BF16 (and, with quant_act,
-    NVFP4 fake-quantised) operands.
+    fake-quantised) operands.  quant_format "nvfp4": blocks of block_size
+    (16, 32, 64, 128, 256) consecutive K elements of each A row with E4M3
+    scales and the global scale act_amax / (6*448) (the article, sec. 6 and
+    7.1); "mxfp4": groups of 32 with power-of-two scales and dst_max (the
+    CANN aclnnFlatQuantV2 page).  A short last block acts as zero-filled.
 
     x: [N, C, D, H, W] values (any float dtype, taken exactly as float32);
     w: [Cout, C, KD, KH, KW]; bias: [Cout] or None.
@@ -264,11 +276,12 @@ def conv3d(x, w, bias=None, stride=(1, 1, 1), pad_lo=(0, 0, 0), pad_hi=None, dil
         ml = np.ascontiguousarray(np.asarray(m_list, dtype=np.int64))
         n_m = ml.size
     y = np.empty((n_m, Cout), dtype=np.float64)
-    rc = lib.oracle_conv3d(_ptr(x), N, C, D, H, W, _ptr(w), Cout, KD, KH, KW,
-                           None if b is None else _ptr(b),
-                           arr(stride), arr(pad_lo), arr(pad_hi), arr(dil), int(bool(quant_act)),
-                           float(np.float32(act_amax)), None if ml is None else _ptr(ml), n_m,
-                           int(nthreads), _ptr(y))
+    qfmt = QUANT_FORMATS[quant_format] if quant_act else 0
+    rc = lib.oracle_conv3d_ex(_ptr(x), N, C, D, H, W, _ptr(w), Cout, KD, KH, KW,
+                              None if b is None else _ptr(b),
+                              arr(stride), arr(pad_lo), arr(pad_hi), arr(dil), qfmt, int(block_size),
+                              float(np.float32(act_amax)), float(np.float32(dst_max)),
+                              None if ml is None else _ptr(ml), n_m, int(nthreads), _ptr(y))
     if rc != 0:
         raise ValueError("oracle_conv3d: invalid arguments")
     if m_list is None:

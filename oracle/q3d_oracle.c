@@ -339,6 +339,7 @@ typedef struct {
     int64_t sd, sh, sw, pd, ph, pw, dd, dh, dw;   /* stride, front pad, dilation */
     int64_t OD, OH, OW;
     int quant; float amax;
+    int qfmt; int qblock; float dst_max;   /* quantiser: 1 NVFP4 blocks of qblock, 2 MXFP4 groups of 32 */
     const double* wb;        /* bf16(w) as binary64, [Cout][K] */
     /* work list */
     const int64_t* m_list; int64_t n_m;
@@ -379,10 +380,19 @@ static void* conv_worker(void* arg)
     for (int64_t i = j->lo; i < j->hi; ++i) {
         int64_t m = j->m_list[i];
         im2col_row(j, m, row);
-        if (j->quant) {
-            /* blocks of 16 consecutive K elements of this row (sec. 6.3) */
-            for (int64_t b = 0; b < K; b += 16) {
-                int nb = (int)((K - b) < 16 ? (K - b) : 16);
+        if (j->quant && j->qfmt == 2) {
+            /* MXFP4 groups of 32 consecutive K elements of this row; a short
+             * last group as if zero-filled (zeros leave its maximum alone) */
+            for (int64_t b = 0; b < K; b += 32) {
+                int nb = (int)((K - b) < 32 ? (K - b) : 32);
+                oracle_mxfp4_block(row + b, nb, j->dst_max, fq + b, NULL);
+            }
+        } else if (j->quant) {
+            /* NVFP4 blocks of qblock (16 in the article's kernel, sec. 6.3;
+             * 32..256 its call's other block sizes, sec. 7.1) consecutive K
+             * elements of this row; a short last block as if zero-filled */
+            for (int64_t b = 0; b < K; b += j->qblock) {
+                int nb = (int)((K - b) < j->qblock ? (K - b) : j->qblock);
                 oracle_fq_block(row + b, nb, j->amax, fq + b);
             }
         } else {
@@ -419,13 +429,16 @@ int64_t oracle_out_dim(int64_t in, int64_t k, int64_t s, int64_t plo, int64_t ph
  * stride/pad_lo/pad_hi/dil are (d, h, w).  Returns 0, or -1 on bad
  * arguments.  nthreads <= 0 uses every online core.
  */
-int oracle_conv3d(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
-                  const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
-                  const float* bias,
-                  const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
-                  const int32_t* dil, int quant_act, float act_amax,
-                  const int64_t* m_list, int64_t n_m, int nthreads, double* y)
+int oracle_conv3d_ex(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
+                     const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
+                     const float* bias,
+                     const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
+                     const int32_t* dil, int qfmt, int qblock, float act_amax, float dst_max,
+                     const int64_t* m_list, int64_t n_m, int nthreads, double* y)
 {
+    if (qfmt < 0 || qfmt > 2) return -1;
+    if (qfmt == 1 && qblock != 16 && qblock != 32 && qblock != 64 && qblock != 128 && qblock != 256) return -1;
+    if (qfmt == 2 && (qblock != 32 || !(dst_max == 0.0f || (dst_max >= 6.0f && dst_max <= 12.0f)))) return -1;
     for (int i = 0; i < 3; ++i)
         if (stride[i] < 1 || dil[i] < 1 || pad_lo[i] < 0 || pad_hi[i] < 0) return -1;
     conv_job base;
@@ -439,7 +452,8 @@ int oracle_conv3d(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, in
     base.OD = oracle_out_dim(D, KD, stride[0], pad_lo[0], pad_hi[0], dil[0]);
     base.OH = oracle_out_dim(H, KH, stride[1], pad_lo[1], pad_hi[1], dil[1]);
     base.OW = oracle_out_dim(W, KW, stride[2], pad_lo[2], pad_hi[2], dil[2]);
-    base.quant = quant_act; base.amax = act_amax;
+    base.quant = qfmt != 0; base.amax = act_amax;
+    base.qfmt = qfmt; base.qblock = qblock; base.dst_max = dst_max;
     int64_t M = N * base.OD * base.OH * base.OW;
     int64_t K = C * KD * KH * KW;
     if (M <= 0 || K <= 0 || Cout <= 0) return -1;
@@ -471,4 +485,16 @@ int oracle_conv3d(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, in
     for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
     free(th); free(jobs); free(wb); free(all);
     return 0;
+}
+
+/* The article's convolution: NVFP4 blocks of 16 when quant_act is set. */
+int oracle_conv3d(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
+                  const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
+                  const float* bias,
+                  const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
+                  const int32_t* dil, int quant_act, float act_amax,
+                  const int64_t* m_list, int64_t n_m, int nthreads, double* y)
+{
+    return oracle_conv3d_ex(x, N, C, D, H, W, w, Cout, KD, KH, KW, bias, stride, pad_lo, pad_hi, dil,
+                            quant_act ? 1 : 0, 16, act_amax, 0.0f, m_list, n_m, nthreads, y);
 }

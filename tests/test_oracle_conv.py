@@ -212,3 +212,54 @@ def test_rejects_bad_arguments():
         oracle.conv3d(x, w, None, (0, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1))
     with pytest.raises(ValueError):
         oracle.conv3d(x, w, None, (1, 1, 1), (-1, 1, 1), (1, 1, 1), (1, 1, 1))
+
+
+# the fused quantiser's other formats: NVFP4 with the article's other block
+# sizes (sec. 7.1) and MXFP4 (the CANN aclnnFlatQuantV2 page); a short last
+# block of a row acts as zero-filled
+FORMATS = [("nvfp4", 32, 0.0), ("nvfp4", 64, 0.0), ("nvfp4", 128, 0.0), ("nvfp4", 256, 0.0),
+           ("mxfp4", 32, 0.0), ("mxfp4", 32, 6.0)]
+
+
+@pytest.mark.parametrize("fmt", FORMATS, ids=[f"{f}{b}_{d:g}" for f, b, d in FORMATS])
+@pytest.mark.parametrize("case", CASES[:5])
+def test_block_formats_match_im2col_with_standalone_quantisers(case, fmt):
+    """conv3d with an explicit format equals numpy im2col, each row quantised
+    by the standalone (separately pinned) block quantiser in blocks of the
+    format's size, and an fp64 matmul over BF16 operands."""
+    qf, bs, dst = fmt
+    xs, cout, k, s, plo, phi, d = case
+    g = torch.Generator().manual_seed(17)
+    x = (torch.randn(xs, generator=g) * 3).numpy()
+    w = torch.randn((cout, xs[1]) + k, generator=g).numpy()
+    amax = float(np.abs(x).max())
+    A, (N, OD, OH, OW) = _im2col_numpy(x, k, s, plo, phi, d)
+    Kdim = A.shape[1]
+    Aq = np.empty_like(A, dtype=np.float32)
+    for r in range(A.shape[0]):
+        for j in range(0, Kdim, bs):
+            blk = np.zeros(bs, np.float32)
+            n = min(bs, Kdim - j)
+            blk[:n] = A[r, j:j + n]
+            q = (oracle.fp4_fake_quant_bs(blk, amax, bs) if qf == "nvfp4" else oracle.mxfp4_fake_quant(blk, dst)[0])
+            Aq[r, j:j + n] = q[:n]
+    Am = oracle.bf16_round(Aq).astype(np.float64)
+    Wm = oracle.bf16_round(w.reshape(cout, -1)).astype(np.float64)
+    ref = (Am @ Wm.T).reshape(N, OD, OH, OW, cout).transpose(0, 4, 1, 2, 3)
+    got = oracle.conv3d(x, w, None, s, plo, phi, d, quant_act=True, act_amax=amax, quant_format=qf, block_size=bs,
+                        dst_max=dst)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-11)
+    # the block size matters: 16 and the format's size disagree somewhere
+    # (when a row holds more than one block of 16)
+    if qf == "nvfp4" and Kdim > 16:
+        g16 = oracle.conv3d(x, w, None, s, plo, phi, d, quant_act=True, act_amax=amax)
+        assert not np.array_equal(g16, got)
+
+
+def test_block_format_arguments_are_checked():
+    x = np.ones((1, 2, 3, 3, 3), np.float32)
+    w = np.ones((2, 2, 3, 3, 3), np.float32)
+    for kw in (dict(block_size=48), dict(quant_format="mxfp4", block_size=16), dict(quant_format="mxfp4", block_size=32,
+                                                                                    dst_max=3.0)):
+        with pytest.raises(ValueError):
+            oracle.conv3d(x, w, None, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1), quant_act=True, act_amax=1.0, **kw)
