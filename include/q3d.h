@@ -129,6 +129,40 @@ Q3D_API q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tens
                                      const int32_t dil[3], int32_t quant_act, q3d_tensor* out,
                                      q3d_stream_t stream);
 
+/* Activation quantiser formats of conv3d_implicit_gemm_ex. */
+typedef enum {
+  Q3D_QUANT_NONE = 0,
+  Q3D_QUANT_NVFP4 = 1,   /* E2M1 values, E4M3 block scales, global scale act_amax / (6*448) */
+  Q3D_QUANT_MXFP4 = 2    /* E2M1 values, power-of-two E8M0 group scales */
+} q3d_quant_format;
+
+/*
+ * conv3d_implicit_gemm_ex -- conv3d_implicit_gemm_pad2 with the activation
+ * quantiser chosen explicitly (same x, w, bias, stride, pad_lo, pad_hi,
+ * dil, out and stream).  Each row of the implicit im2col matrix A is split
+ * into blocks of block_size consecutive K columns (K ordered (c, kd, kh,
+ * kw); a short last block acts as zero-filled), every element is rounded to
+ * E2M1 with its block's scale and dequantised, then rounded to BF16:
+ *   quant_format Q3D_QUANT_NONE   no quantisation (block_size ignored).
+ *   quant_format Q3D_QUANT_NVFP4  the article's quantiser (sec. 6.1-6.3)
+ *       with its call's fp4_block_size (sec. 7.1): block_size 16, 32, 64,
+ *       128 or 256; act_amax required as for conv3d_implicit_gemm.
+ *   quant_format Q3D_QUANT_MXFP4  the CANN aclnnFlatQuantV2 page's per-group
+ *       route: block_size 32, scale 2^E with E = floor(log2(block max)) - 2
+ *       (dst_type_max 0) or the exponent of block max / dst_type_max rounded
+ *       up (dst_type_max in [6, 12]), as in mxfp4_quantize; act_amax unused.
+ * NVFP4 with block_size 16 runs the same kernels as
+ * conv3d_implicit_gemm_pad2 (bit-identical results); the other settings run
+ * the general kernel, which takes each block's maximum in a separate gather
+ * pass.  Q3D_ERR_INVALID_ARG for another format, block size or dst_type_max,
+ * before anything is enqueued.
+ */
+Q3D_API q3d_status conv3d_implicit_gemm_ex(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                           const float* act_amax, const int32_t stride[3],
+                                           const int32_t pad_lo[3], const int32_t pad_hi[3],
+                                           const int32_t dil[3], int32_t quant_format, int32_t block_size,
+                                           float dst_type_max, q3d_tensor* out, q3d_stream_t stream);
+
 /*
  * conv3d_implicit_gemm_noalloc -- as conv3d_implicit_gemm_pad2 (same
  * arguments, same kernels, same result), for callers that may not allocate

@@ -23,7 +23,8 @@ STATUS = {0: "Q3D_OK", 1: "Q3D_ERR_NULLPTR", 2: "Q3D_ERR_INVALID_ARG", 3: "Q3D_E
           4: "Q3D_ERR_ARCH", 5: "Q3D_ERR_CUDA", 6: "Q3D_ERR_DEVICE_TIMEOUT", 7: "Q3D_ERR_UNSUPPORTED_SHAPE"}
 
 # names of the exported C entry points (checked against include/q3d.h by the tests)
-EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_noalloc",
+EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit_gemm_ex",
+           "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "fp4_fake_quant_bs", "mxfp4_quantize", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
            "q3d_selftest_ratio", "q3d_plan_conv", "q3d_plan_conv_tmem")
@@ -62,6 +63,9 @@ def load_library(path: Optional[str] = None):
         lib.conv3d_implicit_gemm.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.conv3d_implicit_gemm_pad2.restype = ctypes.c_int
         lib.conv3d_implicit_gemm_pad2.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
+        lib.conv3d_implicit_gemm_ex.restype = ctypes.c_int
+        lib.conv3d_implicit_gemm_ex.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32,
+                                                ctypes.c_int32, ctypes.c_float, T, vp]
         lib.conv3d_implicit_gemm_noalloc.restype = ctypes.c_int
         lib.conv3d_implicit_gemm_noalloc.argtypes = [T, T, T, vp, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32, T, vp]
         lib.fp4_fake_quant.restype = ctypes.c_int
@@ -194,6 +198,31 @@ def conv3d_implicit_gemm(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.
         st = lib.conv3d_implicit_gemm_pad2(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo),
                                            arr(hi), arr(_triple(dilation)), int(bool(quant_act)), _ref(os_),
                                            _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
+QUANT_FORMATS = {"none": 0, "nvfp4": 1, "mxfp4": 2}
+
+
+def conv3d_implicit_gemm_ex(x: torch.Tensor, w: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                            stride=1, padding=0, dilation=1, act_amax: Optional[torch.Tensor] = None,
+                            quant_format: str = "nvfp4", block_size: int = 16, dst_type_max: float = 0.0,
+                            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """conv3d_implicit_gemm with the activation quantiser chosen explicitly:
+    quant_format "none", "nvfp4" (block_size 16..256, act_amax required) or
+    "mxfp4" (block_size 32, power-of-two scales, dst_type_max 0 or 6..12)."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    if out is None:
+        out = torch.empty(out_shape(x.shape, w.shape, stride, padding, dilation), dtype=x.dtype, device=x.device)
+    _check_amax(act_amax, x, quant_format == "nvfp4")
+    arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    xs, ws, os_, bs = _tensor(x), _tensor(w), _tensor(out), _tensor(bias)
+    amax_ptr = act_amax.data_ptr() if (quant_format == "nvfp4" and act_amax is not None) else None
+    st = lib.conv3d_implicit_gemm_ex(_ref(xs), _ref(ws), _ref(bs), amax_ptr, arr(_triple(stride)), arr(lo), arr(hi),
+                                     arr(_triple(dilation)), QUANT_FORMATS[quant_format], int(block_size),
+                                     float(dst_type_max), _ref(os_), _stream_handle(stream))
     _check(lib, st)
     return out
 

@@ -15,7 +15,10 @@
 //     on the fly, no lookup tables), fake-quantises them in blocks of 16
 //     when requested (sec. 6.3; the block is a register reduction because
 //     the thread owns the whole row segment), rounds to BF16 and writes the
-//     swizzled layout the tensor core reads;
+//     swizzled layout the tensor core reads; the quantiser's other formats
+//     (NVFP4 blocks of 32..256, MXFP4 groups of 32) take each block's
+//     maximum in a gather pass over the block's columns before its first
+//     16-column piece;
 //   - one thread issues tcgen05.mma (M=128, N=n_tile, K=16) x 4 per slice
 //     into an FP32 accumulator in tensor memory, two slices in flight;
 //   - the epilogue reads the accumulator with tcgen05.ld, adds the bias in
@@ -46,6 +49,9 @@ struct BasicParams {
   const float* act_amax;
   unsigned int* err;
   int quant;
+  int qfmt;        // 1: NVFP4 blocks of qblock, 2: MXFP4 groups of 32 (when quant)
+  int qblock;
+  float dst_max;   // MXFP4 only
   int n_tile;
   int tmem_cols;
   int num_k_stages;
@@ -104,10 +110,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int id0 = od * g.sd - g.pd, ih0 = oh * g.sh - g.ph, iw0 = ow * g.sw - g.pw;
   const T* xn = static_cast<const T*>(p.x) + static_cast<int64_t>(nb) * g.C * g.D * g.H * g.W;
   Nvfp4Global G{0.0f, 0.0f, 0.0f};
-  if (p.quant) G = nvfp4_global(__ldg(p.act_amax));
+  if (p.quant && p.qfmt == 1) G = nvfp4_global(__ldg(p.act_amax));  // MXFP4 takes no global amax
   const int khw = g.KH * g.KW;
   const uint32_t idesc = umma_idesc_bf16_f32(kBlockM, static_cast<uint32_t>(p.n_tile));
 
+  // A[m, kk] of this row (column kk of the implicit im2col matrix)
+  auto im2col_at = [&](int kk) -> float {
+    const int c = kk / g.taps;
+    int r = kk - c * g.taps;
+    const int kd = r / khw;
+    r -= kd * khw;
+    const int kh = r / g.KW, kw = r - (r / g.KW) * g.KW;
+    const int id = id0 + kd * g.dd, ih = ih0 + kh * g.dh, iw = iw0 + kw * g.dw;
+    if (static_cast<unsigned>(id) < static_cast<unsigned>(g.D) && static_cast<unsigned>(ih) < static_cast<unsigned>(g.H) &&
+        static_cast<unsigned>(iw) < static_cast<unsigned>(g.W))
+      return DTypeOps<T>::to_f32(xn[((static_cast<int64_t>(c) * g.D + id) * g.H + ih) * g.W + iw]);
+    return 0.0f;
+  };
+  // scale of the current quantisation block of the other formats: NVFP4
+  // (q_a, q_b) = (1/scale, scale), MXFP4 (2^-E, 2^E)
+  float q_a = 1.0f, q_b = 1.0f;
   bool aborted = false;
   bool tma_wait_failed = false;
   int last_tma_stage = -1;
@@ -156,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (p.quant) {
+      if (p.quant && p.qfmt == 1 && p.qblock == 16) {
         float bmax = 0.0f;
 #pragma unroll
         for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(v[j]));
@@ -164,6 +186,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         nvfp4_block_scale(bmax, G, scale, inv);
 #pragma unroll
         for (int i = 0; i < 8; ++i) nvfp4_pair(v[2 * i], v[2 * i + 1], inv, scale, v[2 * i], v[2 * i + 1]);
+      } else if (p.quant) {
+        // a quantisation block of qblock columns (a multiple of 16) starts
+        // here: its |v| maximum over all its columns (a short last block as
+        // if zero-filled) sets the scale its 16-column pieces share
+        const int kb = k0 + blk * 16;
+        if (kb % p.qblock == 0) {
+          float bm = 0.0f;
+          const int ke = min(kb + p.qblock, g.K);
+          for (int kk = kb; kk < ke && row_ok; ++kk) bm = fmaxf(bm, fabsf(im2col_at(kk)));
+          if (p.qfmt == 2) {
+            const int e = mx_scale_exp(bm, p.dst_max);
+            q_a = mx_exp2i(-e);
+            q_b = mx_exp2i(e);
+          } else {
+            nvfp4_block_scale(bm, G, q_b, q_a);
+          }
+        }
+        if (p.qfmt == 2) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx_pair(v[2 * i], v[2 * i + 1], q_a, q_b, v[2 * i], v[2 * i + 1]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) nvfp4_pair(v[2 * i], v[2 * i + 1], q_a, q_b, v[2 * i], v[2 * i + 1]);
+        }
       }
       uint32_t w[8];
 #pragma unroll
@@ -305,7 +351,8 @@ cudaError_t launch_conv3d_basic(const ConvGeom& g, const ConvLaunch& L, cudaStre
   BasicParams p;
   p.g = g;
   p.x = L.x; p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err;
-  p.quant = L.quant; p.n_tile = n_tile; p.tmem_cols = tmem_cols;
+  p.quant = L.quant; p.qfmt = L.qfmt; p.qblock = L.qblock; p.dst_max = L.dst_max;
+  p.n_tile = n_tile; p.tmem_cols = tmem_cols;
   p.num_k_stages = (g.K + kBlockK - 1) / kBlockK;
   size_t smem = 1024 + kStages * kATileBytes + kStages * static_cast<size_t>(n_tile) * 128 + 128;
   // Keep (CTAs per SM) x tmem_cols <= 512 so no CTA ever waits in

@@ -30,31 +30,6 @@ namespace q3d {
 
 namespace {
 
-// 2^k as binary32 for k in [-127, 127] (2^-127 is subnormal).
-__device__ __forceinline__ float exp2i(int k) {
-  return k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23) : __uint_as_float(0x00400000u);
-}
-
-// Unbiased exponent of a binary32 value; zero and subnormals give -127.
-__device__ __forceinline__ int floor_log2_clamped(float a) {
-  const int be = static_cast<int>((__float_as_uint(a) >> 23) & 0xFFu);
-  return be == 0 ? -127 : be - 127;
-}
-
-__device__ __forceinline__ int mx_scale_exp(float amax, float dst_max) {
-  int e;
-  if (dst_max == 0.0f) {
-    e = floor_log2_clamped(amax) - 2;
-  } else {
-    const float s = __fdiv_rn(amax, dst_max);
-    const uint32_t u = __float_as_uint(s);
-    const int be = static_cast<int>((u >> 23) & 0xFFu);
-    e = floor_log2_clamped(s);
-    if (be != 0 && be < 254 && (u & 0x007FFFFFu) != 0) e += 1;
-  }
-  return min(max(e, -127), 127);
-}
-
 template <typename T, bool kVec>
 struct Io16;
 template <typename T>
@@ -140,7 +115,7 @@ __global__ void __launch_bounds__(256) mxfp4_kernel(const T* x, T* y, uint8_t* s
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     const int e = mx_scale_exp(amax, dst_max);
-    const float down = exp2i(-e), up = exp2i(e);
+    const float down = mx_exp2i(-e), up = mx_exp2i(e);
     uint32_t packed[2] = {0u, 0u};
     float o[16];
 #pragma unroll

@@ -265,6 +265,51 @@ const char* q3d_last_error(void) { return g_last_error.c_str(); }
 
 int32_t q3d_version(void) { return 100; }
 
+}  // extern "C"
+
+namespace {
+
+// Weight staging and the kernel chain for a prepared convolution.  The
+// quantiser's formats other than NVFP4 blocks of 16 run in the general kernel.
+q3d_status run_conv(const q3d::ConvGeom& g, q3d::ConvLaunch& L, const q3d_tensor* w, int32_t dtype,
+                    q3d_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t K = g.K, Cout = g.Cout;
+
+  // B operand: BF16 [Cout, ld] with a 16-byte row pitch.  BF16 weights with
+  // K % 8 == 0 and a 16-byte aligned base are used in place; otherwise a
+  // stream-ordered scratch copy is made.
+  void* scratch = nullptr;
+  cudaError_t e;
+  if (dtype == Q3D_BF16 && K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {
+    L.w_bf16 = w->data;
+    L.w_ld = K;
+  } else {
+    const int64_t ld = (K + 7) / 8 * 8;
+    e = L.pool ? cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(Cout * ld * 2), L.pool, s)
+               : cudaMallocAsync(&scratch, static_cast<size_t>(Cout * ld * 2), s);
+    if (e != cudaSuccess) return cuda_fail(e, "stream-ordered allocation (weight staging)");
+    e = q3d::launch_stage_weights(w->data, dtype, (int32_t)Cout, (int32_t)K, ld, scratch, s);
+    if (e != cudaSuccess) { cudaFreeAsync(scratch, s); return cuda_fail(e, "weight staging launch"); }
+    L.w_bf16 = scratch;
+    L.w_ld = ld;
+  }
+
+  const char* why = nullptr;
+  const bool general = L.quant && !(L.qfmt == 1 && L.qblock == 16);
+  e = general ? q3d::launch_conv3d_basic(g, L, s, &why) : launch_conv(g, L, s, &why);
+  if (scratch) cudaFreeAsync(scratch, s);
+  if (e != cudaSuccess) {
+    if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
+    return cuda_fail(e, "conv3d launch");
+  }
+  return Q3D_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
 q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
                                      const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
                                      const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_act,
@@ -274,36 +319,35 @@ q3d_status conv3d_implicit_gemm_pad2(const q3d_tensor* x, const q3d_tensor* w, c
   bool noop = false;
   q3d_status st = prepare_conv(x, w, bias, act_amax, stride, pad_lo, pad_hi, dil, quant_act, out, &g, &L, &noop);
   if (st != Q3D_OK || noop) return st;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t K = g.K, Cout = g.Cout;
+  return run_conv(g, L, w, x->dtype, stream);
+}
 
-  // B operand: BF16 [Cout, ld] with a 16-byte row pitch.  BF16 weights with
-  // K % 8 == 0 and a 16-byte aligned base are used in place; otherwise a
-  // stream-ordered scratch copy is made.
-  void* scratch = nullptr;
-  cudaError_t e;
-  if (x->dtype == Q3D_BF16 && K % 8 == 0 && reinterpret_cast<uintptr_t>(w->data) % 16 == 0) {
-    L.w_bf16 = w->data;
-    L.w_ld = K;
-  } else {
-    const int64_t ld = (K + 7) / 8 * 8;
-    e = L.pool ? cudaMallocFromPoolAsync(&scratch, static_cast<size_t>(Cout * ld * 2), L.pool, s)
-               : cudaMallocAsync(&scratch, static_cast<size_t>(Cout * ld * 2), s);
-    if (e != cudaSuccess) return cuda_fail(e, "stream-ordered allocation (weight staging)");
-    e = q3d::launch_stage_weights(w->data, x->dtype, (int32_t)Cout, (int32_t)K, ld, scratch, s);
-    if (e != cudaSuccess) { cudaFreeAsync(scratch, s); return cuda_fail(e, "weight staging launch"); }
-    L.w_bf16 = scratch;
-    L.w_ld = ld;
+q3d_status conv3d_implicit_gemm_ex(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
+                                   const float* act_amax, const int32_t stride[3], const int32_t pad_lo[3],
+                                   const int32_t pad_hi[3], const int32_t dil[3], int32_t quant_format,
+                                   int32_t block_size, float dst_type_max, q3d_tensor* out, q3d_stream_t stream) {
+  if (quant_format != Q3D_QUANT_NONE && quant_format != Q3D_QUANT_NVFP4 && quant_format != Q3D_QUANT_MXFP4)
+    return fail(Q3D_ERR_INVALID_ARG, "quant_format %d is not NONE, NVFP4 or MXFP4", quant_format);
+  if (quant_format == Q3D_QUANT_NVFP4 && block_size != 16 && block_size != 32 && block_size != 64 &&
+      block_size != 128 && block_size != 256)
+    return fail(Q3D_ERR_INVALID_ARG, "NVFP4 block_size %d is not 16, 32, 64, 128 or 256", block_size);
+  if (quant_format == Q3D_QUANT_MXFP4) {
+    if (block_size != 32) return fail(Q3D_ERR_INVALID_ARG, "MXFP4 block_size %d is not 32", block_size);
+    if (!(dst_type_max == 0.0f || (dst_type_max >= 6.0f && dst_type_max <= 12.0f)))
+      return fail(Q3D_ERR_INVALID_ARG, "dst_type_max must be 0 or in [6, 12]");
   }
-
-  const char* why = nullptr;
-  e = launch_conv(g, L, s, &why);
-  if (scratch) cudaFreeAsync(scratch, s);
-  if (e != cudaSuccess) {
-    if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
-    return cuda_fail(e, "conv3d launch");
-  }
-  return Q3D_OK;
+  q3d::ConvGeom g;
+  q3d::ConvLaunch L;
+  bool noop = false;
+  // NVFP4 needs the global amax; MXFP4 scales come from each group alone
+  q3d_status st = prepare_conv(x, w, bias, quant_format == Q3D_QUANT_NVFP4 ? act_amax : nullptr, stride, pad_lo,
+                               pad_hi, dil, quant_format == Q3D_QUANT_NVFP4 ? 1 : 0, out, &g, &L, &noop);
+  if (st != Q3D_OK || noop) return st;
+  L.quant = quant_format != Q3D_QUANT_NONE ? 1 : 0;
+  L.qfmt = quant_format == Q3D_QUANT_MXFP4 ? 2 : 1;
+  L.qblock = quant_format == Q3D_QUANT_NONE ? 16 : block_size;
+  L.dst_max = dst_type_max;
+  return run_conv(g, L, w, x->dtype, stream);
 }
 
 q3d_status conv3d_implicit_gemm(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,

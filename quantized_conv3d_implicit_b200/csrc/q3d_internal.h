@@ -44,6 +44,9 @@ struct ConvLaunch {
   int64_t w_ld;             // row pitch of w_bf16 in elements
   int dtype;                // 0 f32, 1 f16, 2 bf16
   int quant;
+  int qfmt = 1;             // quantiser when quant: 1 NVFP4 (blocks of qblock), 2 MXFP4 (groups of 32)
+  int qblock = 16;
+  float dst_max = 0.0f;     // MXFP4 only
   unsigned int* err;        // device error word
   int sm_count;
   // stream-ordered pool of the device for the staged BF16 weights (kept

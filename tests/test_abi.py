@@ -204,3 +204,18 @@ def test_mxfp4_validation(lib):
     assert lib.mxfp4_quantize(r(x), 0.0, None, FAKE + 8, None, None) == 2        # scales inside x
     assert lib.mxfp4_quantize(r(x), 0.0, None, FAKE * 4096, FAKE * 4096 + 4, None) == 2   # scales overlap codes
     assert lib.mxfp4_quantize(r(T((0, 64))), 0.0, None, FAKE * 4096, None, None) == 0
+
+
+def test_conv_ex_validation(lib):
+    x, w, out = good()
+    arr = lambda v: (ctypes.c_int32 * 3)(*v)  # noqa: E731
+    r = ctypes.byref
+
+    def ex(fmt, bs, dst, amax=FAKE * 4096):
+        return lib.conv3d_implicit_gemm_ex(r(x), r(w), None, amax, arr((1, 1, 1)), arr((1, 1, 1)), arr((1, 1, 1)),
+                                           arr((1, 1, 1)), fmt, bs, dst, r(out), None)
+    assert ex(3, 16, 0.0) == 2 and b"quant_format" in lib.q3d_last_error()
+    assert ex(1, 48, 0.0) == 2 and b"block_size" in lib.q3d_last_error()
+    assert ex(2, 16, 0.0) == 2
+    assert ex(2, 32, 3.0) == 2 and b"dst_type_max" in lib.q3d_last_error()
+    assert ex(1, 32, 0.0, amax=None) == 1            # NVFP4 needs act_amax

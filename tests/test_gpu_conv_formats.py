@@ -1,0 +1,97 @@
+"""GPU parity of conv3d_implicit_gemm_ex: the fused activation quantiser's
+other formats (NVFP4 with the article's block sizes 32..256, sec. 7.1; MXFP4
+from the CANN aclnnFlatQuantV2 page) against the CPU oracle.
+
+The one-hot-weight readout reproduces the quantised im2col matrix A bit for
+bit (one nonzero product per output), so every element of the quantiser is
+checked exactly; full convolutions are checked with the convolution
+acceptance rule."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_conv3d_implicit_b200 import api, workloads
+from _parity import assert_conv_close, bits, to_np_f32
+
+pytestmark = pytest.mark.gpu
+
+DT = {torch.float32: "float32", torch.float16: "float16", torch.bfloat16: "bfloat16"}
+FORMATS = [("nvfp4", 32, 0.0), ("nvfp4", 64, 0.0), ("nvfp4", 128, 0.0), ("nvfp4", 256, 0.0),
+           ("mxfp4", 32, 0.0), ("mxfp4", 32, 6.0), ("mxfp4", 32, 12.0)]
+FIDS = [f"{f}{b}_{d:g}" for f, b, d in FORMATS]
+
+
+@pytest.mark.parametrize("dtype", list(DT))
+@pytest.mark.parametrize("fmt", FORMATS, ids=FIDS)
+def test_identity_weight_readout_other_formats(cuda_ok, fmt, dtype):
+    qf, bs, dst = fmt
+    # K = 11 * 27 = 297: several blocks of every size and a short last one
+    xs, k = (1, 11, 4, 7, 12), (3, 3, 3)
+    K = 11 * 27
+    g = torch.Generator().manual_seed(21)
+    x = (torch.randn(xs, generator=g) * 3)
+    x[0, 2] *= 40  # blocks with very different maxima
+    x = x.to(dtype)
+    amax = x.float().abs().max().reshape(1)
+    for start in range(0, K, 128):
+        cols = list(range(start, min(K, start + 128)))
+        w = torch.zeros((len(cols), K), dtype=torch.float32)
+        w[torch.arange(len(cols)), torch.tensor(cols)] = 1.0
+        w = w.reshape(len(cols), 11, 3, 3, 3).to(dtype)
+        y = api.conv3d_implicit_gemm_ex(x.cuda(), w.cuda(), None, 1, (2, 0, 1, 1, 1, 1), 1, act_amax=amax.cuda(),
+                                        quant_format=qf, block_size=bs, dst_type_max=dst)
+        assert api.check_device_error() == 0
+        ref = oracle.conv3d(x.float().numpy(), w.float().numpy(), None, (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1),
+                            quant_act=True, act_amax=float(amax.item()), quant_format=qf, block_size=bs,
+                            dst_max=dst)
+        assert np.array_equal(bits(y), oracle.round_to_dtype_bits(ref.astype(np.float32), DT[dtype])), start
+
+
+SHAPES = [
+    ((1, 8, 3, 10, 12), 24, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 1, 1)),   # K = 216
+    ((2, 5, 5, 9, 11), 20, (3, 3, 3), (1, 2, 2), (1, 1, 1), (1, 1, 1), (1, 1, 1)),    # stride, K = 135
+    ((1, 6, 6, 13, 24), 33, (3, 3, 3), (1, 1, 1), (2, 1, 1), (0, 1, 1), (1, 2, 2)),   # dilation, K = 162
+    ((1, 32, 3, 8, 8), 300, (1, 1, 1), (1, 1, 1), (0, 0, 0), (0, 0, 0), (1, 1, 1)),   # pointwise, 2 N tiles
+]
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("fmt", FORMATS, ids=FIDS)
+@pytest.mark.parametrize("case", range(len(SHAPES)))
+def test_conv_other_formats_small_shapes(cuda_ok, case, fmt, dtype):
+    qf, bs, dst = fmt
+    xs, cout, k, s, plo, phi, d = SHAPES[case]
+    inp = workloads.random_conv_inputs(500 + case, xs, cout, k, dtype=dtype, bias=True, device="cuda", scale=2.0)
+    pad6 = (plo[0], phi[0], plo[1], phi[1], plo[2], phi[2])
+    y = api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], inp["bias"], s, pad6, d, act_amax=inp["act_amax"],
+                                    quant_format=qf, block_size=bs, dst_type_max=dst)
+    assert api.check_device_error() == 0
+    ref = oracle.conv3d(to_np_f32(inp["x"]), to_np_f32(inp["w"]), to_np_f32(inp["bias"]), s, plo, phi, d,
+                        quant_act=True, act_amax=float(inp["act_amax"].item()), quant_format=qf, block_size=bs,
+                        dst_max=dst)
+    assert_conv_close(to_np_f32(y), ref, f"case {case} {qf}{bs} {dtype}", dtype)
+
+
+@pytest.mark.parametrize("quant", [False, True])
+def test_ex_matches_regular_entry_for_nvfp4_16_and_none(cuda_ok, quant):
+    xs, cout, k = (1, 16, 5, 12, 32), 48, (3, 3, 3)
+    inp = workloads.random_conv_inputs(61, xs, cout, k, dtype=torch.bfloat16, device="cuda")
+    pad6 = (2, 0, 1, 1, 1, 1)
+    y = api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], inp["bias"], 1, pad6, 1, act_amax=inp["act_amax"],
+                                    quant_format="nvfp4" if quant else "none", block_size=16)
+    r = api.conv3d_implicit_gemm(inp["x"], inp["w"], inp["bias"], 1, pad6, 1, act_amax=inp["act_amax"],
+                                 quant_act=quant)
+    assert api.check_device_error() == 0
+    assert torch.equal(y, r)
+
+
+def test_ex_mxfp4_needs_no_amax(cuda_ok):
+    inp = workloads.random_conv_inputs(62, (1, 8, 3, 8, 16), 16, (3, 3, 3), dtype=torch.bfloat16, device="cuda")
+    y = api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], None, 1, 1, 1, act_amax=None, quant_format="mxfp4",
+                                    block_size=32)
+    ref = oracle.conv3d(to_np_f32(inp["x"]), to_np_f32(inp["w"]), None, (1, 1, 1), (1, 1, 1), (1, 1, 1), (1, 1, 1),
+                        quant_act=True, quant_format="mxfp4", block_size=32)
+    assert_conv_close(to_np_f32(y), ref, "mxfp4 without amax", torch.bfloat16)
