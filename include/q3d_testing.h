@@ -62,6 +62,27 @@ Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_
                                       const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
                                       int32_t dtype, int32_t* plan, int32_t plan_len);
 
+/*
+ * q3d_selftest_withheld_arrive -- TEST HOOK of the bounded waits, not part
+ * of the convolution path.  Enqueues conv3d_implicit_gemm_pad2 (no bias, no
+ * quantisation) on the tensor-memory kernel, except that in CTA 0 one of the
+ * four epilogue warps withholds its arrival on the first hand-back of
+ * accumulator 0: the MMA issuer's wait for that accumulator at CTA 0's second
+ * tile never completes, gives up after the library's wait limit (2 s), sets
+ * the device error word's accumulator-empty site bit (1 << 5) and raises the
+ * CTA's abort flag; every role of CTA 0 then stops, after waiting for the
+ * bulk copies and tensor-core operations it has in flight, and the launch
+ * ends normally.  The other CTAs complete; out is unspecified.  The next
+ * q3d_check_device_error returns Q3D_ERR_DEVICE_TIMEOUT with the site bits
+ * and clears them; later calls are unaffected.
+ *   x, w  BF16, contiguous, K % 8 == 0, w 16-byte aligned; the problem must
+ *         run on the tensor-memory kernel with more tiles than CTAs
+ *         (Q3D_ERR_INVALID_ARG otherwise, nothing enqueued).
+ */
+Q3D_API q3d_status q3d_selftest_withheld_arrive(const q3d_tensor* x, const q3d_tensor* w, const int32_t stride[3],
+                                                const int32_t pad_lo[3], const int32_t pad_hi[3],
+                                                const int32_t dil[3], q3d_tensor* out, q3d_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

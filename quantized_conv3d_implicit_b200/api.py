@@ -27,7 +27,7 @@ EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit
            "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "fp4_fake_quant_bs", "mxfp4_quantize", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
-           "q3d_selftest_ratio", "q3d_plan_conv", "q3d_plan_conv_tmem")
+           "q3d_selftest_ratio", "q3d_selftest_withheld_arrive", "q3d_plan_conv", "q3d_plan_conv_tmem")
 
 
 class Q3DTensor(ctypes.Structure):
@@ -83,6 +83,8 @@ def load_library(path: Optional[str] = None):
         lib.q3d_version.restype = ctypes.c_int32
         lib.q3d_selftest_formats.restype = ctypes.c_int
         lib.q3d_selftest_formats.argtypes = [vp, ctypes.c_int64, vp, vp, vp]
+        lib.q3d_selftest_withheld_arrive.restype = ctypes.c_int
+        lib.q3d_selftest_withheld_arrive.argtypes = [T, T, i32x3, i32x3, i32x3, i32x3, T, vp]
         lib.q3d_selftest_ratio.restype = ctypes.c_int
         lib.q3d_selftest_ratio.argtypes = [vp, vp, ctypes.c_int64, vp, vp]
         i64x5 = ctypes.POINTER(ctypes.c_int64)
@@ -318,6 +320,19 @@ def selftest_formats(v: torch.Tensor, stream=None):
     st = lib.q3d_selftest_formats(v.data_ptr(), v.numel(), e2m1.data_ptr(), e4m3.data_ptr(), _stream_handle(stream))
     _check(lib, st)
     return e2m1, e4m3
+
+
+def selftest_withheld_arrive(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor, stride=1, padding=0,
+                             dilation=1, stream=None):
+    """Test hook of the bounded waits: the convolution with one hand-back
+    arrival withheld in CTA 0, so that CTA's MMA wait gives up and it aborts
+    (see q3d_testing.h)."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    st = lib.q3d_selftest_withheld_arrive(_ref(_tensor(x)), _ref(_tensor(w)), a3(_triple(stride)), a3(lo), a3(hi),
+                                          a3(_triple(dilation)), _ref(_tensor(out)), _stream_handle(stream))
+    _check(lib, st)
 
 
 def selftest_ratio(bmax: torch.Tensor, t: torch.Tensor, stream=None) -> torch.Tensor:

@@ -89,6 +89,7 @@ struct TmemParams {
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
   uint32_t off_dq, off_b, off_halo, off_code, off_epi, off_phase, off_bar;
   int y_vec;  // y is 16-byte aligned and OW a multiple of 16 / sizeof(T): vector stores
+  int withhold_arrive;  // test of the bounded waits only (0 otherwise): see the epilogue
 };
 
 struct TileCoord {
@@ -750,7 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c0 + 16 >= p.sub_n) {  // the accumulator is in registers: hand it back
               tc_fence_before();
               __syncwarp();
-              if (lane == 0) mbar_arrive(bar_acc_empty + 8u * acc);
+              // a test of the bounded waits withholds one of the four arrivals of
+              // CTA 0's first hand-back, so the MMA issuer's wait for it gives up
+              const bool withhold = p.withhold_arrive && blockIdx.x == 0 && it == 0 && acc == 0 && qw == 0;
+              if (lane == 0 && !withhold) mbar_arrive(bar_acc_empty + 8u * acc);
             }
             if (!vec_ok) {
               // rows whose length breaks 16-byte alignment: each lane writes its
@@ -1368,6 +1372,11 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
     if (cr != CUDA_SUCCESS) { *why = "weight tensor map rejected"; return cudaErrorInvalidValue; }
   }
   const int64_t grid64 = std::min<int64_t>(p.num_tiles, L.sm_count);
+  if (L.withhold_arrive) {
+    // the withheld hand-back is only waited for when CTA 0 has a second tile
+    if (p.num_tiles <= grid64) { *why = "the bounded-wait test needs more tiles than CTAs"; return cudaErrorInvalidValue; }
+    p.withhold_arrive = 1;
+  }
   *handled = true;
   switch (L.dtype) {
     case 0: return launch_tmem_typed<float>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);

@@ -542,6 +542,28 @@ q3d_status q3d_conv_out_shape(const int64_t x_shape[5], const int64_t w_shape[5]
   return Q3D_OK;
 }
 
+q3d_status q3d_selftest_withheld_arrive(const q3d_tensor* x, const q3d_tensor* w, const int32_t stride[3],
+                                        const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                                        q3d_tensor* out, q3d_stream_t stream) {
+  q3d::ConvGeom g;
+  q3d::ConvLaunch L;
+  bool noop = false;
+  q3d_status st = prepare_conv(x, w, nullptr, nullptr, stride, pad_lo, pad_hi, dil, 0, out, &g, &L, &noop);
+  if (st != Q3D_OK) return st;
+  if (noop || x->dtype != Q3D_BF16 || g.K % 8 != 0 || reinterpret_cast<uintptr_t>(w->data) % 16 != 0)
+    return fail(Q3D_ERR_INVALID_ARG, "the bounded-wait test takes BF16 weights usable in place and a non-empty output");
+  L.w_bf16 = w->data;
+  L.w_ld = g.K;
+  L.withhold_arrive = 1;
+  const char* why = nullptr;
+  bool handled = false;
+  cudaError_t e = q3d::launch_conv3d_tmem(g, L, reinterpret_cast<cudaStream_t>(stream), &why, &handled);
+  if (e != cudaSuccess)
+    return why ? fail(Q3D_ERR_INVALID_ARG, "%s", why) : cuda_fail(e, "bounded-wait test launch");
+  if (!handled) return fail(Q3D_ERR_INVALID_ARG, "the tensor-memory kernel does not take this problem");
+  return Q3D_OK;
+}
+
 q3d_status q3d_selftest_formats(const float* in, int64_t n, float* e2m1, float* e4m3, q3d_stream_t stream) {
   if (!in || !e2m1 || !e4m3) return fail(Q3D_ERR_NULLPTR, "NULL pointer");
   if (n < 0) return fail(Q3D_ERR_INVALID_ARG, "n < 0");

@@ -47,6 +47,7 @@ struct ConvLaunch {
   int qfmt = 1;             // quantiser when quant: 1 NVFP4 (blocks of qblock), 2 MXFP4 (groups of 32)
   int qblock = 16;
   float dst_max = 0.0f;     // MXFP4 only
+  int withhold_arrive = 0;  // test of the bounded waits (tensor-memory kernel only)
   unsigned int* err;        // device error word
   int sm_count;
   // stream-ordered pool of the device for the staged BF16 weights (kept
