@@ -68,9 +68,12 @@ Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_
  * quantisation) on the tensor-memory kernel, except that in CTA 0 one of the
  * four epilogue warps withholds its arrival on the first hand-back of
  * accumulator 0: the MMA issuer's wait for that accumulator at CTA 0's second
- * tile never completes, gives up after the library's wait limit (2 s), sets
- * the device error word's accumulator-empty site bit (1 << 5) and raises the
- * CTA's abort flag; every role of CTA 0 then stops, after waiting for the
+ * tile never completes, nor do the waits that depend on it (the transform
+ * warps' waits for a free A stage, the producers' for a free stage or slot,
+ * the epilogue's for the next accumulator).  The first of them to reach the
+ * library's wait limit (2 s) gives up, sets its site bit in the device error
+ * word (e.g. 1 << 5 for the accumulator, 1 << 3 for an A stage) and raises
+ * the CTA's abort flag; every role of CTA 0 then stops, after waiting for the
  * bulk copies and tensor-core operations it has in flight, and the launch
  * ends normally.  The other CTAs complete; out is unspecified.  The next
  * q3d_check_device_error returns Q3D_ERR_DEVICE_TIMEOUT with the site bits
