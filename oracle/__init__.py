@@ -13,8 +13,13 @@ GEMM CUDA kernel" article it follows (sections 5.1, 6.1-6.4, 7.1).
 The MXFP4 functions follow the CANN aclnnFlatQuantV2 page instead (its
 per-group route with E2M1 output, steps 3 and 4).
 
+The NVFP4-operand functions (``nvfp4_block_exact``, ``nvfp4_exact``,
+``conv3d_nvfp4``) define the true-FP4 variant: the same codes and block
+scales, the operand value q * s8 * g taken exactly.
+
 Parity pins: tests/test_oracle_formats.py, tests/test_oracle_fake_quant.py,
-tests/test_oracle_conv.py, tests/test_oracle_mxfp4.py.  No function here is
+tests/test_oracle_conv.py, tests/test_oracle_mxfp4.py,
+tests/test_oracle_nvfp4_exact.py.  No function here is
 "parity unpinned".
 """
 from __future__ import annotations
@@ -82,6 +87,13 @@ def _load():
             lib.oracle_conv3d_ex.argtypes = [vp, i64, i64, i64, i64, i64, vp, i64, i64, i64, i64, vp,
                                              i32p, i32p, i32p, i32p, ctypes.c_int, ctypes.c_int, f32, f32,
                                              vp, i64, ctypes.c_int, vp]
+            lib.oracle_nvfp4_block_exact.restype = None
+            lib.oracle_nvfp4_block_exact.argtypes = [vp, ctypes.c_int, f32, vp]
+            lib.oracle_nvfp4_exact.restype = ctypes.c_int
+            lib.oracle_nvfp4_exact.argtypes = [vp, i64, f32, vp]
+            lib.oracle_conv3d_nvfp4.restype = ctypes.c_int
+            lib.oracle_conv3d_nvfp4.argtypes = [vp, i64, i64, i64, i64, i64, vp, i64, i64, i64, i64, vp,
+                                                i32p, i32p, i32p, i32p, f32, f32, vp, i64, ctypes.c_int, vp]
             lib.oracle_conv3d.restype = ctypes.c_int
             lib.oracle_conv3d.argtypes = ([vp, i64, i64, i64, i64, i64, vp, i64, i64, i64, i64, vp,
                                            i32p, i32p, i32p, i32p, ctypes.c_int, f32, vp, i64,
@@ -284,6 +296,72 @@ def conv3d(x, w, bias=None, stride=(1, 1, 1), pad_lo=(0, 0, 0), pad_hi=None, dil
                               None if ml is None else _ptr(ml), n_m, int(nthreads), _ptr(y))
     if rc != 0:
         raise ValueError("oracle_conv3d: invalid arguments")
+    if m_list is None:
+        return y.reshape(N, OD, OH, OW, Cout).transpose(0, 4, 1, 2, 3).copy()
+    return y
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 operands taken exactly: the true-FP4 product (formats of sec. 6.1,
+# 6.2; weights quantised along K as in sec. 7.2)
+# ---------------------------------------------------------------------------
+
+def nvfp4_block_exact(v, amax: float) -> np.ndarray:
+    """One block of up to 16 values as exact NVFP4 operand values
+    sign * q * s8 * g (float64); the same codes and E4M3 scale as
+    ``fq_block``, and zero for a block that takes the 1.0 fallback scale."""
+    lib = _load()
+    v = _f32(v)
+    assert 1 <= v.size <= 16
+    out = np.empty(v.size, dtype=np.float64)
+    lib.oracle_nvfp4_block_exact(_ptr(v), v.size, float(np.float32(amax)), _ptr(out))
+    return out
+
+
+def nvfp4_exact(x, amax: float) -> np.ndarray:
+    """A flat tensor in consecutive blocks of 16, each as ``nvfp4_block_exact``."""
+    lib = _load()
+    x = _f32(x)
+    out = np.empty(x.shape, dtype=np.float64)
+    if lib.oracle_nvfp4_exact(_ptr(x), x.size, float(np.float32(amax)), _ptr(out)) != 0:
+        raise ValueError("nvfp4_exact: numel must be a multiple of 16")
+    return out
+
+
+def conv3d_nvfp4(x, w, bias=None, stride=(1, 1, 1), pad_lo=(0, 0, 0), pad_hi=None, dil=(1, 1, 1),
+                 act_amax: float = 0.0, w_amax: float = 0.0, m_list=None, nthreads: int = 0) -> np.ndarray:
+    """The true-FP4 convolution: every A row and every weight row quantised
+    to NVFP4 operands in blocks of 16 consecutive K elements (act_amax and
+    w_amax give the two global scales), multiplied exactly and summed in
+    binary64, plus the bias.  Shapes and m_list as in ``conv3d``."""
+    lib = _load()
+    x = _f32(x)
+    w = _f32(w)
+    if pad_hi is None:
+        pad_hi = pad_lo
+    N, C, D, H, W = x.shape
+    Cout, Cw, KD, KH, KW = w.shape
+    assert Cw == C
+    b = None if bias is None else _f32(bias)
+    arr = lambda t: (ctypes.c_int32 * 3)(*[int(v) for v in t])  # noqa: E731
+    OD, OH, OW = out_dims((D, H, W), (KD, KH, KW), stride, pad_lo, pad_hi, dil)
+    if min(OD, OH, OW) <= 0:
+        raise ValueError("oracle_conv3d_nvfp4: invalid arguments or empty output")
+    M = N * OD * OH * OW
+    if m_list is None:
+        ml = None
+        n_m = M
+    else:
+        ml = np.ascontiguousarray(np.asarray(m_list, dtype=np.int64))
+        n_m = ml.size
+    y = np.empty((n_m, Cout), dtype=np.float64)
+    rc = lib.oracle_conv3d_nvfp4(_ptr(x), N, C, D, H, W, _ptr(w), Cout, KD, KH, KW,
+                                 None if b is None else _ptr(b),
+                                 arr(stride), arr(pad_lo), arr(pad_hi), arr(dil),
+                                 float(np.float32(act_amax)), float(np.float32(w_amax)),
+                                 None if ml is None else _ptr(ml), n_m, int(nthreads), _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle_conv3d_nvfp4: invalid arguments")
     if m_list is None:
         return y.reshape(N, OD, OH, OW, Cout).transpose(0, 4, 1, 2, 3).copy()
     return y

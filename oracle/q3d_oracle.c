@@ -26,6 +26,12 @@
  * Where the article stops (rounding of E2M1 ties and of the E4M3 scale) the
  * specification of this library fixes round-to-nearest-even for both.
  *
+ * The NVFP4-operand functions (oracle_nvfp4_block_exact, the qfmt 3
+ * convolution) define the true-FP4 variant of the same quantiser: the
+ * article fixes the formats (sec. 6.1, 6.2) and the weight quantisation
+ * along K (sec. 7.2), and the product of the codes is taken exactly; see the
+ * comment above oracle_nvfp4_block_exact.
+ *
  * The MXFP4 functions follow a second page, the CANN aclnnFlatQuantV2
  * article (its per-group route with E2M1 output: groups of 32, a
  * power-of-two E8M0 scale, the dstTypeMax rule); see the comment above
@@ -216,6 +222,56 @@ int oracle_fp4_fake_quant_bs(const float* x, int64_t numel, float amax, int bloc
 }
 
 /* ------------------------------------------------------------------------ */
+/* NVFP4 operands taken exactly (the true-FP4 product)                        */
+/* ------------------------------------------------------------------------ */
+
+/* One block of n values (n <= 16; fewer as if zero-filled) quantised to an
+ * NVFP4 operand: the E2M1 magnitude codes q and the E4M3 block scale s8 are
+ * the ones oracle_fq_block takes (sec. 6.2, 6.3), and the operand value is
+ * sign * q * s8 * g computed exactly in binary64 (q has two significant
+ * bits, s8 four and g twenty-four, so the product is exact), without the
+ * binary32 rounding of scale and of q * scale, nor the BF16 rounding, of the
+ * fake-quantised path.  A block whose scale s8 * g falls below 1e-5 takes
+ * the fallback scale 1.0 in the article; that scale is not an E4M3 value
+ * times g, so in this variant such a block contributes zero. */
+void oracle_nvfp4_block_exact(const float* v, int n, float amax, double* out)
+{
+    /* global scale and the denominator of the block scale, as in oracle_fq_block */
+    float g = amax / 2688.0f;
+    float t = 6.0f * g;
+    float bmax = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(v[i]);
+        if (a > bmax) bmax = a;
+    }
+    float r = bmax / t;
+    r = fminf(r, 448.0f);
+    float s8 = oracle_e4m3_rne_sat(r);
+    float scale = s8 * g;
+    if (scale < 1e-5f) {
+        for (int i = 0; i < n; ++i) out[i] = 0.0;
+        return;
+    }
+    float inv = 1.0f / scale;
+    for (int i = 0; i < n; ++i) {
+        float a = fabsf(v[i]) * inv;
+        float q = oracle_e2m1_rne_sat(a);
+        double d = (double)q * (double)s8 * (double)g;
+        out[i] = signbit(v[i]) ? -d : d;
+    }
+}
+
+/* The flat tensor in consecutive blocks of 16 (sec. 6.4's view), each as
+ * oracle_nvfp4_block_exact.  Returns 0, or -1 if numel is not a multiple of
+ * 16. */
+int oracle_nvfp4_exact(const float* x, int64_t numel, float amax, double* out)
+{
+    if (numel % 16 != 0) return -1;
+    for (int64_t b = 0; b < numel; b += 16) oracle_nvfp4_block_exact(x + b, 16, amax, out + b);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* MXFP4 (E2M1 values, power-of-two E8M0 scale, groups of 32)                */
 /* ------------------------------------------------------------------------ */
 
@@ -339,8 +395,10 @@ typedef struct {
     int64_t sd, sh, sw, pd, ph, pw, dd, dh, dw;   /* stride, front pad, dilation */
     int64_t OD, OH, OW;
     int quant; float amax;
-    int qfmt; int qblock; float dst_max;   /* quantiser: 1 NVFP4 blocks of qblock, 2 MXFP4 groups of 32 */
-    const double* wb;        /* bf16(w) as binary64, [Cout][K] */
+    int qfmt; int qblock; float dst_max;   /* quantiser: 1 NVFP4 blocks of qblock, 2 MXFP4 groups of 32,
+                                               3 NVFP4 operands taken exactly (blocks of 16) */
+    const double* wb;        /* the B operand as binary64, [Cout][K]: bf16(w), or for qfmt 3 the
+                                exact NVFP4 operand of w */
     /* work list */
     const int64_t* m_list; int64_t n_m;
     double* y;               /* [n_m][Cout] */
@@ -380,7 +438,14 @@ static void* conv_worker(void* arg)
     for (int64_t i = j->lo; i < j->hi; ++i) {
         int64_t m = j->m_list[i];
         im2col_row(j, m, row);
-        if (j->quant && j->qfmt == 2) {
+        if (j->quant && j->qfmt == 3) {
+            /* exact NVFP4 operand: blocks of 16 consecutive K elements of this
+             * row, a short last block as if zero-filled; no BF16 rounding */
+            for (int64_t b = 0; b < K; b += 16) {
+                int nb = (int)((K - b) < 16 ? (K - b) : 16);
+                oracle_nvfp4_block_exact(row + b, nb, j->amax, a + b);
+            }
+        } else if (j->quant && j->qfmt == 2) {
             /* MXFP4 groups of 32 consecutive K elements of this row; a short
              * last group as if zero-filled (zeros leave its maximum alone) */
             for (int64_t b = 0; b < K; b += 32) {
@@ -398,8 +463,9 @@ static void* conv_worker(void* arg)
         } else {
             memcpy(fq, row, sizeof(float) * (size_t)K);
         }
-        /* the tensor-core operand is BF16 */
-        for (int64_t k = 0; k < K; ++k) a[k] = (double)oracle_bf16_round(fq[k]);
+        /* the tensor-core operand is BF16 (the exact NVFP4 operand is final) */
+        if (!(j->quant && j->qfmt == 3))
+            for (int64_t k = 0; k < K; ++k) a[k] = (double)oracle_bf16_round(fq[k]);
         for (int64_t co = 0; co < j->Cout; ++co) {
             const double* wr = j->wb + co * K;
             double s = 0.0;
@@ -429,14 +495,15 @@ int64_t oracle_out_dim(int64_t in, int64_t k, int64_t s, int64_t plo, int64_t ph
  * stride/pad_lo/pad_hi/dil are (d, h, w).  Returns 0, or -1 on bad
  * arguments.  nthreads <= 0 uses every online core.
  */
-int oracle_conv3d_ex(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
-                     const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
-                     const float* bias,
-                     const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
-                     const int32_t* dil, int qfmt, int qblock, float act_amax, float dst_max,
-                     const int64_t* m_list, int64_t n_m, int nthreads, double* y)
+static int conv3d_core(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
+                       const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
+                       const float* bias,
+                       const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
+                       const int32_t* dil, int qfmt, int qblock, float act_amax, float dst_max, float w_amax,
+                       const int64_t* m_list, int64_t n_m, int nthreads, double* y)
 {
-    if (qfmt < 0 || qfmt > 2) return -1;
+    if (qfmt < 0 || qfmt > 3) return -1;
+    if (qfmt == 3 && qblock != 16) return -1;
     if (qfmt == 1 && qblock != 16 && qblock != 32 && qblock != 64 && qblock != 128 && qblock != 256) return -1;
     if (qfmt == 2 && (qblock != 32 || !(dst_max == 0.0f || (dst_max >= 6.0f && dst_max <= 12.0f)))) return -1;
     for (int i = 0; i < 3; ++i)
@@ -468,7 +535,17 @@ int oracle_conv3d_ex(const float* x, int64_t N, int64_t C, int64_t D, int64_t H,
         if (m_list[i] < 0 || m_list[i] >= M) { free(all); return -1; }
 
     double* wb = (double*)malloc(sizeof(double) * (size_t)(Cout * K));
-    for (int64_t i = 0; i < Cout * K; ++i) wb[i] = (double)oracle_bf16_round(w[i]);
+    if (qfmt == 3) {
+        /* weights as NVFP4 operands: blocks of 16 along each row's K (sec. 7.2
+         * quantises the weights along the reduction axis), scale from w_amax */
+        for (int64_t co = 0; co < Cout; ++co)
+            for (int64_t b = 0; b < K; b += 16) {
+                int nb = (int)((K - b) < 16 ? (K - b) : 16);
+                oracle_nvfp4_block_exact(w + co * K + b, nb, w_amax, wb + co * K + b);
+            }
+    } else {
+        for (int64_t i = 0; i < Cout * K; ++i) wb[i] = (double)oracle_bf16_round(w[i]);
+    }
     base.wb = wb; base.m_list = m_list; base.n_m = n_m; base.y = y;
 
     if (nthreads <= 0) nthreads = (int)sysconf(_SC_NPROCESSORS_ONLN);
@@ -485,6 +562,35 @@ int oracle_conv3d_ex(const float* x, int64_t N, int64_t C, int64_t D, int64_t H,
     for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
     free(th); free(jobs); free(wb); free(all);
     return 0;
+}
+
+/* The convolution with a fake-quantised activation operand: qfmt 0 (none),
+ * 1 (NVFP4 blocks of qblock) or 2 (MXFP4 groups of 32, qblock 32). */
+int oracle_conv3d_ex(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
+                     const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
+                     const float* bias,
+                     const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
+                     const int32_t* dil, int qfmt, int qblock, float act_amax, float dst_max,
+                     const int64_t* m_list, int64_t n_m, int nthreads, double* y)
+{
+    if (qfmt == 3) return -1;
+    return conv3d_core(x, N, C, D, H, W, w, Cout, KD, KH, KW, bias, stride, pad_lo, pad_hi, dil, qfmt, qblock,
+                       act_amax, dst_max, 0.0f, m_list, n_m, nthreads, y);
+}
+
+/* The true-FP4 convolution: both operands quantised to NVFP4 in blocks of 16
+ * along K (activations with act_amax, weights with w_amax) and multiplied as
+ * exact operands (oracle_nvfp4_block_exact), summed in binary64, plus the
+ * bias. */
+int oracle_conv3d_nvfp4(const float* x, int64_t N, int64_t C, int64_t D, int64_t H, int64_t W,
+                        const float* w, int64_t Cout, int64_t KD, int64_t KH, int64_t KW,
+                        const float* bias,
+                        const int32_t* stride, const int32_t* pad_lo, const int32_t* pad_hi,
+                        const int32_t* dil, float act_amax, float w_amax,
+                        const int64_t* m_list, int64_t n_m, int nthreads, double* y)
+{
+    return conv3d_core(x, N, C, D, H, W, w, Cout, KD, KH, KW, bias, stride, pad_lo, pad_hi, dil, 3, 16,
+                       act_amax, 0.0f, w_amax, m_list, n_m, nthreads, y);
 }
 
 /* The article's convolution: NVFP4 blocks of 16 when quant_act is set. */
