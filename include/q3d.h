@@ -197,6 +197,57 @@ Q3D_API q3d_status conv3d_implicit_gemm_noalloc(const q3d_tensor* x, const q3d_t
                                         q3d_stream_t stream);
 
 /*
+ * The true-FP4 convolution: both operands quantised to NVFP4 and multiplied
+ * by the block-scaled tensor core (tcgen05.mma kind::mxf4nvf4).  The formats
+ * and codes are those of the article's quantiser (sec. 6.1-6.3: E2M1 values,
+ * an E4M3 scale E4M3(min(bmax / (6 g), 448)) per block of 16 consecutive K
+ * elements of a row, g = amax / (6 * 448)), applied to the activations with
+ * act_amax and, along their reduction axis K (sec. 7.2), to the weights with
+ * their own w_amax; the tensor core multiplies the codes and scales exactly
+ * and accumulates in FP32, and the epilogue multiplies by
+ * RN(g_act * g_w) and adds the bias.  The article dequantises to BF16
+ * instead, so the result differs from conv3d_implicit_gemm by the BF16
+ * rounding of both operands (and the weights are quantised here).  A block
+ * whose scale would take the article's 1.0 fallback (E4M3 code times g below
+ * 1e-5) contributes zero: 1.0 is no E4M3 scale times g.
+ *
+ * q3d_fp4_weight_bytes -- size in bytes of the packed weights of a
+ * [Cout, Cin, kd, kh, kw] weight tensor; -1 for a non-positive extent.
+ *
+ * conv3d_fp4_pack_weights -- quantise w into `packed`, once per set of
+ * weights (the convolution reads nothing else of w).
+ *   w        [Cout, Cin, kd, kh, kw] F32/F16/BF16, contiguous, on the device.
+ *   w_amax   device pointer to one float: the weights' global amax, e.g.
+ *            from q3d_act_amax(w).
+ *   packed   device buffer of packed_bytes >= q3d_fp4_weight_bytes(w.shape)
+ *            bytes, 256-byte aligned, not overlapping w; owned by the
+ *            caller.  Layout (opaque to callers, stated for the record): a
+ *            256-byte header whose first word is g_w, then per K slice of
+ *            64 and per N-part of the tile plan an image of the codes in
+ *            the layout the MMA reads and the scale bytes.
+ * Enqueues a memset of the buffer and one kernel on `stream`.
+ *
+ * conv3d_implicit_gemm_fp4 -- the convolution over packed weights.
+ *   x, bias, stride, pad_lo, pad_hi, dil, out, stream  as for
+ *            conv3d_implicit_gemm_pad2 (quant_act implied).
+ *   packed_w the buffer written by conv3d_fp4_pack_weights for weights of
+ *            shape w_shape (not checked against it on the host).
+ *   act_amax device pointer to one float: the activations' global amax.
+ * Runs on the tensor-memory kernel only: x 16-byte aligned with rows of W a
+ * multiple of 16 bytes and at most 343 taps, else
+ * Q3D_ERR_UNSUPPORTED_SHAPE.  Q3D_ERR_NULLPTR / _INVALID_ARG /
+ * _UNSUPPORTED_DTYPE as for conv3d_implicit_gemm_pad2, before anything is
+ * enqueued.
+ */
+Q3D_API int64_t q3d_fp4_weight_bytes(const int64_t w_shape[5]);
+Q3D_API q3d_status conv3d_fp4_pack_weights(const q3d_tensor* w, const float* w_amax, void* packed, int64_t packed_bytes,
+                                           q3d_stream_t stream);
+Q3D_API q3d_status conv3d_implicit_gemm_fp4(const q3d_tensor* x, const void* packed_w, const int64_t w_shape[5],
+                                            const q3d_tensor* bias, const float* act_amax, const int32_t stride[3],
+                                            const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                                            q3d_tensor* out, q3d_stream_t stream);
+
+/*
  * fp4_fake_quant -- out = NVFP4 fake-quantisation of x (sec. 6.4, 7.3).
  *   x     any rank 1..5, dtype F32/F16/BF16, numel % 16 == 0; consecutive
  *         groups of 16 elements in memory order form the blocks.

@@ -63,6 +63,17 @@ Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_
                                       int32_t dtype, int32_t* plan, int32_t plan_len);
 
 /*
+ * q3d_plan_conv_fp4 -- TEST HOOK: the plan conv3d_implicit_gemm_fp4 would
+ * use (host arithmetic only).  The fields of q3d_plan_conv_tmem up to the
+ * halo box extents, then: the first TMEM column of the scale factors, the
+ * TMEM columns per A stage, the bytes of one A stage in shared memory and of
+ * one weight stage.
+ */
+Q3D_API q3d_status q3d_plan_conv_fp4(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                                     const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                                     int32_t dtype, int32_t* plan, int32_t plan_len);
+
+/*
  * q3d_selftest_withheld_arrive -- TEST HOOK of the bounded waits, not part
  * of the convolution path.  Enqueues conv3d_implicit_gemm_pad2 (no bias, no
  * quantisation) on the tensor-memory kernel, except that in CTA 0 one of the

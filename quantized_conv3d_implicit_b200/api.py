@@ -27,7 +27,8 @@ EXPORTS = ("conv3d_implicit_gemm", "conv3d_implicit_gemm_pad2", "conv3d_implicit
            "conv3d_implicit_gemm_noalloc",
            "fp4_fake_quant", "fp4_fake_quant_bs", "mxfp4_quantize", "q3d_act_amax", "q3d_last_error",
            "q3d_check_device_error", "q3d_version", "q3d_conv_out_shape", "q3d_selftest_formats",
-           "q3d_selftest_ratio", "q3d_selftest_withheld_arrive", "q3d_plan_conv", "q3d_plan_conv_tmem")
+           "q3d_selftest_ratio", "q3d_selftest_withheld_arrive", "q3d_plan_conv", "q3d_plan_conv_tmem",
+           "q3d_fp4_weight_bytes", "conv3d_fp4_pack_weights", "conv3d_implicit_gemm_fp4", "q3d_plan_conv_fp4")
 
 
 class Q3DTensor(ctypes.Structure):
@@ -90,7 +91,13 @@ def load_library(path: Optional[str] = None):
         i64x5 = ctypes.POINTER(ctypes.c_int64)
         lib.q3d_conv_out_shape.restype = ctypes.c_int
         lib.q3d_conv_out_shape.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, i64x5]
-        for name in ("q3d_plan_conv", "q3d_plan_conv_tmem"):
+        lib.q3d_fp4_weight_bytes.restype = ctypes.c_int64
+        lib.q3d_fp4_weight_bytes.argtypes = [i64x5]
+        lib.conv3d_fp4_pack_weights.restype = ctypes.c_int
+        lib.conv3d_fp4_pack_weights.argtypes = [T, vp, vp, ctypes.c_int64, vp]
+        lib.conv3d_implicit_gemm_fp4.restype = ctypes.c_int
+        lib.conv3d_implicit_gemm_fp4.argtypes = [T, vp, i64x5, T, vp, i32x3, i32x3, i32x3, i32x3, T, vp]
+        for name in ("q3d_plan_conv", "q3d_plan_conv_tmem", "q3d_plan_conv_fp4"):
             fn = getattr(lib, name)
             fn.restype = ctypes.c_int
             fn.argtypes = [i64x5, i64x5, i32x3, i32x3, i32x3, i32x3, ctypes.c_int32,
@@ -229,6 +236,60 @@ def conv3d_implicit_gemm_ex(x: torch.Tensor, w: torch.Tensor, bias: Optional[tor
     return out
 
 
+class Fp4Weights:
+    """Weights packed for conv3d_implicit_gemm_fp4: the device buffer (uint8)
+    and the original [Cout, Cin, kd, kh, kw] shape."""
+
+    def __init__(self, packed: torch.Tensor, shape):
+        self.packed = packed
+        self.shape = tuple(int(v) for v in shape)
+
+
+def fp4_weight_bytes(w_shape) -> int:
+    """Bytes of the packed NVFP4 weights of a [Cout, Cin, kd, kh, kw] tensor."""
+    lib = load_library()
+    n = lib.q3d_fp4_weight_bytes((ctypes.c_int64 * 5)(*[int(v) for v in w_shape]))
+    if n < 0:
+        raise ValueError("w_shape must have five positive extents")
+    return int(n)
+
+
+def conv3d_fp4_pack_weights(w: torch.Tensor, w_amax: torch.Tensor, stream=None) -> Fp4Weights:
+    """Quantise w to NVFP4 operands (blocks of 16 along K, global scale
+    w_amax / 2688; w_amax a one-element float32 tensor on w's device) into a
+    new packed buffer for conv3d_implicit_gemm_fp4."""
+    lib = load_library()
+    _check_amax(w_amax, w, True)
+    n = fp4_weight_bytes(w.shape)
+    packed = torch.empty(n, dtype=torch.uint8, device=w.device)
+    ws = _tensor(w)
+    _check(lib, lib.conv3d_fp4_pack_weights(_ref(ws), w_amax.data_ptr(), packed.data_ptr(), n,
+                                            _stream_handle(stream)))
+    return Fp4Weights(packed, w.shape)
+
+
+def conv3d_implicit_gemm_fp4(x: torch.Tensor, wq: Fp4Weights, bias: Optional[torch.Tensor] = None, stride=1,
+                             padding=0, dilation=1, act_amax: Optional[torch.Tensor] = None,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The true-FP4 convolution: activations quantised to NVFP4 with act_amax,
+    weights packed by conv3d_fp4_pack_weights, block-scaled FP4 tensor-core
+    products with FP32 accumulation, result in x.dtype."""
+    lib = load_library()
+    lo, hi = _pads(padding)
+    if wq.packed.device != x.device:
+        raise ValueError("the packed weights must be on x's device")
+    if out is None:
+        out = torch.empty(out_shape(x.shape, wq.shape, stride, padding, dilation), dtype=x.dtype, device=x.device)
+    _check_amax(act_amax, x, True)
+    arr = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
+    xs, os_, bs = _tensor(x), _tensor(out), _tensor(bias)
+    st = lib.conv3d_implicit_gemm_fp4(_ref(xs), wq.packed.data_ptr(), (ctypes.c_int64 * 5)(*wq.shape), _ref(bs),
+                                      act_amax.data_ptr(), arr(_triple(stride)), arr(lo), arr(hi),
+                                      arr(_triple(dilation)), _ref(os_), _stream_handle(stream))
+    _check(lib, st)
+    return out
+
+
 def conv3d_implicit_gemm_noalloc(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor,
                                  bias: Optional[torch.Tensor] = None, stride=1, padding=0, dilation=1,
                                  act_amax: Optional[torch.Tensor] = None, quant_act: bool = False,
@@ -353,17 +414,19 @@ PLAN_FIELDS = ("applicable", "TH", "TW", "n_mt", "groups", "n_tile", "n_ntiles",
 
 def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfloat16, kernel="fast") -> dict:
     """Test hook (host only): the tiling/pipeline plan of the shared-memory
-    specialised kernel (kernel="fast") or of the tensor-memory kernel
-    (kernel="tmem", one more field: a_col0)."""
+    specialised kernel (kernel="fast"), of the tensor-memory kernel
+    (kernel="tmem", one more field: a_col0) or of its NVFP4-operand variant
+    (kernel="fp4", four more: sf_col0, sf_cols, a_stage_bytes, b_stage_bytes)."""
     lib = load_library()
     lo, hi = _pads(padding)
     a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
     a5 = lambda t: (ctypes.c_int64 * 5)(*[int(v) for v in t])  # noqa: E731
     out = (ctypes.c_int32 * 32)()
-    fn = lib.q3d_plan_conv_tmem if kernel == "tmem" else lib.q3d_plan_conv
+    fn = {"tmem": lib.q3d_plan_conv_tmem, "fp4": lib.q3d_plan_conv_fp4}.get(kernel, lib.q3d_plan_conv)
     st = fn(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)), _DTYPES[dtype],
             out, 32)
     _check(lib, st)
-    fields = PLAN_FIELDS + (("a_col0",) if kernel == "tmem" else ())
+    extra = {"tmem": ("a_col0",), "fp4": ("sf_col0", "sf_cols", "a_stage_bytes", "b_stage_bytes")}
+    fields = PLAN_FIELDS + extra.get(kernel, ())
     return dict(zip(fields, list(out)[:len(fields)]))
 

@@ -350,6 +350,84 @@ q3d_status conv3d_implicit_gemm_ex(const q3d_tensor* x, const q3d_tensor* w, con
   return run_conv(g, L, w, x->dtype, stream);
 }
 
+int64_t q3d_fp4_weight_bytes(const int64_t w_shape[5]) {
+  if (!w_shape) return -1;
+  for (int i = 0; i < 5; ++i)
+    if (w_shape[i] < 1) return -1;
+  const int64_t K = w_shape[1] * w_shape[2] * w_shape[3] * w_shape[4];
+  q3d::Fp4WeightLayout lay;
+  if (!q3d::fp4_weight_layout(w_shape[0], K, &lay)) return -1;
+  return lay.bytes;
+}
+
+q3d_status conv3d_fp4_pack_weights(const q3d_tensor* w, const float* w_amax, void* packed, int64_t packed_bytes,
+                                   q3d_stream_t stream) {
+  q3d_status st;
+  if ((st = check_tensor(w, "w", 5)) != Q3D_OK) return st;
+  if (!w_amax) return fail(Q3D_ERR_NULLPTR, "w_amax is NULL");
+  if (!packed) return fail(Q3D_ERR_NULLPTR, "packed is NULL");
+  const int64_t need = q3d_fp4_weight_bytes(w->shape);
+  if (need < 0) return fail(Q3D_ERR_INVALID_ARG, "w must have positive extents (and at most 2^20 output channels)");
+  if (packed_bytes < need)
+    return fail(Q3D_ERR_INVALID_ARG, "packed holds %lld bytes; these weights need %lld", (long long)packed_bytes,
+                (long long)need);
+  if (reinterpret_cast<uintptr_t>(packed) % 256 != 0) return fail(Q3D_ERR_INVALID_ARG, "packed must be 256-byte aligned");
+  const uintptr_t p0 = reinterpret_cast<uintptr_t>(packed), w0 = reinterpret_cast<uintptr_t>(w->data);
+  const uintptr_t w1 = w0 + static_cast<uintptr_t>(numel(w) * dtype_size(w->dtype));
+  if (p0 < w1 && w0 < p0 + static_cast<uintptr_t>(need)) return fail(Q3D_ERR_INVALID_ARG, "packed overlaps w");
+  const int64_t K = w->shape[1] * w->shape[2] * w->shape[3] * w->shape[4];
+  if (K > 0x7FFFFFFFll / 2) return fail(Q3D_ERR_UNSUPPORTED_SHAPE, "K exceeds the 32-bit index range");
+  DeviceInfo* dev = nullptr;
+  if ((st = current_device(&dev)) != Q3D_OK) return st;
+  q3d::Fp4WeightLayout lay;
+  q3d::fp4_weight_layout(w->shape[0], K, &lay);
+  const cudaError_t e = q3d::launch_fp4_pack_weights(w->data, w->dtype, static_cast<int32_t>(w->shape[0]),
+                                                     static_cast<int32_t>(K), w_amax, packed, lay,
+                                                     reinterpret_cast<cudaStream_t>(stream), dev->sm_count);
+  if (e != cudaSuccess) return cuda_fail(e, "NVFP4 weight packing");
+  return Q3D_OK;
+}
+
+q3d_status conv3d_implicit_gemm_fp4(const q3d_tensor* x, const void* packed_w, const int64_t w_shape[5],
+                                    const q3d_tensor* bias, const float* act_amax, const int32_t stride[3],
+                                    const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],
+                                    q3d_tensor* out, q3d_stream_t stream) {
+  if (!x) return fail(Q3D_ERR_NULLPTR, "x is NULL");
+  if (!packed_w) return fail(Q3D_ERR_NULLPTR, "packed_w is NULL");
+  if (!w_shape) return fail(Q3D_ERR_NULLPTR, "w_shape is NULL");
+  if (!act_amax) return fail(Q3D_ERR_NULLPTR, "act_amax is NULL");
+  const int64_t need = q3d_fp4_weight_bytes(w_shape);
+  if (need < 0) return fail(Q3D_ERR_INVALID_ARG, "w_shape must have positive extents");
+  if (reinterpret_cast<uintptr_t>(packed_w) % 256 != 0)
+    return fail(Q3D_ERR_INVALID_ARG, "packed_w must be 256-byte aligned");
+  // the weights' shape, for the shared checks (their data is the packed buffer)
+  q3d_tensor wd;
+  wd.data = const_cast<void*>(packed_w);
+  wd.dtype = x->dtype;
+  wd.ndim = 5;
+  for (int i = 0; i < 5; ++i) wd.shape[i] = w_shape[i];
+  q3d::ConvGeom g;
+  q3d::ConvLaunch L;
+  bool noop = false;
+  q3d_status st = prepare_conv(x, &wd, bias, act_amax, stride, pad_lo, pad_hi, dil, 1, out, &g, &L, &noop);
+  if (st != Q3D_OK || noop) return st;
+  const uintptr_t o0 = reinterpret_cast<uintptr_t>(out->data), p0 = reinterpret_cast<uintptr_t>(packed_w);
+  if (o0 < p0 + static_cast<uintptr_t>(need) && p0 < o0 + static_cast<uintptr_t>(numel(out) * dtype_size(out->dtype)))
+    return fail(Q3D_ERR_INVALID_ARG, "out overlaps packed_w");
+  const char* why = nullptr;
+  bool handled = false;
+  const cudaError_t e = q3d::launch_conv3d_fp4(g, L, packed_w, reinterpret_cast<cudaStream_t>(stream), &why, &handled);
+  if (e != cudaSuccess) {
+    if (why) return fail(Q3D_ERR_CUDA, "NVFP4 conv3d launch: %s (%s)", why, cudaGetErrorString(e));
+    return cuda_fail(e, "NVFP4 conv3d launch");
+  }
+  if (!handled)
+    return fail(Q3D_ERR_UNSUPPORTED_SHAPE,
+                "the NVFP4-operand convolution needs a 16-byte aligned x whose rows are a multiple of 16 bytes, at "
+                "most 343 taps, and a tile plan that fits");
+  return Q3D_OK;
+}
+
 q3d_status conv3d_implicit_gemm(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
                                 const float* act_amax, const int32_t stride[3], const int32_t pad[3],
                                 const int32_t dil[3], int32_t quant_act, q3d_tensor* out, q3d_stream_t stream) {
@@ -620,6 +698,16 @@ q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape[5], con
   const q3d_status st = plan_geom(x_shape, w_shape, stride, pad_lo, pad_hi, dil, dtype, plan, &g);
   if (st != Q3D_OK) return st;
   q3d::plan_conv3d_fast(g, dtype, plan, plan_len);
+  return Q3D_OK;
+}
+
+q3d_status q3d_plan_conv_fp4(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
+                             const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3], int32_t dtype,
+                             int32_t* plan, int32_t plan_len) {
+  q3d::ConvGeom g;
+  const q3d_status st = plan_geom(x_shape, w_shape, stride, pad_lo, pad_hi, dil, dtype, plan, &g);
+  if (st != Q3D_OK) return st;
+  q3d::plan_conv3d_fp4(g, dtype, plan, plan_len);
   return Q3D_OK;
 }
 

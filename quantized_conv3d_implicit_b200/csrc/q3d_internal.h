@@ -93,6 +93,30 @@ bool plan_conv3d_fast(const ConvGeom& g, int dtype, int32_t* out, int n_out);
 // vectorised reads = 0; one more entry: the first TMEM column of A).
 bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out);
 
+// Packed NVFP4 weights of the block-scaled convolution variant: a 256-byte
+// header (word 0: the weights' global scale g_w = w_amax / 2688, binary32),
+// then one image per (K slice of 64, N-part) in slice-major order.  An image
+// is sub_n rows x 32 bytes of E2M1 codes (two per byte, element 2i in the low
+// nibble) in the 32-byte-swizzled K-major layout the MMA reads, then n_atoms
+// 512-byte scale atoms (row n of the part at byte 16 * (n % 32) +
+// 4 * ((n / 32) % 4) + block of atom n / 128; unsigned E4M3, 0 for a block
+// that takes the 1.0 fallback).  Rows past Cout and columns past K are zero.
+struct Fp4WeightLayout {
+  int32_t n_tile, n_ntiles, n_sub, sub_n, ks, n_atoms, n_parts;
+  int64_t img_bytes, bytes;
+};
+constexpr int64_t kFp4WeightHeaderBytes = 256;
+bool fp4_weight_layout(int64_t Cout, int64_t K, Fp4WeightLayout* out);
+// Quantise w [Cout, K] (dtype) into `packed` (zeroed first, on s).
+cudaError_t launch_fp4_pack_weights(const void* w, int dtype, int32_t Cout, int32_t K, const float* w_amax,
+                                    void* packed, const Fp4WeightLayout& lay, cudaStream_t s, int sm_count);
+// The NVFP4-operand convolution over packed weights (*handled false when the
+// tensor-memory kernel does not apply to the problem).
+cudaError_t launch_conv3d_fp4(const ConvGeom& g, const ConvLaunch& L, const void* packed, cudaStream_t s,
+                              const char** why, bool* handled);
+// The plan of that variant (test hook; the fields of plan_conv3d_tmem).
+bool plan_conv3d_fp4(const ConvGeom& g, int dtype, int32_t* out, int n_out);
+
 // The implicit-GEMM convolution; returns a CUDA error or cudaSuccess, and a
 // short reason in *why when it rejects the problem before launching.
 cudaError_t launch_conv3d_igemm(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why);

@@ -280,6 +280,82 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_amn(uint32_t M, uint3
   return umma_idesc_bf16_f32(M, N) | (1u << 15);
 }
 
+// ---------------------------------------------------------------------------
+// Block-scaled FP4 MMA (kind::mxf4nvf4, NVFP4: E2M1 operands packed two per
+// byte, element 2i in the low nibble; unsigned E4M3 scale factors, one per 16
+// consecutive K elements of a row, held in tensor memory)
+// ---------------------------------------------------------------------------
+
+// Shared-memory matrix descriptor for a K-major operand in the canonical
+// 32-byte-swizzled layout: rows of 32 bytes (64 E2M1 values, one MMA's K),
+// groups of 8 rows 256 bytes apart, 16-byte chunk j of row r stored at chunk
+// (j ^ ((r >> 2) & 1)).  The tile must start on a 256-byte boundary.
+__device__ __forceinline__ uint64_t umma_desc_kmajor_sw32(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);  // start address, 16-B units
+  d |= (uint64_t)(1u) << 16;                    // leading byte offset (unused: one atom along K)
+  d |= (uint64_t)(256u >> 4) << 32;             // stride byte offset: 8-row group pitch
+  d |= (uint64_t)1u << 46;                      // descriptor version (sm_100)
+  d |= (uint64_t)6u << 61;                      // layout: 32-byte swizzle
+  return d;
+}
+
+// Shared-memory descriptor of a scale-factor atom, the source of
+// tcgen05.cp.32x128b: 32 rows of 16 bytes stored contiguously (no swizzle;
+// core matrices of 8 rows x 16 bytes, 128 bytes apart).
+__device__ __forceinline__ uint64_t umma_desc_sf_atom(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128u >> 4) << 16;
+  d |= (uint64_t)(128u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  return d;  // layout type 0: no swizzle
+}
+
+// Instruction descriptor for kind::mxf4nvf4 with E2M1 A and B (both K-major),
+// UE4M3 scale factors (scale-factor ids 0), FP32 accumulator, M x N, K = 64.
+__host__ __device__ constexpr uint32_t umma_idesc_nvfp4(uint32_t M, uint32_t N) {
+  return (1u << 7)            // A format: E2M1
+         | (1u << 10)         // B format: E2M1
+         | ((N >> 3) << 17)   // N / 8
+         | ((M >> 4) << 24);  // M / 16  (bit 23 = 0: UE4M3 scale factors)
+}
+
+// D (+)= (A x SFA) * (B x SFB) over K = 64, A and B from shared memory, the
+// scale factors at tensor-memory addresses sfa / sfb; the whole (converged)
+// warp calls it and elect.sync picks the issuing lane.
+__device__ __forceinline__ void umma_nvfp4_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                    uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 32-row x 16-byte shared-memory atom into tensor memory, replicated
+// into all four lane quadrants: row r lands in lanes r, 32 + r, 64 + r and
+// 96 + r, bytes 4j..4j+3 of it in column taddr + j.  Issued like the MMA and
+// executed in order with the MMAs this thread issues after it.
+__device__ __forceinline__ void tmem_cp_sf_atom_elect(uint32_t taddr, uint64_t s_desc) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}" ::"r"(taddr), "l"(s_desc)
+      : "memory");
+}
+
+// Bulk copy of `bytes` contiguous bytes (both addresses 16-byte aligned, size
+// a multiple of 16) from global into this CTA's shared memory, completing as
+// transaction bytes on the mbarrier.  No multicast.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // Named barrier over `nthreads` threads (a multiple of 32) with id 1..15.
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

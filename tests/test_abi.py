@@ -219,3 +219,76 @@ def test_conv_ex_validation(lib):
     assert ex(2, 16, 0.0) == 2
     assert ex(2, 32, 3.0) == 2 and b"dst_type_max" in lib.q3d_last_error()
     assert ex(1, 32, 0.0, amax=None) == 1            # NVFP4 needs act_amax
+
+
+def _fp4_layout_bytes(shape):
+    """The packed-weight size the header documents: 256 + ks * parts * image."""
+    cout, K = shape[0], shape[1] * shape[2] * shape[3] * shape[4]
+    n_ntiles, n_tile = 1, (cout + 15) // 16 * 16
+    if n_tile > 448:
+        n_ntiles = -(-cout // 448)
+        n_tile = (-(-cout // n_ntiles) + 15) // 16 * 16
+    n_sub = -(-n_tile // 256)
+    sub_n = (-(-n_tile // n_sub) + 15) // 16 * 16
+    img = sub_n * 32 + -(-sub_n // 128) * 512
+    return 256 + -(-K // 64) * n_ntiles * n_sub * img
+
+
+def test_fp4_weight_bytes(lib):
+    a5 = lambda v: (ctypes.c_int64 * 5)(*v)  # noqa: E731
+    for shape in [(5, 3, 3, 3, 3), (96, 96, 3, 3, 3), (192, 192, 3, 3, 3), (384, 384, 3, 3, 3), (500, 2, 3, 3, 3),
+                  (1024, 512, 1, 1, 1), (16, 16, 3, 3, 3), (33, 37, 1, 1, 1)]:
+        assert lib.q3d_fp4_weight_bytes(a5(shape)) == _fp4_layout_bytes(shape), shape
+        assert api.fp4_weight_bytes(shape) == _fp4_layout_bytes(shape)
+    assert lib.q3d_fp4_weight_bytes(a5((0, 3, 3, 3, 3))) == -1
+    assert lib.q3d_fp4_weight_bytes(None) == -1
+
+
+def test_fp4_validation(lib):
+    arr = lambda v: (ctypes.c_int32 * 3)(*v)  # noqa: E731
+    a5 = lambda v: (ctypes.c_int64 * 5)(*v)  # noqa: E731
+    r = ctypes.byref
+    w = T((5, 4, 3, 3, 3), 2, FAKE)
+    need = _fp4_layout_bytes((5, 4, 3, 3, 3))
+    packed = FAKE * 4096
+    assert lib.conv3d_fp4_pack_weights(None, FAKE * 8, packed, need, None) == 1
+    assert lib.conv3d_fp4_pack_weights(r(w), None, packed, need, None) == 1
+    assert lib.conv3d_fp4_pack_weights(r(w), FAKE * 8, None, need, None) == 1
+    assert lib.conv3d_fp4_pack_weights(r(w), FAKE * 8, packed, need - 16, None) == 2
+    assert lib.conv3d_fp4_pack_weights(r(w), FAKE * 8, packed + 16, need, None) == 2     # alignment
+    assert lib.conv3d_fp4_pack_weights(r(w), FAKE * 8, FAKE, need, None) == 2            # overlaps w
+    assert lib.conv3d_fp4_pack_weights(r(T((5, 4, 3, 3, 3), 7, FAKE)), FAKE * 8, packed, need, None) == 3
+    x, out = T((1, 4, 3, 8, 8), 2, FAKE), T((1, 5, 3, 8, 8), 2, FAKE * 256)
+    ws = a5((5, 4, 3, 3, 3))
+
+    def fp4(x=x, pw=packed, ws=ws, amax=FAKE * 8, out=out, plo=(1, 1, 1)):
+        return lib.conv3d_implicit_gemm_fp4(r(x) if x is not None else None, pw, ws, None, amax, arr((1, 1, 1)),
+                                            arr(plo), arr((1, 1, 1)), arr((1, 1, 1)),
+                                            r(out) if out is not None else None, None)
+    assert fp4(x=None) == 1
+    assert fp4(pw=None) == 1
+    assert fp4(ws=None) == 1
+    assert fp4(amax=None) == 1
+    assert fp4(pw=packed + 16) == 2
+    assert fp4(ws=a5((5, 3, 3, 3, 3))) == 2                       # Cin mismatch
+    assert fp4(out=T((1, 5, 3, 8, 9), 2, FAKE * 256)) == 2         # wrong out shape
+    assert fp4(out=T((1, 5, 3, 8, 8), 2, packed + 64)) == 2        # out overlaps the packed weights
+    assert fp4() in (4, 5)                                         # valid: no GPU here
+
+
+def test_fp4_plans_fit_every_workload():
+    from quantized_conv3d_implicit_b200 import workloads
+    for name, wl in workloads.WORKLOADS.items():
+        ws = (wl.cout, wl.x_shape[1]) + tuple(wl.kernel)
+        pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+        p = api.plan_conv(wl.x_shape, ws, wl.stride, pad6, wl.dil, wl.dtype, kernel="fp4")
+        assert p["applicable"], name
+        assert p["smem"] <= 232448, name
+        # accumulators, then sa scale-factor regions, inside the 512 TMEM columns
+        assert p["n_mt"] * p["n_tile"] <= p["sf_col0"], name
+        assert p["sf_col0"] + p["sa"] * p["sf_cols"] <= 512, name
+        assert p["sf_cols"] == 4 * p["n_mt"] + 4 * -(-p["sub_n"] // 128) * p["n_sub"], name
+        # an A stage holds n_mt subtiles of 128 rows x 32 bytes plus a 512-byte scale atom each
+        assert p["a_stage_bytes"] >= p["n_mt"] * (4096 + 512) and p["a_stage_bytes"] % 1024 == 0, name
+        assert p["b_stage_bytes"] >= p["n_sub"] * (p["sub_n"] * 32 + -(-p["sub_n"] // 128) * 512), name
+        assert 2 <= p["sa"] <= 4 and p["sb"] >= 2, name
