@@ -158,11 +158,13 @@ q3d_status check_tensor(const q3d_tensor* t, const char* name, int ndim) {
 
 // Host-side checks and geometry shared by the convolution entry points.
 // Returns Q3D_OK with *noop set for an empty batch or Cout == 0 (nothing to
-// enqueue); otherwise fills *g and *L (weights not yet staged).
+// enqueue); otherwise fills *g and *L (weights not yet staged).  With
+// w_is_tensor false, w only describes the weights' shape (its data is a
+// packed buffer whose overlap the caller checks).
 q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias, const float* act_amax,
                         const int32_t stride[3], const int32_t pad_lo[3], const int32_t pad_hi[3],
                         const int32_t dil[3], int32_t quant_act, q3d_tensor* out, q3d::ConvGeom* gp,
-                        q3d::ConvLaunch* Lp, bool* noop) {
+                        q3d::ConvLaunch* Lp, bool* noop, bool w_is_tensor = true) {
   *noop = false;
   q3d_status st;
   if ((st = check_tensor(x, "x", 5)) != Q3D_OK) return st;
@@ -192,7 +194,7 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
     *noop = true;
     return Q3D_OK;
   }
-  if (overlaps(out, x) || overlaps(out, w) || (bias && overlaps(out, bias)))
+  if (overlaps(out, x) || (w_is_tensor && overlaps(out, w)) || (bias && overlaps(out, bias)))
     return fail(Q3D_ERR_INVALID_ARG, "out overlaps an input tensor");
   const int64_t K = C * KD * KH * KW;
   const int64_t M = N * o_dims[0] * o_dims[1] * o_dims[2];
@@ -406,14 +408,17 @@ q3d_status conv3d_implicit_gemm_fp4(const q3d_tensor* x, const void* packed_w, c
   wd.dtype = x->dtype;
   wd.ndim = 5;
   for (int i = 0; i < 5; ++i) wd.shape[i] = w_shape[i];
+  if (out && out->ndim == 5 && dtype_ok(out->dtype)) {
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(out->data), p0 = reinterpret_cast<uintptr_t>(packed_w);
+    if (o0 < p0 + static_cast<uintptr_t>(need) && p0 < o0 + static_cast<uintptr_t>(numel(out) * dtype_size(out->dtype)))
+      return fail(Q3D_ERR_INVALID_ARG, "out overlaps packed_w");
+  }
   q3d::ConvGeom g;
   q3d::ConvLaunch L;
   bool noop = false;
-  q3d_status st = prepare_conv(x, &wd, bias, act_amax, stride, pad_lo, pad_hi, dil, 1, out, &g, &L, &noop);
+  q3d_status st = prepare_conv(x, &wd, bias, act_amax, stride, pad_lo, pad_hi, dil, 1, out, &g, &L, &noop,
+                               /*w_is_tensor=*/false);
   if (st != Q3D_OK || noop) return st;
-  const uintptr_t o0 = reinterpret_cast<uintptr_t>(out->data), p0 = reinterpret_cast<uintptr_t>(packed_w);
-  if (o0 < p0 + static_cast<uintptr_t>(need) && p0 < o0 + static_cast<uintptr_t>(numel(out) * dtype_size(out->dtype)))
-    return fail(Q3D_ERR_INVALID_ARG, "out overlaps packed_w");
   const char* why = nullptr;
   bool handled = false;
   const cudaError_t e = q3d::launch_conv3d_fp4(g, L, packed_w, reinterpret_cast<cudaStream_t>(stream), &why, &handled);
