@@ -50,7 +50,10 @@ L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-KERNEL_SOURCES = ("conv3d_igemm_tmem.cu", "sm100_ptx.cuh", "nvfp4.cuh")
+KERNEL_SOURCES = ("conv3d_igemm_tmem.cu", "conv3d_tmem_kernel.cuh", "sm100_ptx.cuh", "nvfp4.cuh")
+# nominal dense FP4 : BF16 tensor throughput of B200 (9 : 2.25 PFLOP/s); the
+# FP4 roofline is the measured BF16 peak times this ratio
+FP4_OVER_BF16 = 4.0
 
 
 def profiled_traffic(workload: str):
@@ -255,14 +258,41 @@ def time_conv_only(api, wl, sets, stream, dev, steps, warmup):
     return statistics.mean(t), min(t)
 
 
+def time_fp4_only(api, wl, sets, stream, dev, steps, warmup):
+    """As time_conv_only for the true-FP4 convolution (weights packed once per
+    input set, outside the timed launches)."""
+    import torch
+    packed = [api.conv3d_fp4_pack_weights(s["w"], api.act_amax(s["w"], stream=stream), stream=stream) for s in sets]
+
+    def call(i):
+        s = sets[i % len(sets)]
+        api.conv3d_implicit_gemm_fp4(s["x"], packed[i % len(sets)], s["bias"], wl.stride, pad6(wl), wl.dil,
+                                     s["act_amax"], out=s["out"], stream=stream)
+    for i in range(warmup):
+        call(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i, (a, b) in enumerate(ev):
+        a.record(stream)
+        call(i)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    if api.check_device_error(stream) != 0:
+        raise RuntimeError(f"device error in the FP4 convolution of {wl.name}")
+    t = [a.elapsed_time(b) for a, b in ev]
+    return statistics.mean(t), min(t)
+
+
 def run_layers(api, args, stream, dev, peak, headline_sets, headline_name, rank):
     """Every workload's convolution alone: us, TFLOP/s and fraction of the
-    measured BF16 peak, with the clocks seen while they ran."""
+    measured BF16 peak, with the clocks seen while they ran; and (unless
+    --no-fp4) the true-FP4 convolution of every quantised workload against
+    the FP4 roofline (measured BF16 peak x FP4_OVER_BF16)."""
     import torch
 
     from quantized_conv3d_implicit_b200 import workloads
     steps = max(5, min(args.steps, 20))
-    out = {}
+    out, fp4 = {}, {}
     sampler = ClockSampler(dev.index)
     sampler.start()
     for name, wl in workloads.WORKLOADS.items():
@@ -271,11 +301,17 @@ def run_layers(api, args, stream, dev, peak, headline_sets, headline_name, rank)
         tf = wl.flops / (mean_ms * 1e-3) / 1e12
         out[name] = {"us": round(mean_ms * 1e3, 2), "us_min": round(min_ms * 1e3, 2), "tflops": round(tf, 2),
                      "frac": round(tf / peak, 4), "launches": steps}
+        if not args.no_fp4 and wl.quant_act:
+            f_ms, f_min = time_fp4_only(api, wl, sets, stream, dev, steps, max(3, args.warmup))
+            ftf = wl.flops / (f_ms * 1e-3) / 1e12
+            fp4[name] = {"us": round(f_ms * 1e3, 2), "us_min": round(f_min * 1e3, 2), "tflops": round(ftf, 2),
+                         "frac": round(ftf / (peak * FP4_OVER_BF16), 4), "speedup_vs_bf16": round(mean_ms / f_ms, 3),
+                         "launches": steps}
         if sets is not headline_sets:
             del sets
             torch.cuda.empty_cache()
     clocks = sampler.stop()
-    return out, clocks
+    return out, fp4, clocks
 
 
 def run_ours(args, world, rank, local):
@@ -345,9 +381,9 @@ def run_ours(args, world, rank, local):
     amax_us = time_act_amax(base["x"], stream, dev, args.steps)
 
     # every workload's convolution alone (outside the step's timed region)
-    layers, layer_clocks = (None, None)
+    layers, layers_fp4, layer_clocks = (None, None, None)
     if not args.no_layers:
-        layers, layer_clocks = run_layers(api, args, stream, dev, peak, sets, wl.name, rank)
+        layers, layers_fp4, layer_clocks = run_layers(api, args, stream, dev, peak, sets, wl.name, rank)
 
     # end-to-end through the public API with pinned host buffers
     e2e = None if args.no_e2e else run_e2e(args, wl, base, stream, dev, world)
@@ -397,6 +433,14 @@ def run_ours(args, world, rank, local):
     if layers is not None:
         result["layers"] = layers
         result["layers_clocks"] = layer_clocks
+    if layers_fp4:
+        result["layers_fp4"] = {
+            "what": ("conv3d_implicit_gemm_fp4: activations and weights NVFP4, block-scaled FP4 MMA "
+                     "(kind::mxf4nvf4), weights packed outside the timed launches"),
+            "peak": round(peak * FP4_OVER_BF16, 1), "unit": "TFLOP/s",
+            "peak_source": f"{peaks_src} bf16_tflops (burst) x {FP4_OVER_BF16:g} (nominal FP4:BF16 dense ratio)",
+            "layers": layers_fp4,
+        }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(wl, base, budget_s=args.cpu_budget)
     if rank == 0:
@@ -581,6 +625,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-layers", action="store_true", help="skip the per-workload convolution timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end timing with host copies")
+    ap.add_argument("--no-fp4", action="store_true", help="skip the true-FP4 convolution timings")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
