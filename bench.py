@@ -195,7 +195,7 @@ def pad6(wl):
     return (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
 
 
-def workload_config(wl, world: int = 1) -> dict:
+def workload_config(wl, world: int = 1, fp4: bool = False) -> dict:
     """The `config` object of the JSON line (identical in both arms)."""
     od, oh, ow = wl.out_spatial()
     esz = {"torch.bfloat16": 2, "torch.float16": 2, "torch.float32": 4}[str(wl.dtype)]
@@ -210,7 +210,8 @@ def workload_config(wl, world: int = 1) -> dict:
         "workload": wl.name, "x": list(wl.x_shape), "w": [wl.cout, wl.x_shape[1], *wl.kernel],
         "stride": list(wl.stride), "pad_lo": list(wl.pad_lo), "pad_hi": list(wl.pad_hi), "dil": list(wl.dil),
         "quant_act": wl.quant_act, "M": wl.m_gemm, "N": wl.cout, "K": wl.k_gemm, "out": [od, oh, ow],
-        "step": "conv3d_implicit_gemm(quant_act) + fp4_fake_quant(x)",
+        "step": ("conv3d_implicit_gemm_fp4 (weights packed beforehand) + fp4_fake_quant(x)" if fp4
+                 else "conv3d_implicit_gemm(quant_act) + fp4_fake_quant(x)"),
         "l2": (f"x+w+y = {set_mib:.0f} MiB per input set; the GPU arm rotates {n_sets} sets "
                f"({n_sets * set_mib:.0f} MiB > 126 MiB L2)"),
         "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -234,6 +235,10 @@ def make_sets(wl, dev, seed, with_fq: bool):
 
 
 def conv_call(api, wl, s, stream):
+    if "wq" in s:   # the true-FP4 convolution over weights packed beforehand
+        api.conv3d_implicit_gemm_fp4(s["x"], s["wq"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
+                                     out=s["out"], stream=stream)
+        return
     api.conv3d_implicit_gemm(s["x"], s["w"], s["bias"], wl.stride, pad6(wl), wl.dil, s["act_amax"],
                              wl.quant_act, out=s["out"], stream=stream)
 
@@ -329,6 +334,10 @@ def run_ours(args, world, rank, local):
     # independent seeded input per rank; rotate copies so the working set exceeds L2
     sets = make_sets(wl, dev, wl.seed + 1000 * rank, True)
     n_sets = len(sets)
+    fp4 = args.conv == "fp4"
+    if fp4:   # weights packed once per set, before the timed region
+        for s_ in sets:
+            s_["wq"] = api.conv3d_fp4_pack_weights(s_["w"], api.act_amax(s_["w"], stream=stream), stream=stream)
     base = sets[0]
 
     def step(s):
@@ -382,13 +391,17 @@ def run_ours(args, world, rank, local):
 
     # every workload's convolution alone (outside the step's timed region)
     layers, layers_fp4, layer_clocks = (None, None, None)
+    if fp4:
+        for s_ in sets:
+            del s_["wq"]
     if not args.no_layers:
         layers, layers_fp4, layer_clocks = run_layers(api, args, stream, dev, peak, sets, wl.name, rank)
 
     # end-to-end through the public API with pinned host buffers
-    e2e = None if args.no_e2e else run_e2e(args, wl, base, stream, dev, world)
+    e2e = None if (args.no_e2e or fp4) else run_e2e(args, wl, base, stream, dev, world)
 
     conv_tflops = wl.flops / (conv_ms * 1e-3) / 1e12
+    conv_peak = peak * (FP4_OVER_BF16 if fp4 else 1.0)
     launches_per_step = 2 + (0 if (wl.dtype == torch.bfloat16 and wl.k_gemm % 8 == 0) else 1)
     fq_bytes = 2 * x_bytes  # read x, write the fake-quantised copy
     result = {
@@ -402,16 +415,19 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[wl.dtype] + "->bf16 mma, f32 acc",
+        "dtype": {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32"}[wl.dtype]
+                 + ("->nvfp4 mma (kind::mxf4nvf4), f32 acc" if fp4 else "->bf16 mma, f32 acc"),
         "data": "synthetic (seeded N(0,1) activations, N(0,1/sqrt(K)) weights)",
-        "config": workload_config(wl, world),
+        "config": workload_config(wl, world, fp4),
         "layer_us": round(conv_ms * 1e3, 2),
         "fake_quant_us": round(fq_ms * 1e3, 2),
-        "layer_frac_of_peak": round(conv_tflops / peak, 4),
+        "layer_frac_of_peak": round(conv_tflops / conv_peak, 4),
         "roofline": {
-            "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(conv_tflops / peak, 4), "traffic": profiled_traffic(wl.name),
-            "kernel": "conv3d_igemm_tmem (dominant)", "peak_source": f"{peaks_src} bf16_tflops (burst)",
+            "bound": "tensor", "achieved": round(conv_tflops, 2), "peak": round(conv_peak, 1), "unit": "TFLOP/s",
+            "frac": round(conv_tflops / conv_peak, 4), "traffic": None if fp4 else profiled_traffic(wl.name),
+            "kernel": "conv3d_igemm_tmem, NVFP4 operands (dominant)" if fp4 else "conv3d_igemm_tmem (dominant)",
+            "peak_source": (f"{peaks_src} bf16_tflops (burst) x {FP4_OVER_BF16:g} (nominal FP4:BF16 dense ratio)"
+                            if fp4 else f"{peaks_src} bf16_tflops (burst)"),
         },
         "fake_quant": {
             "us": round(fq_ms * 1e3, 2), "bytes": fq_bytes, "bound": "hbm",
@@ -508,15 +524,20 @@ def run_e2e(args, wl, base, stream, dev, world):
 # CPU oracle timing (test infrastructure: the only place bench.py runs it)
 # ---------------------------------------------------------------------------
 
-def oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng):
+def oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng, w_amax=None):
     """One scaled-down step on the host cores: `rows` random output rows (all
     Cout) of the convolution and the same fraction rows / M of the
-    fake-quant elements (whole blocks).  Returns (conv s, fake-quant s,
+    fake-quant elements (whole blocks).  With w_amax, the convolution is the
+    true-FP4 one (both operands NVFP4).  Returns (conv s, fake-quant s,
     fraction of the step done)."""
     import oracle
     ms = rng.integers(0, wl.m_gemm, rows)
     t = time.perf_counter()
-    oracle.conv3d(x_np, w_np, b_np, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act, amax, m_list=ms)
+    if w_amax is not None:
+        oracle.conv3d_nvfp4(x_np, w_np, b_np, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, act_amax=amax, w_amax=w_amax,
+                            m_list=ms)
+    else:
+        oracle.conv3d(x_np, w_np, b_np, wl.stride, wl.pad_lo, wl.pad_hi, wl.dil, wl.quant_act, amax, m_list=ms)
     t_conv = time.perf_counter() - t
     frac = rows / wl.m_gemm
     fq_elems = max(16, int(round(x_np.size * frac / 16)) * 16)
@@ -561,14 +582,16 @@ def run_reference(args, world, rank, local):
     w_np = base["w"].float().numpy()
     b_np = None if base["bias"] is None else base["bias"].float().numpy()
     amax = float(base["act_amax"].item())
+    fp4 = args.conv == "fp4"
+    w_amax = float(np.abs(w_np).max()) if fp4 else None
     rng = np.random.default_rng(99)
     rows = _rows_for(wl, x_np, w_np, b_np, amax, rng, 1.0)   # about 1 s of work per step
     for _ in range(args.warmup):
-        oracle_sample_step(wl, x_np, w_np, b_np, amax, max(8, rows // 8), rng)
+        oracle_sample_step(wl, x_np, w_np, b_np, amax, max(8, rows // 8), rng, w_amax)
     tot = 0.0
     frac = rows / wl.m_gemm
     for _ in range(args.steps):
-        tc, tf, frac = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng)
+        tc, tf, frac = oracle_sample_step(wl, x_np, w_np, b_np, amax, rows, rng, w_amax)
         tot += tc + tf
     step_s = tot / args.steps
     value = frac * wl.flops / step_s / 1e12
@@ -580,7 +603,7 @@ def run_reference(args, world, rank, local):
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 accumulate over bf16/fp4 operands (CPU oracle)", "data": "synthetic",
-        "config": workload_config(wl, world),
+        "config": workload_config(wl, world, fp4),
         "sample_fraction": frac,
         "full_layer_ms_estimate": step_s / frac * 1e3,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -626,6 +649,8 @@ def main(argv=None):
     ap.add_argument("--no-layers", action="store_true", help="skip the per-workload convolution timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end timing with host copies")
     ap.add_argument("--no-fp4", action="store_true", help="skip the true-FP4 convolution timings")
+    ap.add_argument("--conv", default="bf16", choices=["bf16", "fp4"],
+                    help="the step's convolution: the fake-quantised BF16 path (default) or the true-FP4 variant")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -78,8 +78,9 @@ Q3D_API q3d_status q3d_plan_conv_fp4(const int64_t x_shape[5], const int64_t w_s
  * of the convolution path.  Enqueues conv3d_implicit_gemm_pad2 (no bias, no
  * quantisation) on the tensor-memory kernel, except that in CTA 0 one of the
  * four epilogue warps withholds its arrival on the first hand-back of
- * accumulator 0: the MMA issuer's wait for that accumulator at CTA 0's second
- * tile never completes, nor do the waits that depend on it (the transform
+ * accumulator 0: the MMA issuer's wait for that accumulator when CTA 0 next
+ * uses it (its second tile, or its third where the plan double-buffers the
+ * accumulators) never completes, nor do the waits that depend on it (the transform
  * warps' waits for a free A stage, the producers' for a free stage or slot,
  * the epilogue's for the next accumulator).  The first of them to reach the
  * library's wait limit (2 s) gives up, sets its site bit in the device error
@@ -90,8 +91,9 @@ Q3D_API q3d_status q3d_plan_conv_fp4(const int64_t x_shape[5], const int64_t w_s
  * q3d_check_device_error returns Q3D_ERR_DEVICE_TIMEOUT with the site bits
  * and clears them; later calls are unaffected.
  *   x, w  BF16, contiguous, K % 8 == 0, w 16-byte aligned; the problem must
- *         run on the tensor-memory kernel with more tiles than CTAs
- *         (Q3D_ERR_INVALID_ARG otherwise, nothing enqueued).
+ *         run on the tensor-memory kernel with more tiles than CTAs times
+ *         accumulator buffers (Q3D_ERR_INVALID_ARG otherwise, nothing
+ *         enqueued).
  */
 Q3D_API q3d_status q3d_selftest_withheld_arrive(const q3d_tensor* x, const q3d_tensor* w, const int32_t stride[3],
                                                 const int32_t pad_lo[3], const int32_t pad_hi[3],

@@ -15,7 +15,7 @@
 // has no E4M3 representation relative to g and contributes zero.
 //
 // This file holds the weight packing kernel and the launcher; the kernel
-// template (its kFp4 instantiation) is in conv3d_tmem_kernel.cuh.
+// template (its NVFP4-operand instantiation) is in conv3d_tmem_kernel.cuh.
 #include "conv3d_tmem_kernel.cuh"
 
 namespace q3d {
@@ -103,7 +103,7 @@ cudaError_t launch_fp4_pack_weights(const void* w, int dtype, int32_t Cout, int3
 bool plan_conv3d_fp4(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   TmemParams p{};
   size_t smem = 0;
-  const bool ok = plan_tmem(g, dtype, p, smem, true);
+  const bool ok = plan_tmem(g, dtype, p, smem, kAOpNvfp4);
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.sf_col0,
@@ -120,7 +120,7 @@ cudaError_t launch_conv3d_fp4(const ConvGeom& g, const ConvLaunch& L, const void
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   TmemParams p{};
   size_t smem = 0;
-  if (!plan_tmem(g, L.dtype, p, smem, true)) return cudaSuccess;
+  if (!plan_tmem(g, L.dtype, p, smem, kAOpNvfp4)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = 1;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;
   p.g_w = static_cast<const float*>(packed);
@@ -132,9 +132,9 @@ cudaError_t launch_conv3d_fp4(const ConvGeom& g, const ConvLaunch& L, const void
   const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, L.sm_count));
   *handled = true;
   switch (L.dtype) {
-    case 0: return launch_tmem_typed<float, true>(p, tmap_x, tmap_w, grid, smem, s);
-    case 1: return launch_tmem_typed<__half, true>(p, tmap_x, tmap_w, grid, smem, s);
-    default: return launch_tmem_typed<__nv_bfloat16, true>(p, tmap_x, tmap_w, grid, smem, s);
+    case 0: return launch_tmem_typed<float, kAOpNvfp4>(p, tmap_x, tmap_w, grid, smem, s);
+    case 1: return launch_tmem_typed<__half, kAOpNvfp4>(p, tmap_x, tmap_w, grid, smem, s);
+    default: return launch_tmem_typed<__nv_bfloat16, kAOpNvfp4>(p, tmap_x, tmap_w, grid, smem, s);
   }
 }
 

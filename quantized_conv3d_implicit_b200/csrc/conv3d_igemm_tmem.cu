@@ -27,6 +27,17 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   TmemParams p{};
   size_t smem = 0;
   if (!plan_tmem(g, L.dtype, p, smem)) return cudaSuccess;
+  {
+    // A in shared memory frees tensor memory for more subtiles per tile or a
+    // second accumulator buffer; take that plan when it gains either
+    TmemParams q{};
+    size_t qsmem = 0;
+    if (plan_tmem(g, L.dtype, q, qsmem, kAOpBf16Smem) &&
+        (q.n_mt > p.n_mt || (q.n_mt == p.n_mt && q.acc_bufs > p.acc_bufs))) {
+      p = q;
+      smem = qsmem;
+    }
+  }
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;
 
@@ -47,15 +58,20 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   }
   const int64_t grid64 = std::min<int64_t>(p.num_tiles, L.sm_count);
   if (L.withhold_arrive) {
-    // the withheld hand-back is only waited for when CTA 0 has a second tile
-    if (p.num_tiles <= grid64) { *why = "the bounded-wait test needs more tiles than CTAs"; return cudaErrorInvalidValue; }
+    // the withheld hand-back is only waited for when CTA 0 reuses accumulator
+    // buffer 0, at its tile acc_bufs (counting from 0)
+    if (p.num_tiles <= static_cast<int64_t>(p.acc_bufs) * grid64) {
+      *why = "the bounded-wait test needs more tiles per CTA than accumulator buffers";
+      return cudaErrorInvalidValue;
+    }
     p.withhold_arrive = 1;
   }
   *handled = true;
+  if (p.aop == kAOpBf16Smem) return launch_tmem_smem_a(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
   switch (L.dtype) {
-    case 0: return launch_tmem_typed<float, false>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
-    case 1: return launch_tmem_typed<__half, false>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
-    default: return launch_tmem_typed<__nv_bfloat16, false>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+    case 0: return launch_tmem_typed<float, kAOpBf16Tmem>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+    case 1: return launch_tmem_typed<__half, kAOpBf16Tmem>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
+    default: return launch_tmem_typed<__nv_bfloat16, kAOpBf16Tmem>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
   }
 }
 

@@ -54,22 +54,8 @@
 
 namespace q3d {
 
-namespace {
-
-
-constexpr int kThreads = 768;
-constexpr int kWarpB = 0;
-constexpr int kWarpMma = 1;
-constexpr int kWarpHalo = 2;
-constexpr int kWarpEpi0 = 4;
-constexpr int kWarpXf0 = 8;
-constexpr int kNumXfWarps = 16;
-constexpr int kBlockK = 64;
-constexpr int kMaxSmem = 232448;  // 227 KB dynamic shared memory per CTA
-constexpr int kMaxAcc = 8;
-constexpr int kMaxTaps = 343;     // 7x7x7
-constexpr uint32_t kTmemCols = 512;
-
+// Kernel parameters (external linkage, so the translation units that
+// instantiate the kernel can hand a plan to each other).
 struct TmemParams {
   ConvGeom g;
   const void* bias;
@@ -92,6 +78,8 @@ struct TmemParams {
   int sa, sb;
   uint32_t b_stage_bytes;
   int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
+  int acc_bufs;           // accumulator buffers (2: tile t + 1 accumulates while tile t drains)
+  int acc_cols;           // TMEM columns of one accumulator buffer (n_mt * n_tile)
   int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
@@ -104,6 +92,8 @@ struct TmemParams {
   // scale factors of both operands are copied into tensor memory, a region
   // per A stage
   int fp4;
+  int aop;                // A operand mode: 0 BF16 in tensor memory, 1 BF16 in shared memory, 2 NVFP4
+  int dtype_code;         // element type of x: 0 f32, 1 f16, 2 bf16
   uint32_t off_a, a_stage_bytes;
   uint32_t b_img_bytes;   // one N-part's image: sub_n rows x 32 bytes of codes, then n_atoms scale atoms
   int n_atoms;            // 512-byte scale-factor atoms per N-part (128 rows each)
@@ -112,6 +102,32 @@ struct TmemParams {
   const uint8_t* wq;      // the first image (slice 0, part 0)
   const float* g_w;       // global scale of the weights (device scalar)
 };
+
+// The BF16 kernel with A in shared memory (instantiated in its own
+// translation unit, conv3d_igemm_tmem_sa.cu).
+cudaError_t launch_tmem_smem_a(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
+                               size_t smem, cudaStream_t s);
+
+namespace {
+
+constexpr int kThreads = 768;
+constexpr int kWarpB = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpHalo = 2;
+constexpr int kWarpEpi0 = 4;
+constexpr int kWarpXf0 = 8;
+constexpr int kNumXfWarps = 16;
+constexpr int kBlockK = 64;
+constexpr int kMaxSmem = 232448;  // 227 KB dynamic shared memory per CTA
+constexpr int kMaxAcc = 16;     // accumulator barriers: buffers x subtiles x N-parts
+constexpr int kMaxTaps = 343;     // 7x7x7
+constexpr uint32_t kTmemCols = 512;
+// Where the transform warps put the A operand and in which format:
+//   BF16 values in tensor memory (tcgen05.st; the MMA reads A from TMEM);
+//   BF16 values in shared memory (128-byte-swizzled K-major, like B);
+//   NVFP4 codes and scale bytes in shared memory (block-scaled MMA).
+constexpr int kAOpBf16Tmem = 0, kAOpBf16Smem = 1, kAOpNvfp4 = 2;
+
 
 struct TileCoord {
   int n, od, oh0, ow0, nt;
@@ -673,7 +689,9 @@ struct MmaBars {
 // wait results are combined over the warp so all lanes take the same path.
 // NMT / NSUB fix the subtile and N-part counts at compile time (0: taken from
 // the plan), so the common shapes issue straight-line code.
-template <int NMT, int NSUB>
+// kSmemA: A is a 128B-swizzled K-major tile in shared memory (16 KB per
+// subtile), read through a descriptor like B; otherwise A is in TMEM.
+template <int NMT, int NSUB, bool kSmemA = false>
 __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t base, uint32_t tmem_base,
                                                const MmaBars& b, volatile int* abort_flag) {
   const int n_mt = NMT ? NMT : p.n_mt;
@@ -686,6 +704,10 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
   RingPos ap{0u, 0u}, bp{0u, 0u};
   bool ok = true;
   for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+    // accumulator buffer of this tile and how many tiles used it before
+    const uint32_t buf = p.acc_bufs == 2 ? (it & 1u) : 0u, use = p.acc_bufs == 2 ? (it >> 1) : it;
+    const int abase = static_cast<int>(buf) * n_mt * n_sub;
+    const uint32_t acc_base = tmem_base + buf * static_cast<uint32_t>(p.acc_cols);
     for (int s = 0; ok && s < p.ks; ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
       const uint32_t ea = ap.e, eb = bp.e;
       ok = wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) &&
@@ -695,7 +717,8 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
         break;
       }
       tc_fence_after();
-      const uint32_t a_stage = tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(n_mt * 32);
+      const uint32_t a_stage = kSmemA ? base + p.off_a + ea * p.a_stage_bytes
+                                      : tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(n_mt * 32);
       const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
       const bool first = (s == 0), last = (s == p.ks - 1);
 #pragma unroll
@@ -704,20 +727,30 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
 #pragma unroll
         for (int ns = 0; ns < (NSUB ? NSUB : 2); ++ns) {
           if (!NSUB && ns >= n_sub) break;
-          const int acc = i * n_sub + ns;
-          if (first && it > 0 && ok) {
+          const int acc = abase + i * n_sub + ns;
+          if (first && use > 0 && ok) {
             ok = __all_sync(0xffffffffu,
-                            wait_or_abort(b.acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag));
+                            wait_or_abort(b.acc_empty + 8u * acc, (use - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag));
             tc_fence_after();
           }
           if (ok) {
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i) * tile_cols + static_cast<uint32_t>(ns) * sub_cols;
-            const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
+            const uint32_t d_tmem =
+                acc_base + static_cast<uint32_t>(i) * tile_cols + static_cast<uint32_t>(ns) * sub_cols;
             const uint64_t bsub = bdesc + static_cast<uint64_t>(ns) * bsub_step;
+            if constexpr (kSmemA) {
+              // K advances 32 bytes (16 BF16) inside the 128-byte swizzle atom
+              const uint64_t asub = umma_desc_kmajor_sw128(a_stage + static_cast<uint32_t>(i) * 16384u);
 #pragma unroll
-            for (int j = 0; j < kBlockK / 16; ++j)
-              umma_bf16_ts_elect(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
-                                 (first && j == 0) ? 0u : 1u);
+              for (int j = 0; j < kBlockK / 16; ++j)
+                umma_bf16_ss_elect(d_tmem, asub + static_cast<uint64_t>(2 * j), bsub + static_cast<uint64_t>(2 * j),
+                                   idesc, (first && j == 0) ? 0u : 1u);
+            } else {
+              const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
+#pragma unroll
+              for (int j = 0; j < kBlockK / 16; ++j)
+                umma_bf16_ts_elect(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
+                                   (first && j == 0) ? 0u : 1u);
+            }
             if (last) umma_commit_elect(b.acc_full + 8u * acc);
           }
         }
@@ -754,6 +787,10 @@ __device__ __forceinline__ void mma_issue_loop_fp4(const TmemParams& p, uint32_t
   RingPos ap{0u, 0u}, bp{0u, 0u};
   bool ok = true;
   for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
+    // accumulator buffer of this tile and how many tiles used it before
+    const uint32_t buf = p.acc_bufs == 2 ? (it & 1u) : 0u, use = p.acc_bufs == 2 ? (it >> 1) : it;
+    const int abase = static_cast<int>(buf) * n_mt * n_sub;
+    const uint32_t acc_base = tmem_base + buf * static_cast<uint32_t>(p.acc_cols);
     for (int s = 0; ok && s < p.ks; ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
       const uint32_t ea = ap.e, eb = bp.e;
       ok = wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) &&
@@ -783,14 +820,15 @@ __device__ __forceinline__ void mma_issue_loop_fp4(const TmemParams& p, uint32_t
 #pragma unroll
         for (int ns = 0; ns < (NSUB ? NSUB : 2); ++ns) {
           if (!NSUB && ns >= n_sub) break;
-          const int acc = i * n_sub + ns;
-          if (first && it > 0 && ok) {
+          const int acc = abase + i * n_sub + ns;
+          if (first && use > 0 && ok) {
             ok = __all_sync(0xffffffffu,
-                            wait_or_abort(b.acc_empty + 8u * acc, (it - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag));
+                            wait_or_abort(b.acc_empty + 8u * acc, (use - 1u) & 1u, p.err, kSiteAccEmpty, abort_flag));
             tc_fence_after();
           }
           if (ok) {
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(i) * tile_cols + static_cast<uint32_t>(ns) * sub_cols;
+            const uint32_t d_tmem =
+                acc_base + static_cast<uint32_t>(i) * tile_cols + static_cast<uint32_t>(ns) * sub_cols;
             umma_nvfp4_ss_elect(d_tmem, umma_desc_kmajor_sw32(a_st + 4096u * i),
                                 umma_desc_kmajor_sw32(b_st + ns * p.b_img_bytes), idesc, sfa + 4u * i,
                                 sfb + 4u * static_cast<uint32_t>(ns * p.n_atoms), first ? 0u : 1u);
@@ -817,10 +855,12 @@ __device__ __forceinline__ void mma_issue_loop_fp4(const TmemParams& p, uint32_t
 // NVFP4-operand variant (A as E2M1 codes and scale bytes in shared memory,
 // prepacked NVFP4 weights, block-scaled MMA, the two global scales applied
 // in the epilogue); otherwise BF16 operands with A in tensor memory.
-template <typename T, bool kPairs, int kDWB, bool kFp4>
+template <typename T, bool kPairs, int kDWB, int kAOp>
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
                              const __grid_constant__ CUtensorMap tmap_w) {
+  constexpr bool kFp4 = kAOp == kAOpNvfp4;
+  constexpr bool kSmemA = kAOp != kAOpBf16Tmem;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -944,11 +984,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         switch (p.n_mt * 4 + p.n_sub) {  // straight-line issue for the common shapes
-          case 1 * 4 + 1: mma_issue_loop<1, 1>(p, base, tb, bars, abort_flag); break;
-          case 1 * 4 + 2: mma_issue_loop<1, 2>(p, base, tb, bars, abort_flag); break;
-          case 2 * 4 + 1: mma_issue_loop<2, 1>(p, base, tb, bars, abort_flag); break;
-          case 2 * 4 + 2: mma_issue_loop<2, 2>(p, base, tb, bars, abort_flag); break;
-          default: mma_issue_loop<0, 0>(p, base, tb, bars, abort_flag); break;
+          case 1 * 4 + 1: mma_issue_loop<1, 1, kSmemA>(p, base, tb, bars, abort_flag); break;
+          case 1 * 4 + 2: mma_issue_loop<1, 2, kSmemA>(p, base, tb, bars, abort_flag); break;
+          case 2 * 4 + 1: mma_issue_loop<2, 1, kSmemA>(p, base, tb, bars, abort_flag); break;
+          case 2 * 4 + 2: mma_issue_loop<2, 2, kSmemA>(p, base, tb, bars, abort_flag); break;
+          case 4 * 4 + 1: mma_issue_loop<4, 1, kSmemA>(p, base, tb, bars, abort_flag); break;
+          default: mma_issue_loop<0, 0, kSmemA>(p, base, tb, bars, abort_flag); break;
         }
       }
       __syncwarp();
@@ -991,6 +1032,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int64_t t = blockIdx.x; ok && t < p.num_tiles; t += gridDim.x, ++it) {
       const TileCoord tc = decode_tile(p, t);
       const int ow = tc.ow0 + tw_u;
+      const uint32_t buf = p.acc_bufs == 2 ? (it & 1u) : 0u, use = p.acc_bufs == 2 ? (it >> 1) : it;
       for (int i = 0; ok && i < p.n_mt; ++i) {
         const int oh = tc.oh0 + i * p.TH + th_u;
         const bool row_ok = oh < g.OH && ow < g.OW;
@@ -998,15 +1040,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t ubase = (static_cast<int64_t>(tc.n) * g.Cout) * S + static_cast<int64_t>(tc.od) * S_hw +
                               static_cast<int64_t>(oh) * g.OW + ow;
         for (int ns = 0; ns < p.n_sub; ++ns) {
-          const int acc = i * p.n_sub + ns;
-          if (!wait_or_abort(bar_acc_full + 8u * acc, it & 1u, p.err, kSiteAccFull, abort_flag)) {
+          const int acc = static_cast<int>(buf) * p.n_mt * p.n_sub + i * p.n_sub + ns;
+          if (!wait_or_abort(bar_acc_full + 8u * acc, use & 1u, p.err, kSiteAccFull, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int co0 = tc.nt * p.n_tile + ns * p.sub_n;
-          const uint32_t taddr =
-              tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + buf * static_cast<uint32_t>(p.acc_cols) +
+                                 static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
           for (int c0 = 0; c0 < p.sub_n; c0 += 16) {
             uint32_t v[16];
             tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
@@ -1179,6 +1221,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t a_code_off =
         static_cast<uint32_t>(row * 32 + ((((b0 >> 1) ^ (row >> 2)) & 1) << 4));
     const uint32_t a_sf_off = static_cast<uint32_t>(p.n_mt * 4096 + lane * 16 + quad * 4 + b0);
+    // BF16 A in shared memory: this thread's row (128 bytes) of a subtile's
+    // 128B-swizzled tile and the swizzled 16-byte chunks of its two blocks
+    // (block b0 + bb holds K columns 16 (b0 + bb) .. +15: chunks 2 (b0 + bb)
+    // and 2 (b0 + bb) + 1, chunk j stored at j ^ (row & 7))
+    const uint32_t a_row16 = static_cast<uint32_t>(row) * 128u;
+    const uint32_t sw7 = static_cast<uint32_t>(row & 7);
+    const uint32_t ach0 = ((2u * b0) ^ sw7) << 4, ach1 = ((2u * b0 + 1u) ^ sw7) << 4;
+    const uint32_t ach2 = ((2u * b0 + 2u) ^ sw7) << 4, ach3 = ((2u * b0 + 3u) ^ sw7) << 4;
     const uint32_t ring = static_cast<uint32_t>(p.ring);
     const int cb = static_cast<int>(p.chan_bytes);
     uint32_t gs_base = 0;                 // global halo slot counter at the start of the tile
@@ -1245,6 +1295,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         // 4096 bytes further for the codes, 512 for the scale bytes)
         const uint32_t a_stage = base + p.off_a + ea * p.a_stage_bytes;
         const uint32_t a_code = a_stage + a_code_off, a_sf = a_stage + a_sf_off;
+        // the 16 BF16 values of block b0 + bb of subtile i, into TMEM or the
+        // shared-memory tile
+        auto put = [&](int i, int bb, const uint32_t (&w)[8]) {
+          if constexpr (kSmemA) {
+            const uint32_t r = a_stage + static_cast<uint32_t>(i) * 16384u + a_row16;
+            st_shared_v4(r + (bb ? ach2 : ach0), w[0], w[1], w[2], w[3]);
+            st_shared_v4(r + (bb ? ach3 : ach1), w[4], w[5], w[6], w[7]);
+          } else {
+            tmem_st8(a_col + 8u * static_cast<uint32_t>(bb) + static_cast<uint32_t>(i * 32), w);
+          }
+        };
         const bool quant = p.quant != 0;
         bool pair_done = false;
         if constexpr (!kPairs && sizeof(T) == 2) {
@@ -1279,8 +1340,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               uint32_t wa[8], wb[8];
               quant8_x2<T>(pa, pb, quant, q, wa, wb);
-              tmem_st8(a_col, wa);
-              tmem_st8(a_col + 8u, wb);
+              put(0, 0, wa);
+              put(0, 1, wb);
             }
             pair_done = true;
           }
@@ -1288,7 +1349,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int bb = 0; bb < 2 && !pair_done; ++bb) {
           const int nv = bb ? nv1 : nv0;
-          const uint32_t colb = a_col + 8u * static_cast<uint32_t>(bb);
           const uint32_t codeb = a_code + 8u * static_cast<uint32_t>(bb), sfb = a_sf + static_cast<uint32_t>(bb);
           if (nv <= 0) {
             // a block entirely past K: zeros (the weights there are zero-filled too)
@@ -1297,7 +1357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fp4_put(codeb + static_cast<uint32_t>(i) * 4096u, sfb + static_cast<uint32_t>(i) * 512u, 0u, 0u, 0u);
             } else {
               uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-              for (int i = 0; i < p.n_mt; ++i) tmem_st8(colb + static_cast<uint32_t>(i * 32), z);
+              for (int i = 0; i < p.n_mt; ++i) put(i, bb, z);
             }
             continue;
           }
@@ -1342,8 +1402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             cb1, sb8);
                   } else {
                     quant8_x2<T>(pa, pb, quant, q, wa, wb);
-                    tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
-                    tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
+                    put(i, bb, wa);
+                    put(i + 1, bb, wb);
                   }
                 }
               }
@@ -1362,7 +1422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   fp4_put(codeb + static_cast<uint32_t>(i) * 4096u, sfb + static_cast<uint32_t>(i) * 512u, c0, c1, s8b);
                 } else {
                   quant8_1<T>(pa, quant, q, wa);
-                  tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
+                  put(i, bb, wa);
                 }
               }
               continue;
@@ -1394,8 +1454,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           sb8);
                 } else {
                   quant8_x2<T>(pa, pb, quant, q, wa, wb);
-                  tmem_st8(colb + static_cast<uint32_t>(i * 32), wa);
-                  tmem_st8(colb + static_cast<uint32_t>((i + 1) * 32), wb);
+                  put(i, bb, wa);
+                  put(i + 1, bb, wb);
                 }
               }
           }
@@ -1407,11 +1467,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               uint32_t w[8];
               row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, quant, q, w);
-              tmem_st8(colb + static_cast<uint32_t>(i * 32), w);
+              put(i, bb, w);
             }
           }
         }
-        if constexpr (kFp4) {
+        if constexpr (kSmemA) {
           // the MMA reads the stage through the async proxy
           fence_proxy_async_smem();
         } else {
@@ -1478,10 +1538,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, bool kPairs, int kDWB, bool kFp4>
+template <typename T, bool kPairs, int kDWB, int kAOp>
 cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid, size_t smem,
                              cudaStream_t s) {
-  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB, kFp4>;
+  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB, kAOp>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
@@ -1490,21 +1550,21 @@ cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const C
 
 // Row gather for 16-bit inputs and kernels three taps wide with W dilation 1
 // or 2; tap-offset gather otherwise.
-template <typename T, bool kFp4>
+template <typename T, int kAOp>
 cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                               size_t smem, cudaStream_t s) {
   const int dwb = row_gather_step(p.g, sizeof(T));
   const bool pairs = p.n_mt >= 2;
   if constexpr (sizeof(T) == 2) {
     if (dwb == 2)
-      return pairs ? launch_tmem_inst<T, true, 2, kFp4>(p, tx, tw, grid, smem, s)
-                   : launch_tmem_inst<T, false, 2, kFp4>(p, tx, tw, grid, smem, s);
+      return pairs ? launch_tmem_inst<T, true, 2, kAOp>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 2, kAOp>(p, tx, tw, grid, smem, s);
     if (dwb == 4)
-      return pairs ? launch_tmem_inst<T, true, 4, kFp4>(p, tx, tw, grid, smem, s)
-                   : launch_tmem_inst<T, false, 4, kFp4>(p, tx, tw, grid, smem, s);
+      return pairs ? launch_tmem_inst<T, true, 4, kAOp>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 4, kAOp>(p, tx, tw, grid, smem, s);
   }
-  return pairs ? launch_tmem_inst<T, true, 0, kFp4>(p, tx, tw, grid, smem, s)
-               : launch_tmem_inst<T, false, 0, kFp4>(p, tx, tw, grid, smem, s);
+  return pairs ? launch_tmem_inst<T, true, 0, kAOp>(p, tx, tw, grid, smem, s)
+               : launch_tmem_inst<T, false, 0, kAOp>(p, tx, tw, grid, smem, s);
 }
 
 // Output channels per tile: all of Cout up to 448 (448 + two 32-column A
@@ -1555,12 +1615,15 @@ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 // a multiple of 16 bytes (TMA stride rule), more than 343 taps, or no plan
 // that fits.
 //
-// fp4: the NVFP4-operand variant.  Its A stages live in shared memory
-// (n_mt x (4096 bytes of codes + a 512-byte scale atom)), its weight stages
-// hold n_sub prepacked images, and tensor memory holds the accumulators and
-// per A stage the scale factors (4 columns per subtile and per 128 rows of
-// an N-part).
-bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool fp4 = false) {
+// aop: the A operand mode.  kAOpBf16Tmem: A stages of n_mt x 32 columns in
+// tensor memory beside the accumulators.  kAOpBf16Smem: A stages of n_mt x
+// 16 KB in shared memory, tensor memory only for the accumulators.
+// kAOpNvfp4: A stages of n_mt x (4096 bytes of codes + a 512-byte scale
+// atom) in shared memory, weight stages of n_sub prepacked images, and in
+// tensor memory the accumulators and per A stage the scale factors (4
+// columns per subtile and per 128 rows of an N-part).
+bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int aop = kAOpBf16Tmem) {
+  const bool fp4 = aop == kAOpNvfp4, smem_a = aop != kAOpBf16Tmem;
   const int esz = dtype == 0 ? 4 : 2;
   const int align = 16 / esz;
   if ((static_cast<int64_t>(g.W) * esz) % 16 != 0) return false;
@@ -1573,14 +1636,20 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
   const int n_tile = np.n_tile, n_ntiles = np.n_ntiles, n_sub = np.n_sub, sub_n = np.sub_n;
   p.n_tile = n_tile; p.n_ntiles = n_ntiles; p.n_sub = n_sub; p.sub_n = sub_n;
   p.fp4 = fp4 ? 1 : 0;
+  p.aop = aop;
+  p.dtype_code = dtype;
   p.n_atoms = (sub_n + 127) / 128;
   p.n_parts = n_ntiles * n_sub;
   p.b_img_bytes = static_cast<uint32_t>(sub_n * 32 + p.n_atoms * 512);
   // TMEM columns after the accumulators (32-aligned), and what one A stage
   // takes there: 32 BF16-pair columns per subtile, or (fp4) the scale factors
-  auto a_col0_of = [&](int mt) { return (mt * n_tile + 31) / 32 * 32; };
-  auto stage_cols = [&](int mt) { return fp4 ? 4 * mt + 4 * p.n_atoms * n_sub : mt * 32; };
-  auto stages_of = [&](int mt) { return (static_cast<int>(kTmemCols) - a_col0_of(mt)) / stage_cols(mt); };
+  auto a_col0_of = [&](int mt, int nb = 1) { return (nb * mt * n_tile + 31) / 32 * 32; };
+  auto stage_cols = [&](int mt) { return fp4 ? 4 * mt + 4 * p.n_atoms * n_sub : smem_a ? 0 : mt * 32; };
+  auto stages_of = [&](int mt, int nb = 1) {
+    const int left = static_cast<int>(kTmemCols) - a_col0_of(mt, nb);
+    if (left < 0) return 0;
+    return stage_cols(mt) == 0 ? 4 : left / stage_cols(mt);
+  };
 
   // tile shape: subtile TH x TW = 128, n_mt subtiles stacked along oh; at
   // least two A stages must fit next to the accumulators
@@ -1588,7 +1657,10 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
   double best = 1e30;
   int bTW = 0, bMT = 0;
   for (int mt = 4; mt >= 1; mt /= 2) {
-    if (mt * n_sub > kMaxAcc || stages_of(mt) < 2) continue;
+    if (2 * mt * n_sub > kMaxAcc || stages_of(mt) < 2) continue;
+    // measured on the 96-channel edge layer with W dilation 2 (NVFP4
+    // operands): four subtiles 14.2 ms, two 11.3 ms (undilated: 7.6 vs 9.6)
+    if (fp4 && g.dw > 1 && mt > 2) continue;
     for (int TW = 128; TW >= 8; TW /= 2) {
       const int TH = 128 / TW, rows = TH * mt;
       const int h_ext = (rows - 1) * g.sh + (g.KH - 1) * g.dh + 1;
@@ -1604,11 +1676,17 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
   }
   if (bTW == 0) return false;
   p.TW = bTW; p.TH = 128 / bTW; p.n_mt = bMT;
-  p.a_col0 = fp4 ? 0 : a_col0_of(bMT);
-  p.sf_col0 = fp4 ? a_col0_of(bMT) : 0;
+  // two accumulator buffers where two A stages still fit beside them: the
+  // MMAs of the next tile then overlap the epilogue's drain of this one
+  p.acc_bufs = stages_of(bMT, 2) >= 2 ? 2 : 1;
+  p.acc_cols = bMT * n_tile;
+  p.a_col0 = smem_a ? 0 : a_col0_of(bMT, p.acc_bufs);
+  p.sf_col0 = fp4 ? a_col0_of(bMT, p.acc_bufs) : 0;
   p.sf_cols = fp4 ? stage_cols(bMT) : 0;
-  p.a_stage_bytes = fp4 ? static_cast<uint32_t>((bMT * (4096 + 512) + 1023) / 1024 * 1024) : 0u;
-  p.sa = std::min(4, stages_of(bMT));
+  p.a_stage_bytes = fp4      ? static_cast<uint32_t>((bMT * (4096 + 512) + 1023) / 1024 * 1024)
+                    : smem_a ? static_cast<uint32_t>(bMT) * 16384u
+                             : 0u;
+  p.sa = std::min(4, stages_of(bMT, p.acc_bufs));
   p.n_owb = ceil_div(g.OW, p.TW);
   p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
   p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;
@@ -1656,7 +1734,7 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
     p.slot_tx = static_cast<uint32_t>(p.c_slot) * p.chan_bytes;
     p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
     // fewer A stages shrink the halo window the ring must cover
-    const int sa_max = std::min(4, stages_of(bMT));
+    const int sa_max = std::min(4, stages_of(bMT, p.acc_bufs));
     for (int a = sa_max; a >= 2; --a) {
       int span = 1;
       for (int s0 = 0; s0 < p.ks; ++s0) {
@@ -1667,7 +1745,7 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
       for (int b = 8; b >= 2; --b) {
         int r = span + 2;
         const int nbar = 2 * r + 2 * b + 2 * a + 2 * kMaxAcc + 1;
-        const int a_bytes = a * static_cast<int>(p.a_stage_bytes);  // fp4 only
+        const int a_bytes = a * static_cast<int>(p.a_stage_bytes);  // A stages in shared memory only
         int total = 1024 + kDqTableBytes + b * static_cast<int>(p.b_stage_bytes) + a_bytes +
                     r * static_cast<int>(p.slot_bytes) + 64 /* pad after the halo ring */ + code_bytes + epi_bytes +
                     phase_bytes + nbar * 8 + 16;
@@ -1680,7 +1758,7 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool f
           p.sa = a; p.sb = b; p.ring = r;
           p.off_dq = 0;
           p.off_b = kDqTableBytes;  // a multiple of 1024, as the swizzled weight stages need
-          p.off_a = p.off_b + b * p.b_stage_bytes;  // fp4: the swizzled A stages, 1024-aligned
+          p.off_a = p.off_b + b * p.b_stage_bytes;  // A stages in shared memory (1024-aligned)
           p.off_halo = p.off_a + static_cast<uint32_t>(a_bytes);
           p.off_code = (p.off_halo + r * p.slot_bytes + 64u + 15u) / 16u * 16u;
           p.off_epi = p.off_code + static_cast<uint32_t>(code_bytes);

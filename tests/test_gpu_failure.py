@@ -34,10 +34,12 @@ DOWNSTREAM = (1 << 0) | (1 << 3) | (1 << 4) | (1 << 5) | (1 << 7)
 def test_withheld_arrival_times_out_and_the_context_stays_usable(cuda_ok):
     lib = api.load_library()
     assert api.check_device_error() == 0                 # start from a clear word
-    xs, cout, k = (1, 16, 8, 128, 128), 32, (3, 3, 3)     # more tiles than CTAs (CTA 0 has a second)
+    # more tiles than CTAs times accumulator buffers: CTA 0 reuses accumulator
+    # buffer 0 (two buffers with this plan: CTA 0 has a third tile)
+    xs, cout, k = (1, 16, 16, 128, 128), 32, (3, 3, 3)
     plan = api.plan_conv(xs, (cout, 16) + k, 1, 1, 1, torch.bfloat16, kernel="tmem")
     assert plan["applicable"] == 1
-    assert xs[2] * plan["n_ohb"] * plan["n_owb"] * plan["n_ntiles"] > 148
+    assert xs[2] * plan["n_ohb"] * plan["n_owb"] * plan["n_ntiles"] > 2 * 148
     inp = workloads.random_conv_inputs(71, xs, cout, k, dtype=torch.bfloat16, bias=False, device="cuda")
     y = torch.empty(api.out_shape(xs, (cout, 16) + k, 1, 1, 1), dtype=torch.bfloat16, device="cuda")
     t0 = time.time()
