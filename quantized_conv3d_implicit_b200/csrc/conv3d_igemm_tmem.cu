@@ -28,12 +28,20 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   size_t smem = 0;
   if (!plan_tmem(g, L.dtype, p, smem)) return cudaSuccess;
   {
-    // A in shared memory frees tensor memory for more subtiles per tile or a
-    // second accumulator buffer; take that plan when it gains either
+    // A in shared memory frees tensor memory for more subtiles per tile, a
+    // second accumulator buffer or more A stages; take that plan when it
+    // gains any of them (measured: edge 96 channels 11.8 -> 10.7 ms with four
+    // subtiles, wan_hi 3.45 -> 3.27 ms with four A stages instead of two; the
+    // 384- and 1024-channel layers, which gain nothing, were 8 % slower with
+    // A in shared memory)
+    // (Q3D_KERNEL=smem_a takes it wherever it applies: the tests run every
+    // shape through this form too)
+    const char* kc = getenv("Q3D_KERNEL");
+    const bool force = kc && !strcmp(kc, "smem_a");
     TmemParams q{};
     size_t qsmem = 0;
     if (plan_tmem(g, L.dtype, q, qsmem, kAOpBf16Smem) &&
-        (q.n_mt > p.n_mt || (q.n_mt == p.n_mt && q.acc_bufs > p.acc_bufs))) {
+        (force || q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)))) {
       p = q;
       smem = qsmem;
     }

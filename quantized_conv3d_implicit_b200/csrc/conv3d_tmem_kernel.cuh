@@ -1658,9 +1658,10 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
   int bTW = 0, bMT = 0;
   for (int mt = 4; mt >= 1; mt /= 2) {
     if (2 * mt * n_sub > kMaxAcc || stages_of(mt) < 2) continue;
-    // measured on the 96-channel edge layer with W dilation 2 (NVFP4
-    // operands): four subtiles 14.2 ms, two 11.3 ms (undilated: 7.6 vs 9.6)
-    if (fp4 && g.dw > 1 && mt > 2) continue;
+    // measured on the 96-channel edge layer with W dilation 2: four subtiles
+    // 14.2 ms, two 11.3 ms with NVFP4 operands (undilated: 7.6 vs 9.6), and
+    // 12.3 vs 11.9 ms with BF16 ones
+    if (smem_a && g.dw > 1 && mt > 2) continue;
     for (int TW = 128; TW >= 8; TW /= 2) {
       const int TH = 128 / TW, rows = TH * mt;
       const int h_ext = (rows - 1) * g.sh + (g.KH - 1) * g.dh + 1;

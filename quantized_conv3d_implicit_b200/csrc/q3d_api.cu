@@ -225,7 +225,9 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
 // The convolution kernels proper, once the BF16 weights are in place: the
 // tensor-memory kernel where it applies, else the shared-memory specialised
 // kernel, else the general one.  Q3D_KERNEL=tmem|fast|basic starts the chain
-// at that kernel (all three compute the same result).
+// at that kernel, and Q3D_KERNEL=smem_a runs the tensor-memory kernel with
+// its A operand in shared memory wherever that form applies (all compute the
+// same result).
 cudaError_t launch_conv(const q3d::ConvGeom& g, const q3d::ConvLaunch& L, cudaStream_t s, const char** why) {
   const char* kc = getenv("Q3D_KERNEL");
   const int first = (kc && !strcmp(kc, "basic")) ? 2 : (kc && !strcmp(kc, "fast")) ? 1 : 0;

@@ -18,10 +18,11 @@ from _parity import assert_conv_close, bits, to_np_f32
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=["auto", "fast", "basic"])
+@pytest.fixture(params=["auto", "smem_a", "fast", "basic"])
 def kernel(request, monkeypatch):
     """Run a test with the library's default kernel choice (the tensor-memory
-    kernel where it applies), with the shared-memory specialised kernel
+    kernel where it applies), with the tensor-memory kernel's shared-memory A
+    form forced where it applies, with the shared-memory specialised kernel
     forced, and with the general-purpose kernel forced: all must meet the
     same bar."""
     if request.param == "auto":
