@@ -7,13 +7,35 @@
 
 namespace q3d {
 
+// The plan the launcher runs: A in tensor memory, or A in shared memory when
+// that frees tensor memory for more subtiles per tile, a second accumulator
+// buffer or more A stages (measured: edge 96 channels 11.8 -> 10.7 ms with
+// four subtiles, wan_hi 3.45 -> 3.27 ms with four A stages instead of two;
+// the 384- and 1024-channel layers, which gain nothing, were 8 % slower with
+// A in shared memory).  Q3D_KERNEL=smem_a takes the shared-memory form
+// wherever it applies (the tests run every shape through it too).
+static bool choose_plan(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem) {
+  if (!plan_tmem(g, dtype, p, smem)) return false;
+  const char* kc = getenv("Q3D_KERNEL");
+  const bool force = kc && !strcmp(kc, "smem_a");
+  TmemParams q{};
+  size_t qsmem = 0;
+  if (plan_tmem(g, dtype, q, qsmem, kAOpBf16Smem) &&
+      (force || q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)))) {
+    p = q;
+    smem = qsmem;
+  }
+  return true;
+}
+
 bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   TmemParams p{};
   size_t smem = 0;
-  const bool ok = plan_tmem(g, dtype, p, smem);
+  const bool ok = choose_plan(g, dtype, p, smem);
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
-                       static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0};
+                       static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0,
+                       p.aop, p.acc_bufs};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
   for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
   return ok;
@@ -26,26 +48,7 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   TmemParams p{};
   size_t smem = 0;
-  if (!plan_tmem(g, L.dtype, p, smem)) return cudaSuccess;
-  {
-    // A in shared memory frees tensor memory for more subtiles per tile, a
-    // second accumulator buffer or more A stages; take that plan when it
-    // gains any of them (measured: edge 96 channels 11.8 -> 10.7 ms with four
-    // subtiles, wan_hi 3.45 -> 3.27 ms with four A stages instead of two; the
-    // 384- and 1024-channel layers, which gain nothing, were 8 % slower with
-    // A in shared memory)
-    // (Q3D_KERNEL=smem_a takes it wherever it applies: the tests run every
-    // shape through this form too)
-    const char* kc = getenv("Q3D_KERNEL");
-    const bool force = kc && !strcmp(kc, "smem_a");
-    TmemParams q{};
-    size_t qsmem = 0;
-    if (plan_tmem(g, L.dtype, q, qsmem, kAOpBf16Smem) &&
-        (force || q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)))) {
-      p = q;
-      smem = qsmem;
-    }
-  }
+  if (!choose_plan(g, L.dtype, p, smem)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;
 

@@ -51,6 +51,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
 
     ks, q_slots, ring, sa, sb, G = (plan[k] for k in ("ks", "q_slots", "ring", "sa", "sb", "groups"))
     n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
+    nbuf = plan.get("acc_bufs", 1) or 1   # accumulator buffers (the tensor-memory kernel may have two)
     n_xf = 16 if kernel == "tmem" else 8   # transform warps; the tensor-memory kernel has one group
     wpg = n_xf // G
     # who hands halo slots back: the MMA thread (shared-memory kernel) or
@@ -102,11 +103,12 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                     yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
                     released += 1
                 yield ("wait", bar("b_full", eb, 1), gb // sb)
+                buf, use = it % nbuf, it // nbuf   # accumulator buffer of this unit, and its earlier uses
                 for i in range(n_mt):
                     for ns in range(n_sub):
-                        acc = i * n_sub + ns
-                        if s == k0 and it > 0:
-                            yield ("wait", bar("acc_empty", acc, 4), it - 1)
+                        acc = (buf * n_mt + i) * n_sub + ns
+                        if s == k0 and use > 0:
+                            yield ("wait", bar("acc_empty", acc, 4), use - 1)
                         if s == k1 - 1:
                             yield ("arrive", bar("acc_full", acc, 1))
                 yield ("arrive", bar("a_empty", ea, 1))
@@ -117,10 +119,11 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
 
     def epilogue():
         for it in range(len(us)):
+            buf, use = it % nbuf, it // nbuf
             for i in range(n_mt):
                 for ns in range(n_sub):
-                    acc = i * n_sub + ns
-                    yield ("wait", bar("acc_full", acc, 1), it)
+                    acc = (buf * n_mt + i) * n_sub + ns
+                    yield ("wait", bar("acc_full", acc, 1), use)
                     yield ("arrive", bar("acc_empty", acc, 4))
 
     def transform(w):
@@ -342,10 +345,16 @@ def _check_tmem_invariants(p, taps):
     if taps < 16:
         # a block spans several channels: slots must hold whole blocks
         assert (p["c_slot"] * taps) % 16 == 0
-    # accumulators [0, n_mt*n_tile), then sa A stages of n_mt * 32 columns
-    assert p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
-    assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512 and p["sa"] >= 2
-    assert p["n_mt"] * p["n_sub"] <= 8
+    nb = p["acc_bufs"]
+    assert nb in (1, 2) and p["aop"] in (0, 1) and p["sa"] >= 2
+    if p["aop"] == 0:
+        # acc_bufs accumulators [0, nb*n_mt*n_tile), then sa A stages of n_mt * 32 columns
+        assert nb * p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
+        assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512
+    else:
+        # A in shared memory: tensor memory holds only the accumulators
+        assert nb * p["n_mt"] * p["n_tile"] <= 512
+    assert nb * p["n_mt"] * p["n_sub"] <= 16
     assert p["n_sub"] * p["sub_n"] == p["n_tile"] and p["sub_n"] % 16 == 0 and 16 <= p["sub_n"] <= 256
     assert p["smem"] <= 232448 and p["TH"] * p["TW"] == 128
     assert p["w_box"] <= 256 and p["h_ext"] <= 256 and p["kd_ext"] <= 256
