@@ -77,3 +77,58 @@ def test_noalloc_in_place_bf16_weights_have_no_size_limit(cuda_ok):
     r = api.conv3d_implicit_gemm(x, w, b, 1, 1, 1, act_amax=amax, quant_act=True)
     assert api.check_device_error() == 0
     assert torch.equal(y, r)
+
+
+def _captured_node_types(call):
+    """Capture `call(stream)` on a fresh stream into a CUDA graph (relaxed
+    mode, never launched) and return the types of the graph's nodes."""
+    from cuda.bindings import runtime as rt
+
+    err, s = rt.cudaStreamCreateWithFlags(rt.cudaStreamNonBlocking)
+    assert err == rt.cudaError_t.cudaSuccess
+    ts = torch.cuda.ExternalStream(int(s))
+    try:
+        err, = rt.cudaStreamBeginCapture(s, rt.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+        assert err == rt.cudaError_t.cudaSuccess
+        call(ts)
+        err, graph = rt.cudaStreamEndCapture(s)
+        assert err == rt.cudaError_t.cudaSuccess
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        assert err == rt.cudaError_t.cudaSuccess
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        assert err == rt.cudaError_t.cudaSuccess
+        types = []
+        for nd in nodes[:n]:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            assert err == rt.cudaError_t.cudaSuccess
+            types.append(t)
+        rt.cudaGraphDestroy(graph)
+        return types
+    finally:
+        rt.cudaStreamDestroy(s)
+
+
+def test_noalloc_enqueues_no_allocation(cuda_ok):
+    """The property the entry point exists for: with weights that must be
+    staged (F16), the regular entry point's captured work contains a
+    stream-ordered allocation and the no-alloc one's does not."""
+    from cuda.bindings import runtime as rt
+
+    xs, cout, k, s, pad6, d, dtype, quant = CASES[0]
+    x, w, b, a = _inputs(400, xs, cout, k, dtype)
+    oshape = api.out_shape(x.shape, w.shape, s, pad6, d)
+    y = torch.empty(oshape, dtype=dtype, device="cuda")
+    # first calls outside any capture (the no-alloc area's address is looked up once)
+    api.conv3d_implicit_gemm_noalloc(x, w, y, b, s, pad6, d, act_amax=a, quant_act=quant)
+    api.conv3d_implicit_gemm(x, w, b, s, pad6, d, act_amax=a, quant_act=quant, out=y)
+    assert api.check_device_error() == 0
+    alloc = rt.cudaGraphNodeType.cudaGraphNodeTypeMemAlloc
+    regular = _captured_node_types(lambda st: api.conv3d_implicit_gemm(x, w, b, s, pad6, d, act_amax=a,
+                                                                      quant_act=quant, out=y, stream=st))
+    noalloc = _captured_node_types(lambda st: api.conv3d_implicit_gemm_noalloc(x, w, y, b, s, pad6, d, act_amax=a,
+                                                                              quant_act=quant, stream=st))
+    assert alloc in regular          # the check can see an allocation
+    assert alloc not in noalloc
+    assert rt.cudaGraphNodeType.cudaGraphNodeTypeKernel in noalloc
+    torch.cuda.synchronize()
+    assert api.check_device_error() == 0
