@@ -50,7 +50,8 @@ L2_BYTES = 126 * 1024 * 1024
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-KERNEL_SOURCES = ("conv3d_igemm_tmem.cu", "conv3d_tmem_kernel.cuh", "sm100_ptx.cuh", "nvfp4.cuh")
+KERNEL_SOURCES = ("conv3d_igemm_tmem.cu", "conv3d_igemm_tmem_sa.cu", "conv3d_tmem_kernel.cuh", "sm100_ptx.cuh",
+                  "nvfp4.cuh")
 # nominal dense FP4 : BF16 tensor throughput of B200 (9 : 2.25 PFLOP/s); the
 # FP4 roofline is the measured BF16 peak times this ratio
 FP4_OVER_BF16 = 4.0
