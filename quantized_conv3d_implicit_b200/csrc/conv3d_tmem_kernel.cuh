@@ -1,12 +1,10 @@
 // conv3d_tmem_kernel.cuh -- the tensor-memory implicit-GEMM Conv3D kernel
 // template, its host planner and launch helpers, shared by the translation
-// units that instantiate it (conv3d_igemm_tmem.cu: BF16 tensor-core
-// operands; conv3d_fp4.cu: NVFP4 operands for the block-scaled MMA).
-// Everything here has internal linkage.
-//
-// The kernel: implicit-GEMM Conv3D for sm_100a with the A
-// operand (the implicit im2col matrix, fake-quantised on the fly) built in
-// tensor memory.
+// units that instantiate it (conv3d_igemm_tmem.cu: BF16 operands, A in
+// tensor memory; conv3d_igemm_tmem_sa.cu: BF16 operands, A in shared memory;
+// conv3d_fp4.cu: NVFP4 operands for the block-scaled MMA).  The kernel
+// parameters (TmemParams) have external linkage; everything else here is
+// internal to each unit.
 //
 // GEMM view as in the Model-Optimizer "Conv3D Implicit GEMM CUDA kernel"
 // article, sec. 5.1 (rows (n, od, oh, ow), columns (c, kd, kh, kw)), with the
@@ -14,31 +12,33 @@
 //
 // A tile is n_mt M-subtiles of 128 output positions (TH x TW rectangles of one
 // (n, od) plane, stacked along oh) times n_tile output channels.  Per 64-wide
-// K slice, the weights arrive by TMA in shared memory (K-major, 128B swizzle)
-// and the A slice is written by the transform warps straight into tensor
-// memory with tcgen05.st, one 32-bit column per pair of consecutive K
-// elements; tcgen05.mma then reads A from tensor memory and B from shared
-// memory.  Shared memory therefore carries only the input halo and the
-// weights, not A.
+// K slice, the weights arrive in shared memory (TMA, K-major, 128B swizzle;
+// prepacked NVFP4 images by bulk copy in the NVFP4 form) and the transform
+// warps build the slice of A from the input halo: BF16 values straight into
+// tensor memory with tcgen05.st (one 32-bit column per pair of consecutive K
+// elements), or BF16 values / NVFP4 codes into a swizzled shared-memory stage.
+// tcgen05.mma reads A from there and B from shared memory, accumulating in
+// FP32 in tensor memory (one or two accumulator buffers).
 //
 // Roles (24 warps, one persistent CTA per SM):
-//   warp 0      weight producer (TMA);
-//   warp 1      TMEM owner and MMA issuer (tcgen05.mma kind::f16, M = 128,
-//               N = n_tile in <= 256-wide instructions, K = 16 per
-//               instruction = one quantisation block);
+//   warp 0      weight producer;
+//   warp 1      TMEM owner and MMA issuer (tcgen05.mma, M = 128, N = n_tile
+//               in <= 256-wide instructions; kind::f16 with K = 16 per
+//               instruction = one quantisation block, or the block-scaled
+//               kind::mxf4nvf4 with K = 64);
 //   warp 2      halo producer: 5-D TMA boxes of x (zero fill outside the
 //               input = the convolution padding) into a ring of slots;
-//   warps 4-7   epilogue: tcgen05.ld, bias in FP32, rounding to the output
-//               dtype, bounds-checked NCDHW stores;
-//   warps 8-23  transform.  Warp w owns TMEM lane quadrant w % 4 (the lanes
-//               its tcgen05.st may reach) and 16-column block (w - 8) / 4 of
-//               every K slice; each thread owns one output position (a TMEM
-//               lane) of every subtile.  Per block it gathers its 16 halo
-//               values with per-CTA tables of tap offsets, takes the block
-//               maximum, derives the E4M3 scale (IEEE division), and
-//               dequantises through a per-row table of the eight BF16
-//               magnitudes q*scale (byte permutes indexed by the E2M1
-//               codes), then stores the 16 BF16 values with one tcgen05.st.
+//   warps 4-7   epilogue: tcgen05.ld, the NVFP4 form's global scales and the
+//               bias in FP32, rounding to the output dtype, bounds-checked
+//               NCDHW stores staged for 16-byte writes;
+//   warps 8-23  transform, in two groups taking alternate K slices.  Warp w
+//               owns lane quadrant w % 4 (the TMEM lanes its tcgen05.st may
+//               reach) and two 16-column blocks of each of its slices; each
+//               thread owns one output position (row) of every subtile.  Per
+//               block it gathers its 16 halo values, takes the block maximum,
+//               looks up the block's quantiser entry (E4M3 scale, 1/scale and
+//               the dequantisation table) in per-CTA tables, and writes the
+//               quantised values.
 // All waits are bounded; a timeout in any role aborts all roles.
 #pragma once
 #include <algorithm>
@@ -91,7 +91,7 @@ struct TmemParams {
   // weights arrive as prepacked images, one per N-part and K slice; the
   // scale factors of both operands are copied into tensor memory, a region
   // per A stage
-  int fp4;
+  int fp4;                // aop == NVFP4 (kept for the host side)
   int aop;                // A operand mode: 0 BF16 in tensor memory, 1 BF16 in shared memory, 2 NVFP4
   int dtype_code;         // element type of x: 0 f32, 1 f16, 2 bf16
   uint32_t off_a, a_stage_bytes;
@@ -1642,7 +1642,8 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
   p.n_parts = n_ntiles * n_sub;
   p.b_img_bytes = static_cast<uint32_t>(sub_n * 32 + p.n_atoms * 512);
   // TMEM columns after the accumulators (32-aligned), and what one A stage
-  // takes there: 32 BF16-pair columns per subtile, or (fp4) the scale factors
+  // takes there: 32 BF16-pair columns per subtile (A in tensor memory), the
+  // scale factors (NVFP4), or nothing (BF16 A in shared memory)
   auto a_col0_of = [&](int mt, int nb = 1) { return (nb * mt * n_tile + 31) / 32 * 32; };
   auto stage_cols = [&](int mt) { return fp4 ? 4 * mt + 4 * p.n_atoms * n_sub : smem_a ? 0 : mt * 32; };
   auto stages_of = [&](int mt, int nb = 1) {

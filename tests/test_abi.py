@@ -292,3 +292,25 @@ def test_fp4_plans_fit_every_workload():
         assert p["a_stage_bytes"] >= p["n_mt"] * (4096 + 512) and p["a_stage_bytes"] % 1024 == 0, name
         assert p["b_stage_bytes"] >= p["n_sub"] * (p["sub_n"] * 32 + -(-p["sub_n"] // 128) * 512), name
         assert 2 <= p["sa"] <= 4 and p["sb"] >= 2, name
+
+
+def test_bf16_plan_choice_per_workload():
+    """The launcher's A placement (plan hook field aop): shared memory where
+    it frees tensor memory for four subtiles or more A stages (measured
+    faster there), tensor memory for the wide layers (measured faster)."""
+    from quantized_conv3d_implicit_b200 import workloads
+    want = {"edge_full_96_bf16": (1, 4), "wan_hi_192_bf16": (1, 2), "wan_mid_384_bf16": (0, 1),
+            "pointwise_512to1024_fp16": (0, 1), "edge_full_96_bf16_dil122": (None, 2)}
+    for name, (aop, mt) in want.items():
+        wl = workloads.WORKLOADS[name]
+        ws = (wl.cout, wl.x_shape[1]) + tuple(wl.kernel)
+        pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+        p = api.plan_conv(wl.x_shape, ws, wl.stride, pad6, wl.dil, wl.dtype, kernel="tmem")
+        assert p["applicable"] == 1, name
+        if aop is not None:
+            assert p["aop"] == aop, (name, p["aop"])
+        assert p["n_mt"] == mt, (name, p["n_mt"])
+        # accumulators (one or two buffers) fit the 512 columns, A stages beside them in tensor memory
+        assert p["acc_bufs"] * p["n_mt"] * p["n_tile"] <= 512
+        if p["aop"] == 0:
+            assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512
