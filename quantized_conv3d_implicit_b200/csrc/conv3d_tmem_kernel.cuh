@@ -1049,10 +1049,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int co0 = tc.nt * p.n_tile + ns * p.sub_n;
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + buf * static_cast<uint32_t>(p.acc_cols) +
                                  static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+          // each step's 16 columns are loaded while the previous step's are
+          // processed, so the accumulator is handed back one step earlier and
+          // the loads' latency is hidden
+          uint32_t nv[16];
+          tmem_ld16(taddr, nv);
           for (int c0 = 0; c0 < p.sub_n; c0 += 16) {
             uint32_t v[16];
-            tmem_ld16(taddr + static_cast<uint32_t>(c0), v);
             tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = nv[j];
+            if (c0 + 16 < p.sub_n) tmem_ld16(taddr + static_cast<uint32_t>(c0 + 16), nv);
             if (c0 + 16 >= p.sub_n) {  // the accumulator is in registers: hand it back
               tc_fence_before();
               __syncwarp();
