@@ -398,6 +398,8 @@ def run_ours(args, world, rank, local):
     if not args.no_layers:
         layers, layers_fp4, layer_clocks = run_layers(api, args, stream, dev, peak, sets, wl.name, rank)
 
+    formats = None if (args.no_formats or fp4) else time_formats(api, wl, base, stream, dev, hbm, peak)
+
     # end-to-end through the public API with pinned host buffers
     e2e = None if (args.no_e2e or fp4) else run_e2e(args, wl, base, stream, dev, world)
 
@@ -450,6 +452,8 @@ def run_ours(args, world, rank, local):
     if layers is not None:
         result["layers"] = layers
         result["layers_clocks"] = layer_clocks
+    if formats is not None:
+        result["formats"] = formats
     if layers_fp4:
         result["layers_fp4"] = {
             "what": ("conv3d_implicit_gemm_fp4: activations and weights NVFP4, block-scaled FP4 MMA "
@@ -641,6 +645,70 @@ def run_reference(args, world, rank, local):
     }), flush=True)
 
 
+def time_formats(api, wl, base, stream, dev, hbm, bf16_peak):
+    """The quantiser formats beyond the article's default: the standalone
+    NVFP4 fake-quant with blocks of 32..256 and MXFP4 (dequantised values,
+    scale bytes and packed codes) on the layer's x, against the HBM roofline
+    (L2 flushed before each launch); and the fused convolution with each
+    format on the wan_mid layer (the general kernel runs every format but
+    NVFP4 blocks of 16), against the BF16 peak."""
+    import torch
+
+    from quantized_conv3d_implicit_b200 import workloads
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    x, amax = base["x"], base["act_amax"]
+    esz = x.element_size()
+    n = x.numel()
+
+    def timed(fn, reps=5):
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b) * 1e3)
+        if api.check_device_error(stream) != 0:
+            raise RuntimeError("device error in a format timing")
+        return statistics.mean(ts)
+
+    out = {"x": wl.name, "standalone": {}, "fused_conv": {}}
+    q = torch.empty_like(x)
+    for bs in (32, 64, 128, 256):
+        us = timed(lambda: api.fp4_fake_quant(x, amax, out=q, stream=stream, block_size=bs))
+        by = 2 * n * esz
+        out["standalone"][f"nvfp4_{bs}"] = {"us": round(us, 1), "gbs": round(by / (us * 1e-6) / 1e9, 1),
+                                           "frac_hbm": round(by / (us * 1e-6) / 1e9 / hbm, 4)}
+    scales = torch.empty(n // 32, dtype=torch.uint8, device=dev)
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    xs, os_ = api._tensor(x), api._tensor(q)
+    lib = api.load_library()
+
+    def mx():
+        api._check(lib, lib.mxfp4_quantize(api._ref(xs), 0.0, api._ref(os_), scales.data_ptr(), codes.data_ptr(),
+                                           api._stream_handle(stream)))
+    us = timed(mx)
+    by = n * esz + n * esz + n // 32 + n // 2
+    out["standalone"]["mxfp4"] = {"us": round(us, 1), "gbs": round(by / (us * 1e-6) / 1e9, 1),
+                                  "frac_hbm": round(by / (us * 1e-6) / 1e9 / hbm, 4)}
+    del q, scales, codes
+    torch.cuda.empty_cache()
+    cw = workloads.get("wan_mid_384_bf16")
+    inp = workloads.make_inputs(cw, device=dev, with_out=True)
+    for fmt, bs, dst in (("nvfp4", 16, 0.0), ("nvfp4", 32, 0.0), ("nvfp4", 128, 0.0), ("mxfp4", 32, 0.0)):
+        us = timed(lambda: api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], inp["bias"], cw.stride, pad6(cw), cw.dil,
+                                                        inp["act_amax"], quant_format=fmt, block_size=bs,
+                                                        dst_type_max=dst, out=inp["out"], stream=stream), reps=3)
+        tf = cw.flops / (us * 1e-6) / 1e12
+        out["fused_conv"][f"{fmt}_{bs}"] = {"layer": cw.name, "us": round(us, 1), "tflops": round(tf, 1),
+                                           "frac": round(tf / bf16_peak, 4)}
+    return out
+
+
 def time_act_amax(x, stream, dev, steps):
     """Mean device time (us) of q3d_act_amax on x (memset of the output word
     + one kernel), CUDA events on the launching stream, L2 flushed before
@@ -678,6 +746,7 @@ def main(argv=None):
     ap.add_argument("--no-layers", action="store_true", help="skip the per-workload convolution timings")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end timing with host copies")
     ap.add_argument("--no-fp4", action="store_true", help="skip the true-FP4 convolution timings")
+    ap.add_argument("--no-formats", action="store_true", help="skip the other quantiser formats' timings")
     ap.add_argument("--conv", default="bf16", choices=["bf16", "fp4"],
                     help="the step's convolution: the fake-quantised BF16 path (default) or the true-FP4 variant")
     args = ap.parse_args(argv)
