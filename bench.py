@@ -650,8 +650,9 @@ def time_formats(api, wl, base, stream, dev, hbm, bf16_peak):
     NVFP4 fake-quant with blocks of 32..256 and MXFP4 (dequantised values,
     scale bytes and packed codes) on the layer's x, against the HBM roofline
     (L2 flushed before each launch); and the fused convolution with each
-    format on the wan_mid layer (the general kernel runs every format but
-    NVFP4 blocks of 16), against the BF16 peak."""
+    format on the wan_mid layer (the tensor-memory kernel runs NVFP4 blocks
+    of 16 and 32 and MXFP4, the general kernel the larger NVFP4 blocks),
+    against the BF16 peak."""
     import torch
 
     from quantized_conv3d_implicit_b200 import workloads

@@ -926,6 +926,7 @@ cudaError_t launch_conv3d_fast(const ConvGeom& g, const ConvLaunch& L, cudaStrea
                                bool* handled) {
   *handled = false;
   if (kernel_choice() == 1) return cudaSuccess;
+  if (L.quant && !(L.qfmt == 1 && L.qblock == 16)) return cudaSuccess;  // NVFP4 blocks of 16 only
   const int esz = L.dtype == 0 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   FastParams p{};

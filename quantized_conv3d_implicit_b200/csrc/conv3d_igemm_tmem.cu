@@ -44,12 +44,24 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
 cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
                                bool* handled) {
   *handled = false;
+  // quantisers: NVFP4 blocks of 16 or 32, MXFP4 (larger NVFP4 blocks span
+  // several warps' columns: the general kernel)
+  int qmode = kQModeNv16;
+  if (L.quant) {
+    if (L.qfmt == 2)
+      qmode = kQModeMx;
+    else if (L.qblock == 32)
+      qmode = kQModeNv32;
+    else if (L.qblock != 16)
+      return cudaSuccess;
+  }
   const int esz = L.dtype == 0 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   TmemParams p{};
   size_t smem = 0;
   if (!choose_plan(g, L.dtype, p, smem)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
+  p.qmode = qmode; p.dst_max = L.dst_max;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;
 
   EncodeTiledFn encode = get_encode_tiled();
@@ -78,6 +90,7 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
     p.withhold_arrive = 1;
   }
   *handled = true;
+  if (L.quant && qmode != kQModeNv16) return launch_tmem_groups(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
   if (p.aop == kAOpBf16Smem) return launch_tmem_smem_a(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);
   switch (L.dtype) {
     case 0: return launch_tmem_typed<float, kAOpBf16Tmem>(p, tmap_x, tmap_w, static_cast<int>(grid64), smem, s);

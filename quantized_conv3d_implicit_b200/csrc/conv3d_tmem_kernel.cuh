@@ -101,11 +101,21 @@ struct TmemParams {
   int sf_col0, sf_cols;   // scale-factor columns of A stage e: sf_col0 + e * sf_cols
   const uint8_t* wq;      // the first image (slice 0, part 0)
   const float* g_w;       // global scale of the weights (device scalar)
+  // BF16 forms, when quant: the activation quantiser (kQMode*) and, for
+  // MXFP4, the largest magnitude a group's maximum is scaled to (0: the
+  // E2M1 rule floor(log2 amax) - 2)
+  int qmode;
+  float dst_max;
 };
 
 // The BF16 kernel with A in shared memory (instantiated in its own
 // translation unit, conv3d_igemm_tmem_sa.cu).
 cudaError_t launch_tmem_smem_a(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
+                               size_t smem, cudaStream_t s);
+// The BF16 kernel with the 32-column-group quantisers (p.qmode NVFP4 blocks
+// of 32 or MXFP4), A in tensor or shared memory as p.aop says (instantiated
+// in conv3d_igemm_tmem_g32.cu).
+cudaError_t launch_tmem_groups(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                                size_t smem, cudaStream_t s);
 
 namespace {
@@ -127,6 +137,12 @@ constexpr uint32_t kTmemCols = 512;
 //   BF16 values in shared memory (128-byte-swizzled K-major, like B);
 //   NVFP4 codes and scale bytes in shared memory (block-scaled MMA).
 constexpr int kAOpBf16Tmem = 0, kAOpBf16Smem = 1, kAOpNvfp4 = 2;
+// The activation quantiser of the BF16 forms: NVFP4 with blocks of 16 (the
+// default), NVFP4 with blocks of 32 (an E4M3 scale per 32 columns), MXFP4
+// (a power-of-two scale per 32 columns).  A warp's two adjacent 16-column
+// blocks of a K slice (b0 even) are one 32-column group, so a group's
+// maximum never leaves the thread that owns its row.
+constexpr int kQModeNv16 = 0, kQModeNv32 = 1, kQModeMx = 2;
 
 
 struct TileCoord {
@@ -318,6 +334,8 @@ struct Half2<__nv_bfloat16> {
   // |x| as an operand modifier of the consuming multiply or max
   static __device__ __forceinline__ float abs_lo(uint32_t w) { return fabsf(__uint_as_float(w << 16)); }
   static __device__ __forceinline__ float abs_hi(uint32_t w) { return fabsf(__uint_as_float(w & 0xFFFF0000u)); }
+  static __device__ __forceinline__ float lo(uint32_t w) { return __uint_as_float(w << 16); }
+  static __device__ __forceinline__ float hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
   static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_bf16x2(a, b); }
   static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) { return w; }
   // entry of a block from the packed |v| maximum of its eight words: the
@@ -335,6 +353,12 @@ struct Half2<__half> {
   }
   static __device__ __forceinline__ float abs_hi(uint32_t w) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>((w >> 16) & 0x7FFFu)));
+  }
+  static __device__ __forceinline__ float lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+  }
+  static __device__ __forceinline__ float hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
   }
   static __device__ __forceinline__ uint32_t maxabs(uint32_t a, uint32_t b) { return maxabs_f16x2(a, b); }
   static __device__ __forceinline__ uint32_t to_bf16x2(uint32_t w) {
@@ -632,6 +656,126 @@ __device__ __forceinline__ void fp4_block_x2(const uint32_t (&pa)[8], const uint
   fp4_codes16<T>(pb, ib, cb0, cb1);
 }
 
+// ---- 32-column groups (NVFP4 blocks of 32, MXFP4) ----
+//
+// The dequantisation table of a scale by direct products, each q * s
+// rounded to binary32 and then to BF16 like every other entry.  An MXFP4
+// scale 2^E reaches the subnormal and the overflow ends of binary32, where
+// the exponent-field steps of dq_table do not hold.
+__device__ __forceinline__ DqTable dq_table_direct(float s) {
+  const uint32_t p01 = cvt_bf16x2(__fmul_rn(0.5f, s), __fmul_rn(0.0f, s));
+  const uint32_t p23 = cvt_bf16x2(__fmul_rn(1.5f, s), s);
+  const uint32_t p45 = cvt_bf16x2(__fmul_rn(3.0f, s), __fmul_rn(2.0f, s));
+  const uint32_t p67 = cvt_bf16x2(__fmul_rn(6.0f, s), __fmul_rn(4.0f, s));
+  DqTable t;
+  t.lo_a = __byte_perm(p01, p23, 0x6420);
+  t.hi_a = __byte_perm(p01, p23, 0x7531);
+  t.lo_b = __byte_perm(p45, p67, 0x6420);
+  t.hi_b = __byte_perm(p45, p67, 0x7531);
+  return t;
+}
+
+// The MXFP4 scale 2^E of a group from its |v| maximum: its table and
+// down = 2^-E (an all-zero group gets E = -127 and only zero codes).
+__device__ __forceinline__ void mx_group_scale(float gmax, float dst_max, DqTable& dt, float& down) {
+  const int e = mx_scale_exp(gmax, dst_max);
+  down = mx_exp2i(-e);
+  dt = dq_table_direct(mx_exp2i(e));
+}
+
+// Two 16-column blocks of one row (eight packed words each) that form one
+// 32-column group: the joint maximum sets one scale for both.
+template <typename T>
+__device__ __forceinline__ void quant_group32(const uint32_t (&pa)[8], const uint32_t (&pb)[8], int qmode,
+                                              float dst_max, const QCtx& q, uint32_t (&wa)[8], uint32_t (&wb)[8]) {
+  using H = Half2<T>;
+  const uint32_t m = H::maxabs(maxabs8<T>(pa), maxabs8<T>(pb));
+  DqTable dt;
+  float inv;
+  if (qmode == kQModeNv32)
+    load_entry(H::entry(m, q), dt, inv);
+  else
+    mx_group_scale(fmaxf(H::abs_lo(m), H::abs_hi(m)), dst_max, dt, inv);
+  quant8<T>(pa, dt, inv, wa);
+  quant8<T>(pb, dt, inv, wb);
+}
+
+// The same for binary32 inputs (16 values per block).
+__device__ __forceinline__ void quant_group32_f32(const float (&va)[16], const float (&vb)[16], int qmode,
+                                                  float dst_max, const QCtx& q, uint32_t (&wa)[8],
+                                                  uint32_t (&wb)[8]) {
+  float gmax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) gmax = fmaxf(gmax, fmaxf(fabsf(va[j]), fabsf(vb[j])));
+  DqTable dt;
+  float inv;
+  if (qmode == kQModeNv32)
+    load_entry(entry_of_max(gmax, q), dt, inv);
+  else
+    mx_group_scale(gmax, dst_max, dt, inv);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = 4 * i;
+    uint32_t s01 = __byte_perm(__float_as_uint(va[j]), __float_as_uint(va[j + 1]), 0x7632);
+    uint32_t s23 = __byte_perm(__float_as_uint(va[j + 2]), __float_as_uint(va[j + 3]), 0x7632);
+    dq4(dt, __fmul_rn(fabsf(va[j]), inv), __fmul_rn(fabsf(va[j + 1]), inv), __fmul_rn(fabsf(va[j + 2]), inv),
+        __fmul_rn(fabsf(va[j + 3]), inv), s01, s23, wa[2 * i], wa[2 * i + 1]);
+    s01 = __byte_perm(__float_as_uint(vb[j]), __float_as_uint(vb[j + 1]), 0x7632);
+    s23 = __byte_perm(__float_as_uint(vb[j + 2]), __float_as_uint(vb[j + 3]), 0x7632);
+    dq4(dt, __fmul_rn(fabsf(vb[j]), inv), __fmul_rn(fabsf(vb[j + 1]), inv), __fmul_rn(fabsf(vb[j + 2]), inv),
+        __fmul_rn(fabsf(vb[j + 3]), inv), s01, s23, wb[2 * i], wb[2 * i + 1]);
+  }
+}
+
+// One block's 16 tap offsets from its phase-table row, the columns from
+// `split` on moved by `adj` (their channel opens the next halo slot).
+template <int kDWB>
+__device__ __forceinline__ void block_taps(uint32_t prow, int phi, int split, int adj, int (&off)[16]) {
+  if constexpr (kDWB > 0)
+    taps_from_rows<kDWB>(prow, phi % 3, off);
+  else
+    load_taps(prow, off);
+  if (adj != 0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) off[j] += (j >= split) ? adj : 0;
+  }
+}
+
+// One row's 32-column group by tap offsets: block a at addr_a with nv_a
+// valid columns, block b (the next 16 columns) at addr_b with nv_b (<= 0:
+// past K, zeros).
+template <typename T, int kDWB>
+__device__ __forceinline__ void group32_taps(uint32_t addr_a, uint32_t prow_a, int phi_a, int split_a, int adj_a,
+                                             int nv_a, uint32_t addr_b, uint32_t prow_b, int phi_b, int split_b,
+                                             int adj_b, int nv_b, int qmode, float dst_max, const QCtx& q,
+                                             uint32_t (&wa)[8], uint32_t (&wb)[8]) {
+  int off[16];
+  if constexpr (sizeof(T) == 2) {
+    uint32_t pa[8], pb[8];
+    block_taps<kDWB>(prow_a, phi_a, split_a, adj_a, off);
+    gather_taps<T>(addr_a, off, nv_a, pa);
+    if (nv_b > 0) {
+      block_taps<kDWB>(prow_b, phi_b, split_b, adj_b, off);
+      gather_taps<T>(addr_b, off, nv_b, pb);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pb[i] = 0u;
+    }
+    quant_group32<T>(pa, pb, qmode, dst_max, q, wa, wb);
+  } else {
+    float va[16], vb[16];
+    block_taps<kDWB>(prow_a, phi_a, split_a, adj_a, off);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      va[j] = j < nv_a ? __uint_as_float(ld_shared_u32(addr_a + static_cast<uint32_t>(off[j]))) : 0.0f;
+    if (nv_b > 0) block_taps<kDWB>(prow_b, phi_b, split_b, adj_b, off);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      vb[j] = j < nv_b ? __uint_as_float(ld_shared_u32(addr_b + static_cast<uint32_t>(off[j]))) : 0.0f;
+    quant_group32_f32(va, vb, qmode, dst_max, q, wa, wb);
+  }
+}
+
 // One row x one 16-column block of any input type, gathered by tap offsets
 // (nvalid < 16 only in a partial last block: the missing columns are zero).
 template <typename T>
@@ -854,8 +998,11 @@ __device__ __forceinline__ void mma_issue_loop_fp4(const TmemParams& p, uint32_t
 // rows with immediate column offsets; 0: gathered by tap offsets.  kFp4: the
 // NVFP4-operand variant (A as E2M1 codes and scale bytes in shared memory,
 // prepacked NVFP4 weights, block-scaled MMA, the two global scales applied
-// in the epilogue); otherwise BF16 operands with A in tensor memory.
-template <typename T, bool kPairs, int kDWB, int kAOp>
+// in the epilogue); otherwise BF16 operands with A in tensor memory.  kQ = 1:
+// the activation quantiser works on 32-column groups (NVFP4 blocks of 32 or
+// MXFP4, p.qmode), a separate instantiation so the default quantiser's
+// forms keep their code; 0: blocks of 16, or no quantisation.
+template <typename T, bool kPairs, int kDWB, int kAOp, int kQ = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     conv3d_igemm_tmem_kernel(const __grid_constant__ TmemParams p, const __grid_constant__ CUtensorMap tmap_x,
                              const __grid_constant__ CUtensorMap tmap_w) {
@@ -1166,7 +1313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // taken in the next channel as if it followed contiguously (chan_bytes
     // further on).
     QCtx q{};
-    q.G = p.quant ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
+    // the NVFP4 tables (MXFP4 takes no global amax: act_amax may be null)
+    const bool nv_tables = p.quant && (kQ == 0 || p.qmode != kQModeMx);
+    q.G = nv_tables ? nvfp4_global(__ldg(p.act_amax)) : Nvfp4Global{0.0f, 0.0f, 0.0f};
     q.dq = base + p.off_dq;
     if constexpr (std::is_same<T, __nv_bfloat16>::value) {
       // the window starts 11 binades below t's binade (pattern 0 if t is
@@ -1177,7 +1326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       q.cb = base + p.off_code - 2u * q.lo;
     }
     {
-      if (p.quant) {
+      if (nv_tables) {
         if (xf_tid < 128) {
           uint32_t h2;
           asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<unsigned short>(xf_tid & 0x7F)));
@@ -1315,7 +1464,78 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         const bool quant = p.quant != 0;
         bool pair_done = false;
-        if constexpr (!kPairs && sizeof(T) == 2) {
+        if constexpr (!kFp4 && kQ == 1) {
+          {
+            // NVFP4 blocks of 32 or MXFP4 (always quantised): the warp's
+            // blocks b0, b0 + 1 of a row are one group; both are gathered
+            // per subtile and share the scale of their joint maximum
+            pair_done = true;
+            if (nv0 <= 0) {
+              uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+              for (int i = 0; i < p.n_mt; ++i) {
+                put(i, 0, z);
+                put(i, 1, z);
+              }
+            } else {
+              const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb);
+              const uint32_t org1 = halo_base + h1.e * p.slot_bytes + static_cast<uint32_t>(cs1 * cb);
+              const uint32_t prow0 = phase_tab + static_cast<uint32_t>(phi * 64);
+              const uint32_t prow1 = phase_tab + static_cast<uint32_t>(phi1 * 64);
+              // a block whose second channel opens the next slot: its columns there move by adj
+              int adj0 = 0, adj1 = 0;
+              if (cross0) {
+                RingPos hn = h0;
+                hn.next(ring);
+                adj0 = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org0) - cb;
+              }
+              if (cross1) {
+                RingPos hn = h1;
+                hn.next(ring);
+                adj1 = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org1) - cb;
+              }
+              bool rows_done = false;
+              if constexpr (kDWB > 0 && sizeof(T) == 2) {
+                if (nv1 >= 16) {
+                  // both blocks full: row gathers (block b0 + 1 starts one
+                  // column further in the row pattern, taps being a multiple of 3)
+                  const int p3 = phi % 3;
+                  uint32_t r0[6], r1[6];
+                  row_bases(org0 + thr0, prow0, cross0 ? (g.taps - phi + p3) / 3 : 6, adj0, r0);
+                  row_bases(org1 + thr0, prow1, cross1 ? (g.taps - phi1 + phi1 % 3) / 3 : 6, adj1, r1);
+                  for (int i = 0; i < p.n_mt; ++i) {
+                    uint32_t pa[8], pb[8], wa[8], wb[8];
+                    switch (p3) {
+                      case 0: gather_rows<0, kDWB>(r0, pa); gather_rows<1, kDWB>(r1, pb); break;
+                      case 1: gather_rows<1, kDWB>(r0, pa); gather_rows<2, kDWB>(r1, pb); break;
+                      default: gather_rows<2, kDWB>(r0, pa); gather_rows<0, kDWB>(r1, pb); break;
+                    }
+                    quant_group32<T>(pa, pb, p.qmode, p.dst_max, q, wa, wb);
+                    put(i, 0, wa);
+                    put(i, 1, wb);
+#pragma unroll
+                    for (int r = 0; r < 6; ++r) {
+                      r0[r] += thr_step;
+                      r1[r] += thr_step;
+                    }
+                  }
+                  rows_done = true;
+                }
+              }
+              if (!rows_done) {
+                uint32_t a0 = org0 + thr0, a1 = org1 + thr0;
+#pragma unroll 1
+                for (int i = 0; i < p.n_mt; ++i, a0 += thr_step, a1 += thr_step) {
+                  uint32_t wa[8], wb[8];
+                  group32_taps<T, kDWB>(a0, prow0, phi, split0, adj0, nv0, a1, prow1, phi1, split1, adj1, nv1, p.qmode,
+                                        p.dst_max, q, wa, wb);
+                  put(i, 0, wa);
+                  put(i, 1, wb);
+                }
+              }
+            }
+          }
+        }
+        if constexpr (!kPairs && sizeof(T) == 2 && kQ == 0) {
           // single subtile, both blocks full and within their slots: one interleaved pass
           if (nv0 >= 32 && !cross0 && !cross1) {
             const uint32_t org0 = halo_base + h0.e * p.slot_bytes + static_cast<uint32_t>(cs0 * cb) + thr0;
@@ -1545,10 +1765,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <typename T, bool kPairs, int kDWB, int kAOp>
+template <typename T, bool kPairs, int kDWB, int kAOp, int kQ>
 cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid, size_t smem,
                              cudaStream_t s) {
-  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB, kAOp>;
+  auto kern = conv3d_igemm_tmem_kernel<T, kPairs, kDWB, kAOp, kQ>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, s>>>(p, tx, tw);
@@ -1557,21 +1777,21 @@ cudaError_t launch_tmem_inst(const TmemParams& p, const CUtensorMap& tx, const C
 
 // Row gather for 16-bit inputs and kernels three taps wide with W dilation 1
 // or 2; tap-offset gather otherwise.
-template <typename T, int kAOp>
+template <typename T, int kAOp, int kQ = 0>
 cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                               size_t smem, cudaStream_t s) {
   const int dwb = row_gather_step(p.g, sizeof(T));
   const bool pairs = p.n_mt >= 2;
   if constexpr (sizeof(T) == 2) {
     if (dwb == 2)
-      return pairs ? launch_tmem_inst<T, true, 2, kAOp>(p, tx, tw, grid, smem, s)
-                   : launch_tmem_inst<T, false, 2, kAOp>(p, tx, tw, grid, smem, s);
+      return pairs ? launch_tmem_inst<T, true, 2, kAOp, kQ>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 2, kAOp, kQ>(p, tx, tw, grid, smem, s);
     if (dwb == 4)
-      return pairs ? launch_tmem_inst<T, true, 4, kAOp>(p, tx, tw, grid, smem, s)
-                   : launch_tmem_inst<T, false, 4, kAOp>(p, tx, tw, grid, smem, s);
+      return pairs ? launch_tmem_inst<T, true, 4, kAOp, kQ>(p, tx, tw, grid, smem, s)
+                   : launch_tmem_inst<T, false, 4, kAOp, kQ>(p, tx, tw, grid, smem, s);
   }
-  return pairs ? launch_tmem_inst<T, true, 0, kAOp>(p, tx, tw, grid, smem, s)
-               : launch_tmem_inst<T, false, 0, kAOp>(p, tx, tw, grid, smem, s);
+  return pairs ? launch_tmem_inst<T, true, 0, kAOp, kQ>(p, tx, tw, grid, smem, s)
+               : launch_tmem_inst<T, false, 0, kAOp, kQ>(p, tx, tw, grid, smem, s);
 }
 
 // Output channels per tile: all of Cout up to 448 (448 + two 32-column A

@@ -224,7 +224,9 @@ q3d_status prepare_conv(const q3d_tensor* x, const q3d_tensor* w, const q3d_tens
 
 // The convolution kernels proper, once the BF16 weights are in place: the
 // tensor-memory kernel where it applies, else the shared-memory specialised
-// kernel, else the general one.  Q3D_KERNEL=tmem|fast|basic starts the chain
+// kernel, else the general one.  Each declines what it does not cover: the
+// tensor-memory kernel takes NVFP4 blocks of 16 or 32 and MXFP4, the
+// specialised one NVFP4 blocks of 16 only, the general one every format.  Q3D_KERNEL=tmem|fast|basic starts the chain
 // at that kernel, and Q3D_KERNEL=smem_a runs the tensor-memory kernel with
 // its A operand in shared memory wherever that form applies (all compute the
 // same result).
@@ -273,8 +275,7 @@ int32_t q3d_version(void) { return 100; }
 
 namespace {
 
-// Weight staging and the kernel chain for a prepared convolution.  The
-// quantiser's formats other than NVFP4 blocks of 16 run in the general kernel.
+// Weight staging and the kernel chain for a prepared convolution.
 q3d_status run_conv(const q3d::ConvGeom& g, q3d::ConvLaunch& L, const q3d_tensor* w, int32_t dtype,
                     q3d_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -300,8 +301,7 @@ q3d_status run_conv(const q3d::ConvGeom& g, q3d::ConvLaunch& L, const q3d_tensor
   }
 
   const char* why = nullptr;
-  const bool general = L.quant && !(L.qfmt == 1 && L.qblock == 16);
-  e = general ? q3d::launch_conv3d_basic(g, L, s, &why) : launch_conv(g, L, s, &why);
+  e = launch_conv(g, L, s, &why);
   if (scratch) cudaFreeAsync(scratch, s);
   if (e != cudaSuccess) {
     if (why) return fail(Q3D_ERR_CUDA, "conv3d launch: %s (%s)", why, cudaGetErrorString(e));
