@@ -1196,6 +1196,101 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int co0 = tc.nt * p.n_tile + ns * p.sub_n;
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(qw * 32) << 16) + buf * static_cast<uint32_t>(p.acc_cols) +
                                  static_cast<uint32_t>(i * p.n_tile + ns * p.sub_n);
+          if constexpr (kEsz == 2) {
+            if (vec_ok) {
+              // 16-bit outputs in 16-byte stores: the 16x256b TMEM shape gives
+              // each thread channel pairs of two positions, which stmatrix
+              // stores transposed straight into the staging rows (channel j:
+              // 32 positions), two shared-memory stores per step instead of
+              // one per channel.  Thread t's stmatrix row: channel
+              // 8 (mi / 2) + t % 8, position group 2 hh + mi % 2, mi = t / 8.
+              const int mi = lane >> 3;
+              const uint32_t srow = stage + static_cast<uint32_t>(8 * (mi >> 1) + (lane & 7)) * kPitch +
+                                    static_cast<uint32_t>(mi & 1) * 16u;
+              const int cpair = 2 * (lane & 3);  // the thread's first channel in each 8-channel half
+              uint32_t nv[16];
+              tmem_ld_16x256b_x2(taddr, *reinterpret_cast<uint32_t(*)[8]>(&nv[0]));
+              tmem_ld_16x256b_x2(taddr + (16u << 16), *reinterpret_cast<uint32_t(*)[8]>(&nv[8]));
+              for (int c0 = 0; c0 < p.sub_n; c0 += 16) {
+                uint32_t v[16];
+                tmem_wait_ld_regs(nv);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = nv[j];
+                if (c0 + 16 < p.sub_n) {
+                  const uint32_t tn = taddr + static_cast<uint32_t>(c0 + 16);
+                  tmem_ld_16x256b_x2(tn, *reinterpret_cast<uint32_t(*)[8]>(&nv[0]));
+                  tmem_ld_16x256b_x2(tn + (16u << 16), *reinterpret_cast<uint32_t(*)[8]>(&nv[8]));
+                } else {  // the accumulator is in registers: hand it back
+                  tc_fence_before();
+                  __syncwarp();
+                  const bool withhold = p.withhold_arrive && blockIdx.x == 0 && it == 0 && acc == 0 && qw == 0;
+                  if (lane == 0 && !withhold) mbar_arrive(bar_acc_empty + 8u * acc);
+                }
+                // scale, bias, rounding to channel pairs: m[4 hh + 2 cc + bot]
+                // is positions 16 hh + 8 bot + lane / 4, channels 8 cc + cpair + {0, 1}
+                uint32_t m[8];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                  const int co = co0 + c0 + 8 * cc + cpair;
+                  float b0 = 0.0f, b1 = 0.0f;
+                  if (bias) {
+                    if (co < g.Cout) b0 = DTypeOps<T>::to_f32(__ldg(bias + co));
+                    if (co + 1 < g.Cout) b1 = DTypeOps<T>::to_f32(__ldg(bias + co + 1));
+                  }
+#pragma unroll
+                  for (int hb = 0; hb < 4; ++hb) {  // hb = 2 hh + bot
+                    const int src = (hb >> 1) * 8 + cc * 4 + (hb & 1) * 2;
+                    float f0 = __uint_as_float(v[src]), f1 = __uint_as_float(v[src + 1]);
+                    if constexpr (kFp4) {
+                      f0 = __fmul_rn(f0, gg);
+                      f1 = __fmul_rn(f1, gg);
+                    }
+                    if (bias) {
+                      f0 = __fadd_rn(f0, b0);
+                      f1 = __fadd_rn(f1, b1);
+                    }
+                    uint32_t w;
+                    if constexpr (std::is_same<T, __half>::value) {
+                      const __half2 h = __floats2half2_rn(f0, f1);
+                      memcpy(&w, &h, 4);
+                    } else {
+                      w = cvt_bf16x2(f1, f0);
+                    }
+                    m[(hb >> 1) * 4 + cc * 2 + (hb & 1)] = w;
+                  }
+                }
+                stmatrix_x4_trans(srow, m[0], m[1], m[2], m[3]);
+                stmatrix_x4_trans(srow + 32u, m[4], m[5], m[6], m[7]);
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < kUnits; ++k) {
+                  const int j = lane / kGroups + k * (32 / kGroups);
+                  const int co = co0 + c0 + j;
+                  if (co < g.Cout && row_ok) {
+                    const uint32_t a = stage + static_cast<uint32_t>(j) * kPitch + static_cast<uint32_t>(gq * 16);
+                    int w0, w1, w2, w3;
+                    ld_shared_v4(a, w0, w1, w2, w3);
+                    T* dst = y + ubase + static_cast<int64_t>(co) * S;
+                    if (full) {
+                      __stcs(reinterpret_cast<int4*>(dst), make_int4(w0, w1, w2, w3));
+                    } else {
+                      const uint32_t ws[4] = {static_cast<uint32_t>(w0), static_cast<uint32_t>(w1),
+                                              static_cast<uint32_t>(w2), static_cast<uint32_t>(w3)};
+#pragma unroll
+                      for (int e = 0; e < kPer; ++e) {
+                        if (ow + e < g.OW) {
+                          const unsigned short b = static_cast<unsigned short>(ws[e >> 1] >> (16 * (e & 1)));
+                          memcpy(dst + e, &b, 2);
+                        }
+                      }
+                    }
+                  }
+                }
+                __syncwarp();
+              }
+              continue;
+            }
+          }
           // each step's 16 columns are loaded while the previous step's are
           // processed, so the accumulator is handed back one step earlier and
           // the loads' latency is hidden

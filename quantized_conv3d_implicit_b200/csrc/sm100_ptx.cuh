@@ -239,6 +239,35 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+// 16 TMEM lanes x 16 columns (the 16x256b shape, two 8-column repetitions):
+// thread t holds lanes t/4 and t/4 + 8 of the 16 and, in each 8-column half
+// h, columns 2 (t % 4) and 2 (t % 4) + 1:
+//   r[4h + 0], r[4h + 1]: lane t/4,     columns 8h + 2 (t % 4) + {0, 1}
+//   r[4h + 2], r[4h + 3]: lane t/4 + 8, the same columns
+// (the layout of an m16n8 accumulator fragment).
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+// tcgen05.wait::ld that also orders every later use of the 16 loaded
+// registers after the wait.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
+// Four 8x8 matrices of 16-bit elements, each stored transposed: thread i
+// gives the shared address of stored row i % 8 of matrix i / 8; register m
+// holds the thread's element pair (row t / 4, columns 2 (t % 4) + {0, 1}) of
+// matrix m, and stored row k of a matrix is its column k.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t m0, uint32_t m1, uint32_t m2, uint32_t m3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(m0), "r"(m1),
+               "r"(m2), "r"(m3)
+               : "memory");
+}
 
 // ---------------------------------------------------------------------------
 // UMMA descriptors
