@@ -132,10 +132,10 @@ def test_identity_weight_readout_is_bit_exact(cuda_ok, kernel, mode, dtype, widt
 @pytest.mark.parametrize("mode", ("noquant", "max", "max/50"))
 def test_identity_readout_half_slice_stages(cuda_ok, kernel, mode, dtype):
     # four subtiles of TH 2 x TW 64 with an A stage per half of them: the
-    # second half's rows land in their own stage, bit for bit (OH = 52 leaves
+    # second half's rows land in their own stage, bit for bit (OH = 36 leaves
     # a ragged last tile)
     quant = mode != "noquant"
-    xs = (1, 5, 4, 52, 64)
+    xs = (1, 5, 4, 36, 64)
     K = 5 * 27
     g = torch.Generator().manual_seed(13)
     x = (torch.randn(xs, generator=g) * 3).to(dtype)
