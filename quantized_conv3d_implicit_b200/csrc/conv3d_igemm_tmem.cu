@@ -21,8 +21,7 @@ static bool choose_plan(const ConvGeom& g, int dtype, TmemParams& p, size_t& sme
   TmemParams q{};
   size_t qsmem = 0;
   if (plan_tmem(g, dtype, q, qsmem, kAOpBf16Smem) &&
-      (force || q.n_mt > p.n_mt ||
-       (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa / q.a_split > p.sa / p.a_split)))) {
+      (force || q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)))) {
     p = q;
     smem = qsmem;
   }
@@ -36,7 +35,7 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0,
-                       p.aop, p.acc_bufs, p.a_split};
+                       p.aop, p.acc_bufs};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
   for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
   return ok;

@@ -80,7 +80,6 @@ struct TmemParams {
   int a_col0;             // first TMEM column of the A stages (accumulators start at column 0)
   int acc_bufs;           // accumulator buffers (2: tile t + 1 accumulates while tile t drains)
   int acc_cols;           // TMEM columns of one accumulator buffer (n_mt * n_tile)
-  int a_split;            // A stages per K slice (2: a stage per half of the subtiles; sa counts those stages)
   int dk2_c, dk2_phi;     // 128 = dk2_c * taps + dk2_phi (a transform warp's step: two slices)
   int dk16_c, dk16_phi;   // 16 = dk16_c * taps + dk16_phi (from one block to the next)
   int slot_aligned;       // c_slot * taps is a multiple of 16: no block straddles two halo slots
@@ -839,10 +838,7 @@ struct MmaBars {
 template <int NMT, int NSUB, bool kSmemA = false>
 __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t base, uint32_t tmem_base,
                                                const MmaBars& b, volatile int* abort_flag) {
-  // NMT: subtiles per A stage (a slice's subtiles come in a_split stages)
-  const int a_split = p.a_split;
-  const int n_half = NMT ? NMT : p.n_mt / a_split;
-  const int n_mt = p.n_mt;
+  const int n_mt = NMT ? NMT : p.n_mt;
   const int n_sub = NSUB ? NSUB : p.n_sub;
   const uint32_t idesc = umma_idesc_bf16_f32(128, static_cast<uint32_t>(p.sub_n));
   const uint32_t sub_cols = static_cast<uint32_t>(p.sub_n);
@@ -856,14 +852,10 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
     const uint32_t buf = p.acc_bufs == 2 ? (it & 1u) : 0u, use = p.acc_bufs == 2 ? (it >> 1) : it;
     const int abase = static_cast<int>(buf) * n_mt * n_sub;
     const uint32_t acc_base = tmem_base + buf * static_cast<uint32_t>(p.acc_cols);
-    for (int s = 0; ok && s < p.ks; ++s, bp.next(static_cast<uint32_t>(p.sb))) {
-      const uint32_t eb = bp.e;
-      const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
-      const bool first = (s == 0), last = (s == p.ks - 1);
-      for (int hh = 0; ok && hh < a_split; ++hh, ap.next(static_cast<uint32_t>(p.sa))) {
-      const uint32_t ea = ap.e;
+    for (int s = 0; ok && s < p.ks; ++s, ap.next(static_cast<uint32_t>(p.sa)), bp.next(static_cast<uint32_t>(p.sb))) {
+      const uint32_t ea = ap.e, eb = bp.e;
       ok = wait_or_abort(b.a_full + 8u * ea, ap.ph, p.err, kSiteAStageFull, abort_flag) &&
-           (hh > 0 || wait_or_abort(b.b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag));
+           wait_or_abort(b.b_full + 8u * eb, bp.ph, p.err, kSiteTmaFull, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -871,10 +863,11 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
       tc_fence_after();
       const uint32_t a_stage = kSmemA ? base + p.off_a + ea * p.a_stage_bytes
                                       : tmem_base + static_cast<uint32_t>(p.a_col0) + ea * static_cast<uint32_t>(n_mt * 32);
+      const uint64_t bdesc = umma_desc_kmajor_sw128(base + p.off_b + eb * p.b_stage_bytes);
+      const bool first = (s == 0), last = (s == p.ks - 1);
 #pragma unroll
-      for (int il = 0; il < (NMT ? NMT : 4); ++il) {
-        if (!NMT && il >= n_half) break;
-        const int i = hh * n_half + il;  // the subtile (accumulator); il: its place in the stage
+      for (int i = 0; i < (NMT ? NMT : 4); ++i) {
+        if (!NMT && i >= n_mt) break;
 #pragma unroll
         for (int ns = 0; ns < (NSUB ? NSUB : 2); ++ns) {
           if (!NSUB && ns >= n_sub) break;
@@ -890,13 +883,13 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
             const uint64_t bsub = bdesc + static_cast<uint64_t>(ns) * bsub_step;
             if constexpr (kSmemA) {
               // K advances 32 bytes (16 BF16) inside the 128-byte swizzle atom
-              const uint64_t asub = umma_desc_kmajor_sw128(a_stage + static_cast<uint32_t>(il) * 16384u);
+              const uint64_t asub = umma_desc_kmajor_sw128(a_stage + static_cast<uint32_t>(i) * 16384u);
 #pragma unroll
               for (int j = 0; j < kBlockK / 16; ++j)
                 umma_bf16_ss_elect(d_tmem, asub + static_cast<uint64_t>(2 * j), bsub + static_cast<uint64_t>(2 * j),
                                    idesc, (first && j == 0) ? 0u : 1u);
             } else {
-              const uint32_t a_sub = a_stage + static_cast<uint32_t>(il * 32);
+              const uint32_t a_sub = a_stage + static_cast<uint32_t>(i * 32);
 #pragma unroll
               for (int j = 0; j < kBlockK / 16; ++j)
                 umma_bf16_ts_elect(d_tmem, a_sub + 8u * j, bsub + static_cast<uint64_t>(2 * j), idesc,
@@ -908,8 +901,6 @@ __device__ __forceinline__ void mma_issue_loop(const TmemParams& p, uint32_t bas
       }
       if (!ok) break;
       umma_commit_elect(b.a_empty + 8u * ea);
-      }
-      if (!ok) break;
       umma_commit_elect(b.b_empty + 8u * eb);
     }
   }
@@ -1139,7 +1130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           default: mma_issue_loop_fp4<0, 0>(p, base, tb, bars, abort_flag); break;
         }
       } else {
-        switch ((p.n_mt / p.a_split) * 4 + p.n_sub) {  // straight-line issue for the common shapes
+        switch (p.n_mt * 4 + p.n_sub) {  // straight-line issue for the common shapes
           case 1 * 4 + 1: mma_issue_loop<1, 1, kSmemA>(p, base, tb, bars, abort_flag); break;
           case 1 * 4 + 2: mma_issue_loop<1, 2, kSmemA>(p, base, tb, bars, abort_flag); break;
           case 2 * 4 + 1: mma_issue_loop<2, 1, kSmemA>(p, base, tb, bars, abort_flag); break;
@@ -1494,15 +1485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t gs_base = 0;                 // global halo slot counter at the start of the tile
     uint32_t ga = 0;                      // global K-slice counter at the start of the tile
     uint32_t gslice = static_cast<uint32_t>(grp);  // global index of this group's next slice
-    // A stages: a slice takes a_split consecutive ones (one per subtile half;
-    // the planner splits only tiles of subtile pairs gathered by rows with A
-    // in shared memory, and the launcher checks it, so every other form
-    // keeps a_split = 1 at compile time)
-    constexpr bool kCanSplit = kSmemA && !kFp4 && kPairs && kDWB > 0;
-    const int a_split = kCanSplit ? p.a_split : 1, n_half = p.n_mt / a_split;
-    const uint32_t sa_u = static_cast<uint32_t>(p.sa);
-    const bool few_slices = p.ks * a_split < p.sa;  // fewer K slices per tile than slices in flight
-    RingPos as = ring_pos(static_cast<uint32_t>(grp * a_split), sa_u);  // its first A stage
+    RingPos as{static_cast<uint32_t>(grp) % static_cast<uint32_t>(p.sa), 0u};  // its A stage
     RingPos hr{0u, 0u};                   // next halo slot this warp hands back
     bool ok = true;
     for (int64_t tt = blockIdx.x; ok && tt < p.num_tiles; tt += gridDim.x) {
@@ -1524,13 +1507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int cs0 = c0 - q0 * p.c_slot;
       RingPos h0 = ring_pos(gs_base + static_cast<uint32_t>(q0), ring);
       int released = 0;  // halo slots of this tile this warp has handed back
-      for (; s < p.ks; s += 2, gslice += 2) {
-        // the slice's stages e0 .. e0 + a_split - 1 (sa is a multiple of
-        // a_split, so they share one pass of the ring and its parity)
-        const uint32_t e0 = as.e, ph0 = as.ph;
-        for (int k = 0; k < 2 * a_split; ++k) as.next(sa_u);
-        if (gslice * static_cast<uint32_t>(a_split) >= sa_u &&
-            !wait_or_abort(bar_a_empty + 8u * e0, ph0 ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
+      for (; s < p.ks; s += 2, gslice += 2, as.next(static_cast<uint32_t>(p.sa)), as.next(static_cast<uint32_t>(p.sa))) {
+        const uint32_t ea = as.e;
+        if (gslice >= static_cast<uint32_t>(p.sa) &&
+            !wait_or_abort(bar_a_empty + 8u * ea, as.ph ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
           ok = false;
           break;
         }
@@ -1560,20 +1540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         tc_fence_after();
-#pragma unroll 1
-        for (int hh = 0; hh < a_split; ++hh) {
-        const uint32_t ea = e0 + static_cast<uint32_t>(hh);
-        if (hh > 0) {
-          // the second half's stage
-          if (gslice * static_cast<uint32_t>(a_split) + static_cast<uint32_t>(hh) >= sa_u &&
-              !wait_or_abort(bar_a_empty + 8u * ea, ph0 ^ 1u, p.err, kSiteMmaDone, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-        // subtiles mt0 .. mt1 - 1 go to this stage
-        const int mt0 = hh * n_half, mt1 = mt0 + n_half;
         const uint32_t a_col = tmem_base + lane_field + static_cast<uint32_t>(p.a_col0) +
                                ea * static_cast<uint32_t>(p.n_mt * 32) + static_cast<uint32_t>(b0 * 8);
         // NVFP4 operands: this slice's A stage in shared memory (subtile i
@@ -1584,11 +1550,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // shared-memory tile
         auto put = [&](int i, int bb, const uint32_t (&w)[8]) {
           if constexpr (kSmemA) {
-            const uint32_t r = a_stage + static_cast<uint32_t>(i - mt0) * 16384u + a_row16;
+            const uint32_t r = a_stage + static_cast<uint32_t>(i) * 16384u + a_row16;
             st_shared_v4(r + (bb ? ach2 : ach0), w[0], w[1], w[2], w[3]);
             st_shared_v4(r + (bb ? ach3 : ach1), w[4], w[5], w[6], w[7]);
           } else {
-            tmem_st8(a_col + 8u * static_cast<uint32_t>(bb) + static_cast<uint32_t>((i - mt0) * 32), w);
+            tmem_st8(a_col + 8u * static_cast<uint32_t>(bb) + static_cast<uint32_t>(i * 32), w);
           }
         };
         const bool quant = p.quant != 0;
@@ -1601,7 +1567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pair_done = true;
             if (nv0 <= 0) {
               uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-              for (int i = mt0; i < mt1; ++i) {
+              for (int i = 0; i < p.n_mt; ++i) {
                 put(i, 0, z);
                 put(i, 1, z);
               }
@@ -1629,10 +1595,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                   // column further in the row pattern, taps being a multiple of 3)
                   const int p3 = phi % 3;
                   uint32_t r0[6], r1[6];
-                  const uint32_t sub0 = thr0 + static_cast<uint32_t>(mt0) * thr_step;
-                  row_bases(org0 + sub0, prow0, cross0 ? (g.taps - phi + p3) / 3 : 6, adj0, r0);
-                  row_bases(org1 + sub0, prow1, cross1 ? (g.taps - phi1 + phi1 % 3) / 3 : 6, adj1, r1);
-                  for (int i = mt0; i < mt1; ++i) {
+                  row_bases(org0 + thr0, prow0, cross0 ? (g.taps - phi + p3) / 3 : 6, adj0, r0);
+                  row_bases(org1 + thr0, prow1, cross1 ? (g.taps - phi1 + phi1 % 3) / 3 : 6, adj1, r1);
+                  for (int i = 0; i < p.n_mt; ++i) {
                     uint32_t pa[8], pb[8], wa[8], wb[8];
                     switch (p3) {
                       case 0: gather_rows<0, kDWB>(r0, pa); gather_rows<1, kDWB>(r1, pb); break;
@@ -1652,10 +1617,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
               if (!rows_done) {
-                uint32_t a0 = org0 + thr0 + static_cast<uint32_t>(mt0) * thr_step;
-                uint32_t a1 = org1 + thr0 + static_cast<uint32_t>(mt0) * thr_step;
+                uint32_t a0 = org0 + thr0, a1 = org1 + thr0;
 #pragma unroll 1
-                for (int i = mt0; i < mt1; ++i, a0 += thr_step, a1 += thr_step) {
+                for (int i = 0; i < p.n_mt; ++i, a0 += thr_step, a1 += thr_step) {
                   uint32_t wa[8], wb[8];
                   group32_taps<T, kDWB>(a0, prow0, phi, split0, adj0, nv0, a1, prow1, phi1, split1, adj1, nv1, p.qmode,
                                         p.dst_max, q, wa, wb);
@@ -1711,11 +1675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (nv <= 0) {
             // a block entirely past K: zeros (the weights there are zero-filled too)
             if constexpr (kFp4) {
-              for (int i = mt0; i < mt1; ++i)
+              for (int i = 0; i < p.n_mt; ++i)
                 fp4_put(codeb + static_cast<uint32_t>(i) * 4096u, sfb + static_cast<uint32_t>(i) * 512u, 0u, 0u, 0u);
             } else {
               uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-              for (int i = mt0; i < mt1; ++i) put(i, bb, z);
+              for (int i = 0; i < p.n_mt; ++i) put(i, bb, z);
             }
             continue;
           }
@@ -1731,7 +1695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             hn.next(ring);
             adj = static_cast<int>(halo_base + hn.e * p.slot_bytes) - static_cast<int>(org) - cb;
           }
-          int i = mt0;
+          int i = 0;
           if constexpr (kDWB > 0) {
             if (nv >= 16) {
               // rows of three taps: the rows of the next channel start at
@@ -1740,7 +1704,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint32_t rb0[6];
               row_bases(org + thr0, prow, crossb ? (g.taps - phb + p3) / 3 : 6, adj, rb0);
               if constexpr (kPairs) {
-                for (; i + 1 < mt1; i += 2) {
+                for (; i + 1 < p.n_mt; i += 2) {
                   uint32_t ra[6], rb[6], pa[8], pb[8], wa[8], wb[8];
 #pragma unroll
                   for (int r = 0; r < 6; ++r) {
@@ -1765,7 +1729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   }
                 }
               }
-              for (; i < mt1; ++i) {
+              for (; i < p.n_mt; ++i) {
                 uint32_t ra[6], pa[8], wa[8];
 #pragma unroll
                 for (int r = 0; r < 6; ++r) ra[r] = rb0[r] + static_cast<uint32_t>(i) * thr_step;
@@ -1799,7 +1763,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if constexpr (kPairs && sizeof(T) == 2) {
             // full blocks, subtiles in pairs: interleaved chains
             if (nv >= 16)
-              for (; i + 1 < mt1; i += 2) {
+              for (; i + 1 < p.n_mt; i += 2) {
                 uint32_t pa[8], pb[8], wa[8], wb[8];
                 const uint32_t ra = org + thr0 + static_cast<uint32_t>(i) * thr_step;
                 gather_taps<T>(ra, off, 16, pa);
@@ -1817,7 +1781,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
           }
-          for (; i < mt1; ++i) {
+          for (; i < p.n_mt; ++i) {
             if constexpr (kFp4) {
               uint32_t c0, c1, s8b;
               fp4_row_block<T>(org + thr0 + static_cast<uint32_t>(i) * thr_step, off, nv, q, c0, c1, s8b);
@@ -1837,9 +1801,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
         }
         __syncwarp();
-        if (hh + 1 < a_split && lane == 0) mbar_arrive(bar_a_full + 8u * ea);  // the slice's last stage: below
-        }
-        if (!ok) break;
         // this warp's next slice is two on: its blocks move 128 columns
         k0 += 2 * kBlockK;
         phi += p.dk2_phi;
@@ -1855,7 +1816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           h0.next(ring);
         }
         if (lane == 0) {
-          mbar_arrive(bar_a_full + 8u * (e0 + static_cast<uint32_t>(a_split - 1)));
+          mbar_arrive(bar_a_full + 8u * ea);
           // Later blocks of this warp start at slot q0 or above: hand the
           // slots below back (a slot is free once all transform warps have).
           // With fewer K slices per tile than A stages, sa slices span
@@ -1866,11 +1827,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           // within a ring lap.
           const int keep = (s + 2 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
           for (; ok && released < keep; ++released, hr.next(ring)) {
-            if (few_slices) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+            if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
             mbar_arrive(bar_halo_empty + 8u * hr.e);
           }
         }
-        if (few_slices) {  // sa slices can span more slots than the ring: only there can the hand-back fail
+        if (p.ks < p.sa) {  // sa slices can span more slots than the ring: only there can the hand-back fail
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
         }
@@ -1883,10 +1844,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // in an earlier phase.
       if (lane == 0)
         for (; ok && released < p.q_slots; ++released, hr.next(ring)) {
-          if (few_slices) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+          if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
           mbar_arrive(bar_halo_empty + 8u * hr.e);
         }
-      if (few_slices) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (p.ks < p.sa) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       gs_base += static_cast<uint32_t>(p.q_slots);
       ga += static_cast<uint32_t>(p.ks);
     }
@@ -1916,10 +1877,6 @@ cudaError_t launch_tmem_typed(const TmemParams& p, const CUtensorMap& tx, const 
                               size_t smem, cudaStream_t s) {
   const int dwb = row_gather_step(p.g, sizeof(T));
   const bool pairs = p.n_mt >= 2;
-  // stages per half of the subtiles exist only in the row-gather forms with
-  // A in shared memory (the transform of every other form builds whole slices)
-  if (p.a_split != 1 && (p.a_split != 2 || !pairs || dwb == 0 || kAOp != kAOpBf16Smem || p.n_mt % 2 != 0))
-    return cudaErrorInvalidValue;
   if constexpr (sizeof(T) == 2) {
     if (dwb == 2)
       return pairs ? launch_tmem_inst<T, true, 2, kAOp, kQ>(p, tx, tw, grid, smem, s)
@@ -2002,7 +1959,6 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
   p.n_tile = n_tile; p.n_ntiles = n_ntiles; p.n_sub = n_sub; p.sub_n = sub_n;
   p.fp4 = fp4 ? 1 : 0;
   p.aop = aop;
-  p.a_split = 1;
   p.dtype_code = dtype;
   p.n_atoms = (sub_n + 127) / 128;
   p.n_parts = n_ntiles * n_sub;
@@ -2051,15 +2007,10 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
   p.a_col0 = smem_a ? 0 : a_col0_of(bMT, p.acc_bufs);
   p.sf_col0 = fp4 ? a_col0_of(bMT, p.acc_bufs) : 0;
   p.sf_cols = fp4 ? stage_cols(bMT) : 0;
-  // BF16 A in shared memory with four subtiles: an A stage per half of
-  // them, so a transform group starts its next slice while the MMA still
-  // reads the second half of the previous one (the stage ring is as large
-  // in bytes as two whole-slice stages)
-  p.a_split = (smem_a && !fp4 && bMT == 4 && row_gather_step(g, esz) > 0) ? 2 : 1;
   p.a_stage_bytes = fp4      ? static_cast<uint32_t>((bMT * (4096 + 512) + 1023) / 1024 * 1024)
-                    : smem_a ? static_cast<uint32_t>(bMT / p.a_split) * 16384u
+                    : smem_a ? static_cast<uint32_t>(bMT) * 16384u
                              : 0u;
-  p.sa = std::min(4, stages_of(bMT, p.acc_bufs)) * p.a_split;
+  p.sa = std::min(4, stages_of(bMT, p.acc_bufs));
   p.n_owb = ceil_div(g.OW, p.TW);
   p.n_ohb = ceil_div(g.OH, p.TH * p.n_mt);
   p.h_ext = (p.TH * p.n_mt - 1) * g.sh + (g.KH - 1) * g.dh + 1;
@@ -2107,13 +2058,12 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
     p.slot_tx = static_cast<uint32_t>(p.c_slot) * p.chan_bytes;
     p.slot_bytes = (p.slot_tx + 127u) / 128u * 128u;
     // fewer A stages shrink the halo window the ring must cover
-    const int sa_max = std::min(4, stages_of(bMT, p.acc_bufs)) * p.a_split;
-    for (int a = sa_max; a >= 2 * p.a_split; a -= p.a_split) {
-      const int a_sl = (a + p.a_split - 1) / p.a_split;  // K slices in flight
+    const int sa_max = std::min(4, stages_of(bMT, p.acc_bufs));
+    for (int a = sa_max; a >= 2; --a) {
       int span = 1;
       for (int s0 = 0; s0 < p.ks; ++s0) {
         const int lo = ((kBlockK * s0) / g.taps) / p.c_slot;
-        const int hi = (std::min(kBlockK * (s0 + a_sl) - 1, g.K - 1) / g.taps) / p.c_slot;
+        const int hi = (std::min(kBlockK * (s0 + a) - 1, g.K - 1) / g.taps) / p.c_slot;
         span = std::max(span, hi - lo + 1);
       }
       for (int b = 8; b >= 2; --b) {

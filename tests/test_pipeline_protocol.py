@@ -52,8 +52,6 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
     ks, q_slots, ring, sa, sb, G = (plan[k] for k in ("ks", "q_slots", "ring", "sa", "sb", "groups"))
     n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
     nbuf = plan.get("acc_bufs", 1) or 1   # accumulator buffers (the tensor-memory kernel may have two)
-    a_split = plan.get("a_split", 1) or 1  # A stages per K slice (tensor-memory kernel: one per subtile half)
-    n_half = n_mt // a_split
     n_xf = 16 if kernel == "tmem" else 8   # transform warps; the tensor-memory kernel has one group
     wpg = n_xf // G
     # who hands halo slots back: the MMA thread (shared-memory kernel) or
@@ -98,27 +96,24 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
         for it, (k0, k1) in enumerate(us):
             released = 0
             for s in range(k0, k1):
-                eb = gb % sb
+                ea, eb = ga % sa, gb % sb
+                yield ("wait", bar("a_full", ea, 8 if kernel == "tmem" else wpg), ga // sa)
+                keep = slot_lo(s + 1) if s + 1 < ks else q_slots
+                while not xf_release and released < keep:
+                    yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
+                    released += 1
+                yield ("wait", bar("b_full", eb, 1), gb // sb)
                 buf, use = it % nbuf, it // nbuf   # accumulator buffer of this unit, and its earlier uses
-                for hh in range(a_split):
-                    ea = ga % sa
-                    yield ("wait", bar("a_full", ea, 8 if kernel == "tmem" else wpg), ga // sa)
-                    if hh == 0:
-                        keep = slot_lo(s + 1) if s + 1 < ks else q_slots
-                        while not xf_release and released < keep:
-                            yield ("arrive", bar("halo_empty", (gs_base + released) % ring, 1))
-                            released += 1
-                        yield ("wait", bar("b_full", eb, 1), gb // sb)
-                    for i in range(hh * n_half, (hh + 1) * n_half):
-                        for ns in range(n_sub):
-                            acc = (buf * n_mt + i) * n_sub + ns
-                            if s == k0 and use > 0:
-                                yield ("wait", bar("acc_empty", acc, 4), use - 1)
-                            if s == k1 - 1:
-                                yield ("arrive", bar("acc_full", acc, 1))
-                    yield ("arrive", bar("a_empty", ea, 1))
-                    ga += 1
+                for i in range(n_mt):
+                    for ns in range(n_sub):
+                        acc = (buf * n_mt + i) * n_sub + ns
+                        if s == k0 and use > 0:
+                            yield ("wait", bar("acc_empty", acc, 4), use - 1)
+                        if s == k1 - 1:
+                            yield ("arrive", bar("acc_full", acc, 1))
+                yield ("arrive", bar("a_empty", ea, 1))
                 yield ("arrive", bar("b_empty", eb, 1))
+                ga += 1
                 gb += 1
             gs_base += q_slots
 
@@ -187,9 +182,8 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
             s = k0u + gslice - ga
             released = 0
             while s < k1u:
-                gh = gslice * a_split   # global index of the slice's first A stage
-                ea, ua = gh % sa, gh // sa
-                if gh >= sa:
+                ea, ua = gslice % sa, gslice // sa
+                if gslice >= sa:
                     yield ("wait", bar("a_empty", ea, 1), ua - 1)
                 k0 = 64 * s + 16 * b0
                 if k0 < K:
@@ -206,13 +200,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                         assert q_lo <= q < q_lo + n_q, "a block reads a slot outside its unit"
                         g = gs_base + q - q_lo
                         yield ("wait", bar("halo_full", g % ring, 1), g // ring)
-                # the slice's subtile halves, each in its own A stage
-                for hh in range(a_split):
-                    if hh > 0:
-                        ea, ua = (gh + hh) % sa, (gh + hh) // sa
-                        if gh + hh >= sa:
-                            yield ("wait", bar("a_empty", ea, 1), ua - 1)
-                    yield ("arrive", bar("a_full", ea, 8))
+                yield ("arrive", bar("a_full", ea, 8))
                 if s + 2 < k1u:
                     keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot - q_lo, n_q)
                 else:
@@ -221,7 +209,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                     # with ks < sa, sa slices span several tiles' slots and a
                     # warp hands back slots it never read: it waits for each
                     # slot's fill first so it cannot do so a ring lap early
-                    if ks * a_split < sa:
+                    if ks < sa:
                         yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                     yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                     released += 1
@@ -232,7 +220,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                 # with ks < sa a slot handed back at the end of a tile waits
                 # for its fill first: a warp with no slice in the tile would
                 # otherwise run a ring lap ahead and arrive in an earlier phase
-                if ks * a_split < sa:
+                if ks < sa:
                     yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                 yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                 released += 1
@@ -359,11 +347,6 @@ def _check_tmem_invariants(p, taps):
         assert (p["c_slot"] * taps) % 16 == 0
     nb = p["acc_bufs"]
     assert nb in (1, 2) and p["aop"] in (0, 1) and p["sa"] >= 2
-    # A stages per half of four subtiles only with A in shared memory; the
-    # ring then holds at least two slices
-    assert p["a_split"] in (1, 2)
-    if p["a_split"] == 2:
-        assert p["aop"] == 1 and p["n_mt"] == 4 and p["sa"] >= 4
     if p["aop"] == 0:
         # acc_bufs accumulators [0, nb*n_mt*n_tile), then sa A stages of n_mt * 32 columns
         assert nb * p["n_mt"] * p["n_tile"] <= p["a_col0"] and p["a_col0"] % 32 == 0
@@ -433,15 +416,3 @@ def test_tmem_kernel_single_slice_tiles_do_not_lap_the_ring(order):
     plan, K, taps = _plan(((1, 64, 32, 64, 256), (32, 64, 1, 1, 1), 1, 0, 1, torch.bfloat16), kernel="tmem")
     assert plan["ks"] == 1 and 7 * plan["q_slots"] > 2 * plan["ring"]
     run(plan, K, taps, 7, order=order, seed=5, kernel="tmem")
-
-
-@pytest.mark.parametrize("cin", [1, 3, 8, 24])
-@pytest.mark.parametrize("order", ["rr", "rev", "random"])
-def test_tmem_kernel_half_slice_stages(cin, order):
-    """A stages per half of four subtiles (A in shared memory, row gathers):
-    one to seven K slices per tile, so with one slice the two halves of the
-    slice are the only stages in flight and the hand-back waits for fills."""
-    plan, K, taps = _plan(((1, cin, 6, 32, 128), (96, cin, 3, 3, 3), 1, 1, 1, torch.bfloat16), kernel="tmem")
-    assert plan["a_split"] == 2 and plan["n_mt"] == 4 and plan["sa"] % 2 == 0
-    _check_tmem_invariants(plan, taps)
-    run(plan, K, taps, ntiles=5, order=order, seed=cin, kernel="tmem")
