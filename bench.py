@@ -651,7 +651,7 @@ def time_formats(api, wl, base, stream, dev, hbm, bf16_peak):
     scale bytes and packed codes) on the layer's x, against the HBM roofline
     (L2 flushed before each launch); and the fused convolution with each
     format on the wan_mid layer (the tensor-memory kernel runs NVFP4 blocks
-    of 16 and 32 and MXFP4, the general kernel the larger NVFP4 blocks),
+    of 16, 32 and 64 and MXFP4, the general kernel blocks of 128 and 256),
     against the BF16 peak."""
     import torch
 
@@ -700,7 +700,8 @@ def time_formats(api, wl, base, stream, dev, hbm, bf16_peak):
     torch.cuda.empty_cache()
     cw = workloads.get("wan_mid_384_bf16")
     inp = workloads.make_inputs(cw, device=dev, with_out=True)
-    for fmt, bs, dst in (("nvfp4", 16, 0.0), ("nvfp4", 32, 0.0), ("nvfp4", 128, 0.0), ("mxfp4", 32, 0.0)):
+    for fmt, bs, dst in (("nvfp4", 16, 0.0), ("nvfp4", 32, 0.0), ("nvfp4", 64, 0.0), ("nvfp4", 128, 0.0),
+                         ("mxfp4", 32, 0.0)):
         us = timed(lambda: api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], inp["bias"], cw.stride, pad6(cw), cw.dil,
                                                         inp["act_amax"], quant_format=fmt, block_size=bs,
                                                         dst_type_max=dst, out=inp["out"], stream=stream), reps=3)

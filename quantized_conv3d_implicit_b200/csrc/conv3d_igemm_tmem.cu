@@ -44,14 +44,16 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
 cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStream_t s, const char** why,
                                bool* handled) {
   *handled = false;
-  // quantisers: NVFP4 blocks of 16 or 32, MXFP4 (larger NVFP4 blocks span
-  // several warps' columns: the general kernel)
+  // quantisers: NVFP4 blocks of 16, 32 or 64, MXFP4 (blocks of 128 and 256
+  // span the two transform groups' K slices: the general kernel)
   int qmode = kQModeNv16;
   if (L.quant) {
     if (L.qfmt == 2)
       qmode = kQModeMx;
     else if (L.qblock == 32)
       qmode = kQModeNv32;
+    else if (L.qblock == 64)
+      qmode = kQModeNv64;
     else if (L.qblock != 16)
       return cudaSuccess;
   }
@@ -59,7 +61,12 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   TmemParams p{};
   size_t smem = 0;
-  if (!choose_plan(g, L.dtype, p, smem)) return cudaSuccess;
+  if (qmode == kQModeNv64) {
+    // blocks of 64 pair two lanes per row, which only A in shared memory allows
+    if (!plan_tmem(g, L.dtype, p, smem, kAOpBf16Smem)) return cudaSuccess;
+  } else if (!choose_plan(g, L.dtype, p, smem)) {
+    return cudaSuccess;
+  }
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
   p.qmode = qmode; p.dst_max = L.dst_max;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;

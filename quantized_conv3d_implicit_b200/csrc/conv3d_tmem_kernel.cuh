@@ -139,10 +139,13 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kAOpBf16Tmem = 0, kAOpBf16Smem = 1, kAOpNvfp4 = 2;
 // The activation quantiser of the BF16 forms: NVFP4 with blocks of 16 (the
 // default), NVFP4 with blocks of 32 (an E4M3 scale per 32 columns), MXFP4
-// (a power-of-two scale per 32 columns).  A warp's two adjacent 16-column
-// blocks of a K slice (b0 even) are one 32-column group, so a group's
-// maximum never leaves the thread that owns its row.
-constexpr int kQModeNv16 = 0, kQModeNv32 = 1, kQModeMx = 2;
+// (a power-of-two scale per 32 columns), NVFP4 with blocks of 64.  A warp's
+// two adjacent 16-column blocks of a K slice (b0 even) are one 32-column
+// group, so a group's maximum never leaves the thread that owns its row.  A
+// 64-column block is a whole K slice: with A in shared memory the threads
+// are then mapped so that lanes l and l + 16 of a warp hold the two halves
+// of one row, and the block maximum is one shuffle away.
+constexpr int kQModeNv16 = 0, kQModeNv32 = 1, kQModeMx = 2, kQModeNv64 = 3;
 
 
 struct TileCoord {
@@ -689,10 +692,13 @@ template <typename T>
 __device__ __forceinline__ void quant_group32(const uint32_t (&pa)[8], const uint32_t (&pb)[8], int qmode,
                                               float dst_max, const QCtx& q, uint32_t (&wa)[8], uint32_t (&wb)[8]) {
   using H = Half2<T>;
-  const uint32_t m = H::maxabs(maxabs8<T>(pa), maxabs8<T>(pb));
+  uint32_t m = H::maxabs(maxabs8<T>(pa), maxabs8<T>(pb));
+  // blocks of 64: the row's other 32 columns are held by lane ^ 16 (every
+  // lane of the warp reaches this shuffle)
+  if (qmode == kQModeNv64) m = H::maxabs(m, __shfl_xor_sync(0xffffffffu, m, 16));
   DqTable dt;
   float inv;
-  if (qmode == kQModeNv32)
+  if (qmode != kQModeMx)
     load_entry(H::entry(m, q), dt, inv);
   else
     mx_group_scale(fmaxf(H::abs_lo(m), H::abs_hi(m)), dst_max, dt, inv);
@@ -707,9 +713,10 @@ __device__ __forceinline__ void quant_group32_f32(const float (&va)[16], const f
   float gmax = 0.0f;
 #pragma unroll
   for (int j = 0; j < 16; ++j) gmax = fmaxf(gmax, fmaxf(fabsf(va[j]), fabsf(vb[j])));
+  if (qmode == kQModeNv64) gmax = fmaxf(gmax, __shfl_xor_sync(0xffffffffu, gmax, 16));
   DqTable dt;
   float inv;
-  if (qmode == kQModeNv32)
+  if (qmode != kQModeMx)
     load_entry(entry_of_max(gmax, q), dt, inv);
   else
     mx_group_scale(gmax, dst_max, dt, inv);
@@ -1392,8 +1399,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int xw = warp - kWarpXf0;
     const int quad = warp & 3;                 // TMEM lanes 32*quad..+31
     const int grp = xw >> 3;                   // global slices of this parity
-    const int b0 = ((xw >> 2) & 1) * 2;        // first of the warp's two blocks
-    const int row = quad * 32 + lane;          // output position within a subtile
+    // blocks of 64 (A in shared memory only): the quad's two warps take 16
+    // rows each, lanes l and l + 16 the two halves of row l % 16 of them
+    const bool blk64 = kQ == 1 && kSmemA && p.qmode == kQModeNv64;
+    const int b0 = blk64 ? 2 * (lane >> 4) : ((xw >> 2) & 1) * 2;  // first of the thread's two blocks
+    const int row = blk64 ? quad * 32 + ((xw >> 2) & 1) * 16 + (lane & 15)
+                          : quad * 32 + lane;  // output position within a subtile
     const int th = row / p.TW, tw = row % p.TW;
     const uint32_t halo_base = base + p.off_halo;
     const uint32_t phase_tab = base + p.off_phase;
@@ -1565,7 +1576,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // blocks b0, b0 + 1 of a row are one group; both are gathered
             // per subtile and share the scale of their joint maximum
             pair_done = true;
-            if (nv0 <= 0) {
+            // blocks of 64 keep every lane on one path: the block maximum is
+            // exchanged by a shuffle in each subtile's quantisation
+            if (nv0 <= 0 && !blk64) {
               uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
               for (int i = 0; i < p.n_mt; ++i) {
                 put(i, 0, z);
@@ -1590,7 +1603,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               bool rows_done = false;
               if constexpr (kDWB > 0 && sizeof(T) == 2) {
-                if (nv1 >= 16) {
+                if (blk64 ? g.K - kBlockK * s >= kBlockK : nv1 >= 16) {
                   // both blocks full: row gathers (block b0 + 1 starts one
                   // column further in the row pattern, taps being a multiple of 3)
                   const int p3 = phi % 3;

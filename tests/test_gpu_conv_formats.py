@@ -98,12 +98,15 @@ def test_ex_mxfp4_needs_no_amax(cuda_ok):
 
 
 # ---------------------------------------------------------------------------
-# The tensor-memory kernel's 32-column formats (NVFP4 blocks of 32, MXFP4):
-# a warp's two 16-column blocks of a K slice form one group.  Rows of x are a
-# multiple of 16 bytes here, so the kernel's tensor maps apply.
+# The tensor-memory kernel's 32- and 64-column formats (NVFP4 blocks of 32
+# and 64, MXFP4): a thread's two 16-column blocks of a K slice form one
+# group; for blocks of 64 (A in shared memory) lanes l and l + 16 hold the
+# two halves of a row.  Rows of x are a multiple of 16 bytes here, so the
+# kernel's tensor maps apply; every shape but the 96-channel one in FP32 has
+# a plan with A in shared memory.
 # ---------------------------------------------------------------------------
 
-TMEM_FORMATS = [("nvfp4", 32, 0.0), ("mxfp4", 32, 0.0), ("mxfp4", 32, 6.0), ("mxfp4", 32, 12.0)]
+TMEM_FORMATS = [("nvfp4", 32, 0.0), ("nvfp4", 64, 0.0), ("mxfp4", 32, 0.0), ("mxfp4", 32, 6.0), ("mxfp4", 32, 12.0)]
 TMEM_FIDS = [f"{f}{b}_{d:g}" for f, b, d in TMEM_FORMATS]
 
 
