@@ -314,3 +314,19 @@ def test_bf16_plan_choice_per_workload():
         assert p["acc_bufs"] * p["n_mt"] * p["n_tile"] <= 512
         if p["aop"] == 0:
             assert p["a_col0"] + p["sa"] * p["n_mt"] * 32 <= 512
+
+
+def test_blocks_of_64_have_a_shared_memory_plan(monkeypatch):
+    """NVFP4 blocks of 64 pair two lanes per row, which the tensor-memory
+    kernel allows only with A in shared memory: the format's GPU parity
+    shapes must have that plan (Q3D_KERNEL=smem_a makes the plan hook report
+    it), or the launcher would quietly hand them to the general kernel."""
+    monkeypatch.setenv("Q3D_KERNEL", "smem_a")
+    shapes = [((1, 11, 4, 7, 16), 41), ((1, 6, 6, 13, 24), 33), ((1, 32, 3, 8, 16), 300), ((1, 3, 7, 9, 16), 8),
+              ((1, 8, 3, 8, 32), 192), ((1, 96, 3, 16, 64), 96), ((1, 11, 4, 7, 16), 128),
+              ((1, 384, 5, 60, 104), 384)]
+    for xs, cout in shapes:
+        k = (1, 1, 1) if cout == 300 else (5, 5, 5) if xs[1] == 3 else (3, 3, 3)
+        for dt in (torch.bfloat16, torch.float16):
+            p = api.plan_conv(xs, (cout, xs[1]) + k, 1, (2, 0, 1, 1, 1, 1), 1, dt, kernel="tmem")
+            assert p["applicable"] == 1 and p["aop"] == 1, (xs, cout, dt)
