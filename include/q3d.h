@@ -152,10 +152,15 @@ typedef enum {
  *       (dst_type_max 0) or the exponent of block max / dst_type_max rounded
  *       up (dst_type_max in [6, 12]), as in mxfp4_quantize; act_amax unused.
  * NVFP4 with block_size 16 runs the same kernels as
- * conv3d_implicit_gemm_pad2 (bit-identical results); the other settings run
- * the general kernel, which takes each block's maximum in a separate gather
- * pass.  Q3D_ERR_INVALID_ARG for another format, block size or dst_type_max,
- * before anything is enqueued.
+ * conv3d_implicit_gemm_pad2 (bit-identical results).  NVFP4 blocks of 32
+ * and 64 and MXFP4 run the tensor-memory kernel where its tensor maps apply
+ * (rows of x a multiple of 16 bytes; blocks of 64 also need its plan with A
+ * in shared memory), with each group's maximum taken inside the thread or
+ * thread pair that builds the row; blocks of 128 and 256, and every setting
+ * the tensor-memory kernel does not take, run the general kernel, which
+ * takes each block's maximum in a separate gather pass.  All kernels give
+ * the same result.  Q3D_ERR_INVALID_ARG for another format, block size or
+ * dst_type_max, before anything is enqueued.
  */
 Q3D_API q3d_status conv3d_implicit_gemm_ex(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
                                            const float* act_amax, const int32_t stride[3],
