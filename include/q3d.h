@@ -158,8 +158,8 @@ typedef enum {
  * in shared memory), with each group's maximum taken inside the thread or
  * thread pair that builds the row; blocks of 128 and 256, and every setting
  * the tensor-memory kernel does not take, run the general kernel, which
- * takes each block's maximum in a separate gather pass.  All kernels give
- * the same result.  Q3D_ERR_INVALID_ARG for another format, block size or
+ * takes each block's maximum in a separate gather pass.  All kernels build
+ * the same quantised operand, bit for bit.  Q3D_ERR_INVALID_ARG for another format, block size or
  * dst_type_max, before anything is enqueued.
  */
 Q3D_API q3d_status conv3d_implicit_gemm_ex(const q3d_tensor* x, const q3d_tensor* w, const q3d_tensor* bias,
