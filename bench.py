@@ -400,6 +400,9 @@ def run_ours(args, world, rank, local):
 
     formats = None if (args.no_formats or fp4) else time_formats(api, wl, base, stream, dev, hbm, peak)
 
+    # context only: the same convolutions without quantisation in cuDNN
+    cudnn = None if (args.no_cudnn or fp4) else time_cudnn(dev, peak, layers)
+
     # end-to-end through the public API with pinned host buffers
     e2e = None if (args.no_e2e or fp4) else run_e2e(args, wl, base, stream, dev, world)
 
@@ -454,6 +457,8 @@ def run_ours(args, world, rank, local):
         result["layers_clocks"] = layer_clocks
     if formats is not None:
         result["formats"] = formats
+    if cudnn is not None:
+        result["cudnn_context"] = cudnn
     if layers_fp4:
         result["layers_fp4"] = {
             "what": ("conv3d_implicit_gemm_fp4: activations and weights NVFP4, block-scaled FP4 MMA "
@@ -711,6 +716,51 @@ def time_formats(api, wl, base, stream, dev, hbm, bf16_peak):
     return out
 
 
+def time_cudnn(dev, bf16_peak, layers):
+    """Context, not a baseline of the method: torch's cuDNN convolution
+    (F.conv3d, autotuned) on the Wan and edge layers without quantisation
+    (cuDNN has no fused activation quantiser), the input padded outside the
+    timed launches (the causal temporal padding is asymmetric), L2 flushed
+    before each launch, CUDA events on the launching stream."""
+    import torch
+    import torch.nn.functional as F
+
+    from quantized_conv3d_implicit_b200 import workloads
+    torch.backends.cudnn.benchmark = True
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    cur = torch.cuda.current_stream(dev)
+    out = {"what": "torch.nn.functional.conv3d (cuDNN), no quantisation; ours: this library with quantisation on "
+                   "(and off where a quant-off workload exists)", "layers": {}}
+    for name in ("wan_mid_384_bf16", "wan_hi_192_bf16", "edge_full_96_bf16"):
+        cw = workloads.get(name)
+        inp = workloads.make_inputs(cw, device=dev)
+        xp = F.pad(inp["x"], (cw.pad_lo[2], cw.pad_hi[2], cw.pad_lo[1], cw.pad_hi[1], cw.pad_lo[0], cw.pad_hi[0]))
+        del inp["x"]
+        fn = lambda: F.conv3d(xp, inp["w"], inp["bias"], stride=cw.stride, dilation=cw.dil)  # noqa: E731
+        for _ in range(3):
+            y = fn()
+        ts = []
+        for _ in range(5):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(cur)
+            y = fn()
+            b.record(cur)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b) * 1e3)
+        del y, xp, inp
+        torch.cuda.empty_cache()
+        us = statistics.median(ts)
+        tf = cw.flops / (us * 1e-6) / 1e12
+        row = {"us": round(us, 1), "tflops": round(tf, 1), "frac": round(tf / bf16_peak, 4)}
+        if layers and name in layers:
+            row["ours_quant_on_us"] = layers[name]["us"]
+        if layers and name + "_noquant" in layers:
+            row["ours_quant_off_us"] = layers[name + "_noquant"]["us"]
+        out["layers"][name] = row
+    return out
+
+
 def time_act_amax(x, stream, dev, steps):
     """Mean device time (us) of q3d_act_amax on x (memset of the output word
     + one kernel), CUDA events on the launching stream, L2 flushed before
@@ -749,6 +799,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end timing with host copies")
     ap.add_argument("--no-fp4", action="store_true", help="skip the true-FP4 convolution timings")
     ap.add_argument("--no-formats", action="store_true", help="skip the other quantiser formats' timings")
+    ap.add_argument("--no-cudnn", action="store_true", help="skip the cuDNN context timings")
     ap.add_argument("--conv", default="bf16", choices=["bf16", "fp4"],
                     help="the step's convolution: the fake-quantised BF16 path (default) or the true-FP4 variant")
     args = ap.parse_args(argv)
