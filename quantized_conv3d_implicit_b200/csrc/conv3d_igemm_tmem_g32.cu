@@ -12,6 +12,9 @@ namespace q3d {
 
 cudaError_t launch_tmem_groups(const TmemParams& p, const CUtensorMap& tx, const CUtensorMap& tw, int grid,
                                size_t smem, cudaStream_t s) {
+  // blocks of 64 pair two lanes per row, a mapping only the shared-memory
+  // A placement has (with A in tensor memory a lane writes its own row)
+  if (p.qmode == kQModeNv64 && p.aop != kAOpBf16Smem) return cudaErrorInvalidValue;
   if (p.aop == kAOpBf16Smem) {
     switch (p.dtype_code) {
       case 0: return launch_tmem_typed<float, kAOpBf16Smem, 1>(p, tx, tw, grid, smem, s);
