@@ -38,9 +38,12 @@ class Bar:
         return (self.phase & 1) != (phase & 1)
 
 
-def roles(plan, K, taps, ntiles, kernel="fast", units=None):
+def roles(plan, K, taps, ntiles, kernel="fast", units=None, blk64=False):
     """units (tensor-memory kernel): the CTA's work as (k0, k1) K-slice
-    ranges of successive tiles; default ntiles whole tiles."""
+    ranges of successive tiles; default ntiles whole tiles.  blk64
+    (tensor-memory kernel, NVFP4 blocks of 64): every warp holds all four
+    blocks of its rows (lanes l and l + 16 two each), waits for all their
+    slots and hands back slots by block 0's position."""
     bars = {}
 
     def bar(name, i, count):
@@ -174,6 +177,8 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
         # parity; warp w handles blocks b0, b0 + 1 of each, waits for the halo
         # slots those read and hands back the slots below its next pair
         grp, b0 = w >> 3, ((w >> 2) & 1) * 2
+        b0s = (0, 2) if blk64 else (b0,)   # the blocks the warp's lanes start at
+        b_rel = 0 if blk64 else b0         # lane 0's block: the hand-back position
         gs_base = ga = 0
         gslice = grp
         hr = 0  # next global slot to hand back
@@ -185,8 +190,10 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                 ea, ua = gslice % sa, gslice // sa
                 if gslice >= sa:
                     yield ("wait", bar("a_empty", ea, 1), ua - 1)
-                k0 = 64 * s + 16 * b0
-                if k0 < K:
+                for bw in b0s:
+                    k0 = 64 * s + 16 * bw
+                    if k0 >= K:
+                        continue
                     c0, phi = divmod(k0, taps)
                     q0, cs0 = divmod(c0, c_slot)
                     c1, phi1 = divmod(k0 + 16, taps)
@@ -202,7 +209,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
                         yield ("wait", bar("halo_full", g % ring, 1), g // ring)
                 yield ("arrive", bar("a_full", ea, 8))
                 if s + 2 < k1u:
-                    keep = min(((64 * (s + 2) + 16 * b0) // taps) // c_slot - q_lo, n_q)
+                    keep = min(((64 * (s + 2) + 16 * b_rel) // taps) // c_slot - q_lo, n_q)
                 else:
                     keep = n_q
                 while released < keep:
@@ -236,8 +243,8 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None):
     return r
 
 
-def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast", units=None):
-    rs = roles(plan, K, taps, ntiles, kernel, units)
+def run(plan, K, taps, ntiles, order="rr", seed=0, kernel="fast", units=None, blk64=False):
+    rs = roles(plan, K, taps, ntiles, kernel, units, blk64)
     names = list(rs)
     cur = {k: None for k in names}
     done = set()
@@ -416,3 +423,18 @@ def test_tmem_kernel_single_slice_tiles_do_not_lap_the_ring(order):
     plan, K, taps = _plan(((1, 64, 32, 64, 256), (32, 64, 1, 1, 1), 1, 0, 1, torch.bfloat16), kernel="tmem")
     assert plan["ks"] == 1 and 7 * plan["q_slots"] > 2 * plan["ring"]
     run(plan, K, taps, 7, order=order, seed=5, kernel="tmem")
+
+
+@pytest.mark.parametrize("shape", [((1, 96, 3, 16, 64), 96), ((1, 384, 5, 60, 104), 384), ((1, 11, 4, 7, 16), 41),
+                                   ((1, 3, 7, 9, 16), 8), ((1, 96, 17, 480, 832), 96)])
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_tmem_kernel_blocks_of_64_lane_pairs(shape, order, monkeypatch):
+    """NVFP4 blocks of 64 (A in shared memory, the plan the launcher forces):
+    each warp waits for the slots of all four blocks of its rows and hands
+    back by block 0's position; no interleaving deadlocks or aliases."""
+    monkeypatch.setenv("Q3D_KERNEL", "smem_a")
+    xs, cout = shape
+    k = (5, 5, 5) if xs[1] == 3 else (3, 3, 3)
+    plan, K, taps = _plan((xs, (cout, xs[1]) + k, 1, (2, 0, 1, 1, 1, 1), 1, torch.bfloat16), kernel="tmem")
+    assert plan["applicable"] == 1 and plan["aop"] == 1
+    run(plan, K, taps, ntiles=3, order=order, seed=len(xs) + cout, kernel="tmem", blk64=True)
