@@ -56,7 +56,10 @@ Q3D_API q3d_status q3d_plan_conv(const int64_t x_shape[5], const int64_t w_shape
  * slices of one parity) is always 2, TMEM columns 512, vectorised reads 0,
  * and more entries follow the halo box extents: the first TMEM column of
  * the A stages, the A operand's place (0 tensor memory, 1 shared memory: the
- * launcher's choice) and the number of accumulator buffers.  applicable = 0 where that kernel does not apply (x rows
+ * launcher's choice), the number of accumulator buffers and whether the
+ * transform warps wait for a halo slot's fill before handing it back (1 where
+ * the ring does not by itself keep every hand-back in its phase).
+ * applicable = 0 where that kernel does not apply (x rows
  * not a multiple of 16 bytes, more than 343 taps, or no plan that fits).
  */
 Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],

@@ -415,8 +415,9 @@ PLAN_FIELDS = ("applicable", "TH", "TW", "n_mt", "groups", "n_tile", "n_ntiles",
 def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfloat16, kernel="fast") -> dict:
     """Test hook (host only): the tiling/pipeline plan of the shared-memory
     specialised kernel (kernel="fast"), of the tensor-memory kernel
-    (kernel="tmem", three more fields: a_col0, aop = where A lives (0 tensor
-    memory, 1 shared memory), acc_bufs) or of its NVFP4-operand variant
+    (kernel="tmem", four more fields: a_col0, aop = where A lives (0 tensor
+    memory, 1 shared memory), acc_bufs, hb_wait = halo hand-backs wait for
+    the slot's fill) or of its NVFP4-operand variant
     (kernel="fp4", four more: sf_col0, sf_cols, a_stage_bytes, b_stage_bytes)."""
     lib = load_library()
     lo, hi = _pads(padding)
@@ -427,7 +428,7 @@ def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfl
     st = fn(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)), _DTYPES[dtype],
             out, 32)
     _check(lib, st)
-    extra = {"tmem": ("a_col0", "aop", "acc_bufs"), "fp4": ("sf_col0", "sf_cols", "a_stage_bytes", "b_stage_bytes")}
+    extra = {"tmem": ("a_col0", "aop", "acc_bufs", "hb_wait"), "fp4": ("sf_col0", "sf_cols", "a_stage_bytes", "b_stage_bytes")}
     fields = PLAN_FIELDS + extra.get(kernel, ())
     return dict(zip(fields, list(out)[:len(fields)]))
 

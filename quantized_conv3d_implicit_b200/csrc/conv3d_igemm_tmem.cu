@@ -14,18 +14,28 @@ namespace q3d {
 // the 384- and 1024-channel layers, which gain nothing, were 8 % slower with
 // A in shared memory).  Q3D_KERNEL=smem_a takes the shared-memory form
 // wherever it applies (the tests run every shape through it too).
-static bool choose_plan(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem) {
-  if (!plan_tmem(g, dtype, p, smem)) return false;
+//
+// The shared-memory form's halo ring is sized for the plans this rule picks
+// (checked against a model of the barrier protocol on the CPU); where the
+// form is taken otherwise (forced, or required by blocks of 64) its
+// transform warps wait for each slot's fill before handing it back, which
+// keeps every hand-back in its own phase whatever the ring.
+static bool choose_plan(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, bool need_smem_a = false) {
+  const bool tmem_ok = plan_tmem(g, dtype, p, smem);
   const char* kc = getenv("Q3D_KERNEL");
-  const bool force = kc && !strcmp(kc, "smem_a");
+  const bool force = need_smem_a || (kc && !strcmp(kc, "smem_a"));
   TmemParams q{};
   size_t qsmem = 0;
-  if (plan_tmem(g, dtype, q, qsmem, kAOpBf16Smem) &&
-      (force || q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)))) {
+  if (!plan_tmem(g, dtype, q, qsmem, kAOpBf16Smem)) return tmem_ok && !need_smem_a;
+  const bool better =
+      tmem_ok && (q.n_mt > p.n_mt || (q.n_mt == p.n_mt && (q.acc_bufs > p.acc_bufs || q.sa > p.sa)));
+  if (better || force) {
+    if (!better) q.hb_wait = 1;
     p = q;
     smem = qsmem;
+    return true;
   }
-  return true;
+  return tmem_ok;
 }
 
 bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
@@ -35,7 +45,7 @@ bool plan_conv3d_tmem(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.a_col0,
-                       p.aop, p.acc_bufs};
+                       p.aop, p.acc_bufs, p.hb_wait};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
   for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
   return ok;
@@ -61,12 +71,8 @@ cudaError_t launch_conv3d_tmem(const ConvGeom& g, const ConvLaunch& L, cudaStrea
   if (reinterpret_cast<uintptr_t>(L.x) % 16 != 0) return cudaSuccess;
   TmemParams p{};
   size_t smem = 0;
-  if (qmode == kQModeNv64) {
-    // blocks of 64 pair two lanes per row, which only A in shared memory allows
-    if (!plan_tmem(g, L.dtype, p, smem, kAOpBf16Smem)) return cudaSuccess;
-  } else if (!choose_plan(g, L.dtype, p, smem)) {
-    return cudaSuccess;
-  }
+  // blocks of 64 pair two lanes per row, which only A in shared memory allows
+  if (!choose_plan(g, L.dtype, p, smem, qmode == kQModeNv64)) return cudaSuccess;
   p.bias = L.bias; p.y = L.y; p.act_amax = L.act_amax; p.err = L.err; p.quant = L.quant;
   p.qmode = qmode; p.dst_max = L.dst_max;
   p.y_vec = (reinterpret_cast<uintptr_t>(L.y) % 16 == 0 && g.OW % (16 / esz) == 0) ? 1 : 0;

@@ -106,6 +106,9 @@ struct TmemParams {
   // E2M1 rule floor(log2 amax) - 2)
   int qmode;
   float dst_max;
+  // transform warps wait for each halo slot's fill before handing it back
+  // (plans whose warps could otherwise hand back a slot a ring lap early)
+  int hb_wait;
 };
 
 // The BF16 kernel with A in shared memory (instantiated in its own
@@ -1832,19 +1835,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar_a_full + 8u * ea);
           // Later blocks of this warp start at slot q0 or above: hand the
           // slots below back (a slot is free once all transform warps have).
-          // With fewer K slices per tile than A stages, sa slices span
-          // several tiles' slots, more than the ring holds, and a warp
-          // hands back slots it never read: there each waits for the
-          // slot's fill first, or the hand-back could land in the previous
-          // use's phase.  Otherwise the stage coupling keeps every warp
-          // within a ring lap.
+          // A warp also hands back slots it never read (the other group's
+          // slices).  Where its lead over the slowest warp can reach a ring
+          // lap (fewer K slices per tile than A stages: sa slices span
+          // several tiles' slots; or a ring sized for another plan's
+          // coupling) each hand-back waits for the slot's fill first, or it
+          // could land in the previous use's phase (p.hb_wait, set by the
+          // planner).  Otherwise the stage coupling keeps every warp within
+          // a ring lap.
           const int keep = (s + 2 < p.ks) ? min(q0, p.q_slots) : p.q_slots;
           for (; ok && released < keep; ++released, hr.next(ring)) {
-            if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+            if (p.hb_wait) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
             mbar_arrive(bar_halo_empty + 8u * hr.e);
           }
         }
-        if (p.ks < p.sa) {  // sa slices can span more slots than the ring: only there can the hand-back fail
+        if (p.hb_wait) {  // only a hand-back that waits for a fill can fail
           ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
           if (!ok) break;
         }
@@ -1857,10 +1862,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // in an earlier phase.
       if (lane == 0)
         for (; ok && released < p.q_slots; ++released, hr.next(ring)) {
-          if (p.ks < p.sa) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
+          if (p.hb_wait) ok = wait_or_abort(bar_halo_full + 8u * hr.e, hr.ph, p.err, kSiteHaloFull, abort_flag);
           mbar_arrive(bar_halo_empty + 8u * hr.e);
         }
-      if (p.ks < p.sa) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (p.hb_wait) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       gs_base += static_cast<uint32_t>(p.q_slots);
       ga += static_cast<uint32_t>(p.ks);
     }
@@ -2093,6 +2098,7 @@ bool plan_tmem(const ConvGeom& g, int dtype, TmemParams& p, size_t& smem, int ao
             total += extra * (static_cast<int>(p.slot_bytes) + 16);
           }
           p.sa = a; p.sb = b; p.ring = r;
+          p.hb_wait = p.ks < p.sa ? 1 : 0;
           p.off_dq = 0;
           p.off_b = kDqTableBytes;  // a multiple of 1024, as the swizzled weight stages need
           p.off_a = p.off_b + b * p.b_stage_bytes;  // A stages in shared memory (1024-aligned)

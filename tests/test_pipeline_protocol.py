@@ -55,6 +55,8 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None, blk64=False):
     ks, q_slots, ring, sa, sb, G = (plan[k] for k in ("ks", "q_slots", "ring", "sa", "sb", "groups"))
     n_mt, n_sub, c_slot = plan["n_mt"], plan["n_sub"], plan["c_slot"]
     nbuf = plan.get("acc_bufs", 1) or 1   # accumulator buffers (the tensor-memory kernel may have two)
+    # tensor-memory kernel: hand-backs wait for each slot's fill first
+    hb_wait = bool(plan.get("hb_wait", 0)) or plan["ks"] < plan["sa"]
     n_xf = 16 if kernel == "tmem" else 8   # transform warps; the tensor-memory kernel has one group
     wpg = n_xf // G
     # who hands halo slots back: the MMA thread (shared-memory kernel) or
@@ -216,7 +218,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None, blk64=False):
                     # with ks < sa, sa slices span several tiles' slots and a
                     # warp hands back slots it never read: it waits for each
                     # slot's fill first so it cannot do so a ring lap early
-                    if ks < sa:
+                    if hb_wait:
                         yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                     yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                     released += 1
@@ -227,7 +229,7 @@ def roles(plan, K, taps, ntiles, kernel="fast", units=None, blk64=False):
                 # with ks < sa a slot handed back at the end of a tile waits
                 # for its fill first: a warp with no slice in the tile would
                 # otherwise run a ring lap ahead and arrive in an earlier phase
-                if ks < sa:
+                if hb_wait:
                     yield ("wait", bar("halo_full", hr % ring, 1), hr // ring)
                 yield ("arrive", bar("halo_empty", hr % ring, 16), hr // ring)
                 released += 1
@@ -438,3 +440,17 @@ def test_tmem_kernel_blocks_of_64_lane_pairs(shape, order, monkeypatch):
     plan, K, taps = _plan((xs, (cout, xs[1]) + k, 1, (2, 0, 1, 1, 1, 1), 1, torch.bfloat16), kernel="tmem")
     assert plan["applicable"] == 1 and plan["aop"] == 1
     run(plan, K, taps, ntiles=3, order=order, seed=len(xs) + cout, kernel="tmem", blk64=True)
+
+
+@pytest.mark.parametrize("name", sorted(workloads.WORKLOADS))
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_tmem_kernel_forced_shared_memory_plans(name, order, monkeypatch):
+    """A in shared memory where the launcher would not choose it (forced, as
+    the GPU tests and blocks of 64 do): the plan's hand-backs wait for the
+    fills, and no interleaving deadlocks or aliases, for the default mapping
+    and for the blocks-of-64 lane pairs."""
+    monkeypatch.setenv("Q3D_KERNEL", "smem_a")
+    plan, K, taps = _plan(workloads.WORKLOADS[name], kernel="tmem")
+    assert plan["applicable"] == 1 and plan["aop"] == 1
+    for blk64 in (False, True):
+        run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)), kernel="tmem", blk64=blk64)
