@@ -71,7 +71,8 @@ Q3D_API q3d_status q3d_plan_conv_tmem(const int64_t x_shape[5], const int64_t w_
  * use (host arithmetic only).  The fields of q3d_plan_conv_tmem up to the
  * halo box extents, then: the first TMEM column of the scale factors, the
  * TMEM columns per A stage, the bytes of one A stage in shared memory and of
- * one weight stage.
+ * one weight stage, the number of accumulator buffers and the hand-back
+ * fill-wait flag (as for q3d_plan_conv_tmem).
  */
 Q3D_API q3d_status q3d_plan_conv_fp4(const int64_t x_shape[5], const int64_t w_shape[5], const int32_t stride[3],
                                      const int32_t pad_lo[3], const int32_t pad_hi[3], const int32_t dil[3],

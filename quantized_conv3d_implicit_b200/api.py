@@ -418,7 +418,8 @@ def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfl
     (kernel="tmem", four more fields: a_col0, aop = where A lives (0 tensor
     memory, 1 shared memory), acc_bufs, hb_wait = halo hand-backs wait for
     the slot's fill) or of its NVFP4-operand variant
-    (kernel="fp4", four more: sf_col0, sf_cols, a_stage_bytes, b_stage_bytes)."""
+    (kernel="fp4", six more: sf_col0, sf_cols, a_stage_bytes, b_stage_bytes,
+    acc_bufs, hb_wait)."""
     lib = load_library()
     lo, hi = _pads(padding)
     a3 = lambda t: (ctypes.c_int32 * 3)(*t)  # noqa: E731
@@ -428,7 +429,7 @@ def plan_conv(x_shape, w_shape, stride=1, padding=0, dilation=1, dtype=torch.bfl
     st = fn(a5(x_shape), a5(w_shape), a3(_triple(stride)), a3(lo), a3(hi), a3(_triple(dilation)), _DTYPES[dtype],
             out, 32)
     _check(lib, st)
-    extra = {"tmem": ("a_col0", "aop", "acc_bufs", "hb_wait"), "fp4": ("sf_col0", "sf_cols", "a_stage_bytes", "b_stage_bytes")}
+    extra = {"tmem": ("a_col0", "aop", "acc_bufs", "hb_wait"), "fp4": ("sf_col0", "sf_cols", "a_stage_bytes", "b_stage_bytes", "acc_bufs", "hb_wait")}
     fields = PLAN_FIELDS + extra.get(kernel, ())
     return dict(zip(fields, list(out)[:len(fields)]))
 

@@ -107,7 +107,8 @@ bool plan_conv3d_fp4(const ConvGeom& g, int dtype, int32_t* out, int n_out) {
   const int64_t v[] = {ok ? 1 : 0, p.TH, p.TW, p.n_mt, 2, p.n_tile, p.n_ntiles, p.n_sub, p.sub_n, p.ks,
                        p.c_slot, p.q_slots, p.ring, p.sa, p.sb, static_cast<int64_t>(kTmemCols),
                        static_cast<int64_t>(smem), p.n_ohb, p.n_owb, 0, p.w_box, p.h_ext, p.kd_ext, p.sf_col0,
-                       p.sf_cols, static_cast<int64_t>(p.a_stage_bytes), static_cast<int64_t>(p.b_stage_bytes)};
+                       p.sf_cols, static_cast<int64_t>(p.a_stage_bytes), static_cast<int64_t>(p.b_stage_bytes),
+                       p.acc_bufs, p.hb_wait};
   const int nv = static_cast<int>(sizeof(v) / sizeof(v[0]));
   for (int i = 0; i < n_out; ++i) out[i] = i < nv ? static_cast<int32_t>(v[i]) : 0;
   return ok;

@@ -454,3 +454,42 @@ def test_tmem_kernel_forced_shared_memory_plans(name, order, monkeypatch):
     assert plan["applicable"] == 1 and plan["aop"] == 1
     for blk64 in (False, True):
         run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)), kernel="tmem", blk64=blk64)
+
+
+def _plan_fp4(xs, ws, s, pad6, d, dt):
+    p = api.plan_conv(xs, ws, s, pad6, d, dt, kernel="fp4")
+    return p, ws[1] * ws[2] * ws[3] * ws[4], ws[2] * ws[3] * ws[4]
+
+
+@pytest.mark.parametrize("name", sorted(workloads.WORKLOADS))
+@pytest.mark.parametrize("order", ["rr", "rev", "random"])
+def test_fp4_variant_plans_are_deadlock_and_alias_free(name, order):
+    """The NVFP4-operand form keeps the roles and barriers (its MMA warp
+    also copies scale factors, which the commits already order): its plans
+    replayed like the BF16 ones."""
+    wl = workloads.WORKLOADS[name]
+    ws = (wl.cout, wl.x_shape[1]) + tuple(wl.kernel)
+    pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+    plan, K, taps = _plan_fp4(wl.x_shape, ws, wl.stride, pad6, wl.dil, wl.dtype)
+    assert plan["applicable"] == 1
+    run(plan, K, taps, ntiles=3, order=order, seed=sum(map(ord, name)), kernel="tmem")
+
+
+def test_fp4_variant_random_shapes():
+    rng = random.Random(3)
+    checked = 0
+    for _ in range(80):
+        k = rng.choice([(3, 3, 3), (5, 5, 5), (1, 1, 1), (1, 3, 3), (3, 1, 1), (2, 2, 2)])
+        cin = rng.choice([1, 3, 8, 16, 37, 64, 96, 192])
+        cout = rng.choice([8, 16, 40, 96, 192, 256, 384, 512, 1024])
+        xs = (rng.choice([1, 2]), cin, rng.randint(k[0], 9), rng.randint(k[1], 40), 8 * rng.randint(1, 30))
+        dt = rng.choice([torch.bfloat16, torch.float16, torch.float32])
+        try:
+            plan, K, taps = _plan_fp4(xs, (cout, cin) + k, 1, (1, 1, 1, 1, 1, 1), 1, dt)
+        except api.Q3DError:
+            continue
+        if not plan["applicable"]:
+            continue
+        run(plan, K, taps, ntiles=2, order="random", seed=checked, kernel="tmem")
+        checked += 1
+    assert checked >= 40
