@@ -204,3 +204,30 @@ def test_conv_tensor_memory_kernel_formats(cuda_ok, tmem_form, case, fmt, dtype)
                         quant_act=True, act_amax=float(inp["act_amax"].item()), quant_format=qf, block_size=bs,
                         dst_max=dst)
     assert_conv_close(to_np_f32(y), ref, f"case {case} {qf}{bs} {dtype}", dtype)
+
+
+FULL_FORMAT_LAYERS = ["wan_mid_384_bf16", "edge_full_96_bf16", "down_s122_128to256_fp16"]
+
+
+@pytest.mark.parametrize("fmt", TMEM_FORMATS[:3], ids=TMEM_FIDS[:3])
+@pytest.mark.parametrize("name", FULL_FORMAT_LAYERS)
+def test_full_size_layers_other_formats_sampled(cuda_ok, name, fmt):
+    """The full-size layers (as the bench times them) with NVFP4 blocks of 32
+    and 64 and MXFP4: seeded output rows, every channel, against the oracle
+    (the rows at the padding faces and the first and last rows included)."""
+    import test_gpu_conv as tg
+    qf, bs, dst = fmt
+    wl = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(wl, device="cuda")
+    pad6 = (wl.pad_lo[0], wl.pad_hi[0], wl.pad_lo[1], wl.pad_hi[1], wl.pad_lo[2], wl.pad_hi[2])
+    y = api.conv3d_implicit_gemm_ex(inp["x"], inp["w"], inp["bias"], wl.stride, pad6, wl.dil,
+                                    act_amax=inp["act_amax"], quant_format=qf, block_size=bs, dst_type_max=dst)
+    assert api.check_device_error() == 0
+    ms = tg._sample_rows(wl, np.random.default_rng(17), 256)
+    ref = oracle.conv3d(to_np_f32(inp["x"]), to_np_f32(inp["w"]),
+                        None if inp["bias"] is None else to_np_f32(inp["bias"]), wl.stride, wl.pad_lo, wl.pad_hi,
+                        wl.dil, quant_act=True, act_amax=float(inp["act_amax"].item()), m_list=ms,
+                        quant_format=qf, block_size=bs, dst_max=dst)
+    Co = y.shape[1]
+    got = to_np_f32(y.permute(0, 2, 3, 4, 1).reshape(-1, Co)[torch.from_numpy(ms).cuda()])
+    assert_conv_close(got, ref, f"{name} {qf}{bs}", wl.dtype)
