@@ -493,3 +493,30 @@ def test_fp4_variant_random_shapes():
         run(plan, K, taps, ntiles=2, order="random", seed=checked, kernel="tmem")
         checked += 1
     assert checked >= 40
+
+
+def test_tmem_kernel_forced_shared_memory_random_shapes(monkeypatch):
+    """Random shapes with A in shared memory forced (the GPU tests' smem_a
+    switch, blocks of 64): deadlock- and alias-free for both lane mappings."""
+    monkeypatch.setenv("Q3D_KERNEL", "smem_a")
+    rng = random.Random(19)
+    checked = 0
+    for _ in range(80):
+        k = rng.choice([(3, 3, 3), (5, 5, 5), (1, 1, 1), (1, 3, 3), (3, 1, 1), (2, 2, 2)])
+        cin = rng.choice([1, 3, 8, 16, 37, 64, 96, 192, 256])
+        cout = rng.choice([1, 8, 16, 40, 96, 100, 192, 256, 300, 384, 448, 512, 1024])
+        xs = (rng.choice([1, 2]), cin, rng.randint(k[0], 9), rng.randint(k[1], 40), 8 * rng.randint(1, 30))
+        s = (1, rng.choice([1, 1, 2]), rng.choice([1, 1, 2]))
+        d = (1, rng.choice([1, 2]), rng.choice([1, 2]))
+        pad6 = tuple(rng.randint(0, 2) for _ in range(6))
+        dt = rng.choice([torch.bfloat16, torch.float16, torch.float32])
+        try:
+            plan, K, taps = _plan((xs, (cout, cin) + k, s, pad6, d, dt), kernel="tmem")
+        except api.Q3DError:
+            continue
+        if not plan["applicable"] or plan["aop"] != 1:
+            continue
+        for blk64 in (False, True):
+            run(plan, K, taps, ntiles=2, order="random", seed=checked, kernel="tmem", blk64=blk64)
+        checked += 1
+    assert checked >= 30
