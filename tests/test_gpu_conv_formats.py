@@ -231,3 +231,19 @@ def test_full_size_layers_other_formats_sampled(cuda_ok, name, fmt):
     Co = y.shape[1]
     got = to_np_f32(y.permute(0, 2, 3, 4, 1).reshape(-1, Co)[torch.from_numpy(ms).cuda()])
     assert_conv_close(got, ref, f"{name} {qf}{bs}", wl.dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("bs", [32, 64])
+@pytest.mark.parametrize("mode", ["zero", "max/50", "2688", "1e-6"])
+def test_group_readout_amax_edge_cases(cuda_ok, tmem_form, mode, bs, dtype):
+    """NVFP4 blocks of 32 and 64 through the group path with the global
+    amax at its edges: 0 and 1e-6 (every block takes the 1e-5 fallback),
+    max/50 (block maxima above amax: the ratio clamps at 448 and E2M1
+    saturates) and 2688 (g = 1): bit-exact against the oracle."""
+    xs, k = (1, 11, 4, 7, 16), (3, 3, 3)
+    g = torch.Generator().manual_seed(43)
+    x = (torch.randn(xs, generator=g) * 3).to(dtype)
+    m = float(x.float().abs().max())
+    amax = torch.tensor([{"zero": 0.0, "max/50": m / 50.0, "2688": 2688.0, "1e-6": 1e-6}[mode]], dtype=torch.float32)
+    _readout(x, amax, k, (2, 0, 1, 1, 1, 1), (2, 1, 1), (0, 1, 1), "nvfp4", bs, 0.0)
